@@ -1,0 +1,453 @@
+"""Pins of the float64 oracle to facts fixed outside the oracle itself.
+
+Each test ties one oracle function to something it cannot satisfy by
+construction: hand-worked examples (tests/golden), closed forms, algebraic
+invariants stated on the pages, or a brute-force search written differently
+from the oracle's arithmetic.  A plausible slip in the oracle (a dropped factor,
+a transposed operand, a wrong sign, a swapped label, a wrong tie rule) fails at
+least one of them.
+"""
+import math
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+
+from oracle import wush_oracle as O
+from workloads import make_inputs, workload, bf16_bits_from_f64
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+# ---------------------------------------------------------------- Hadamard
+
+
+def test_hadamard_textbook_order_4():
+    # Sylvester construction of order 4, normalised by 1/2 (textbook value).
+    H4 = 0.5 * np.array([[1, 1, 1, 1], [1, -1, 1, -1], [1, 1, -1, -1], [1, -1, -1, 1]], float)
+    assert np.array_equal(O.sylvester_hadamard(4), H4)
+
+
+@pytest.mark.parametrize("G", [1, 2, 8, 16, 32, 64])
+def test_hadamard_orthonormal_pm_entries(G):
+    H = O.sylvester_hadamard(G)
+    assert np.allclose(H @ H.T, np.eye(G), atol=1e-15)
+    assert np.allclose(np.abs(H), G ** -0.5, atol=0)
+    assert np.all(H[0] > 0)
+
+
+def test_hadamard_rejects_non_power_of_two():
+    with pytest.raises(ValueError):
+        O.sylvester_hadamard(24)
+
+
+# ---------------------------------------------------------------- construction invariants
+
+
+def _tiny_build(lam=0.0, G=32):
+    wl = workload("tiny_mxfp4")
+    inp = make_inputs(wl)
+    return inp, O.build_transforms(inp.w, inp.xcal_bits, G, lam=lam)
+
+
+def test_inverse_transpose_identity():
+    """T_xvsh^T T_wush = I to 1e-9 (unbiasedness constraint T_W = T_X^-T)."""
+    _, b = _tiny_build(lam=0.01)
+    for Tw, Tx in zip(b["T_wush"], b["T_xvsh"]):
+        assert np.max(np.abs(Tx.T @ Tw - np.eye(Tw.shape[0]))) < 1e-9
+
+
+def test_transformed_second_moments_are_HSH():
+    """T_wush Sx T_wush^T = T_xvsh Sw T_xvsh^T = H S H^T, diagonal constant tr(S)/G.
+
+    This also fixes which side gets which transform: with the labels swapped the
+    first equality fails."""
+    _, b = _tiny_build(lam=0.0)
+    G = 32
+    H = O.sylvester_hadamard(G)
+    for i in range(b["T_wush"].shape[0]):
+        Tw, Tx, s = b["T_wush"][i], b["T_xvsh"][i], b["s"][i]
+        A = Tw @ b["Sx"][i] @ Tw.T
+        B = Tx @ b["Sw"][i] @ Tx.T
+        HSH = H @ np.diag(s) @ H.T
+        scale = np.max(np.abs(HSH))
+        assert np.max(np.abs(A - HSH)) < 1e-9 * scale
+        assert np.max(np.abs(B - HSH)) < 1e-9 * scale
+        assert np.allclose(np.diag(A), s.sum() / G, rtol=1e-9)
+        swapped = Tx @ b["Sx"][i] @ Tx.T
+        assert np.max(np.abs(swapped - HSH)) > 1e-3 * scale
+
+
+def test_inverse_column_norms_equal_mean_singular_value():
+    """With T = T_wush W'^-T = H S^-1/2 U^T every column of T^-1 has squared norm tr(S)/G."""
+    _, b = _tiny_build(lam=0.01)
+    G = 32
+    for i in range(b["T_wush"].shape[0]):
+        T = b["T_wush"][i] @ np.linalg.inv(b["Wp"][i].T)
+        Ti = np.linalg.inv(T)
+        norms = np.sum(Ti ** 2, axis=0)
+        assert np.allclose(norms, b["s"][i].sum() / G, rtol=1e-9)
+
+
+def test_singular_values_descending_positive_and_sign_convention():
+    _, b = _tiny_build(lam=0.01)
+    s = b["s"]
+    assert np.all(s > 0)
+    assert np.all(np.diff(s, axis=1) <= 0)
+    for U in b["U"]:
+        j = np.argmax(np.abs(U), axis=0)
+        assert np.all(U[j, np.arange(U.shape[1])] > 0)
+
+
+def test_closed_form_identity_weight_diagonal_activation():
+    """Sigma_w = I, Sigma_x = diag(sigma^2), sigma distinct and descending:
+    W' = I, X' = diag(sigma), U = V = I, S = diag(sigma), so
+    T_wush = H diag(sigma)^-1/2 and T_xvsh = H diag(sigma)^1/2 exactly."""
+    G = 16
+    sig = np.linspace(3.0, 0.25, G)
+    Sw = np.eye(G)[None]
+    Sx = np.diag(sig ** 2)[None]
+    b = O.transforms_from_moments(Sw, Sx)
+    H = O.sylvester_hadamard(G)
+    assert np.allclose(b["T_wush"][0], H @ np.diag(sig ** -0.5), atol=1e-12)
+    assert np.allclose(b["T_xvsh"][0], H @ np.diag(sig ** 0.5), atol=1e-12)
+    assert np.allclose(b["s"][0], sig, atol=1e-12)
+
+
+def test_closed_form_unsorted_diagonal_uses_sorting_permutation():
+    """Unsorted sigma: U = V = P (the permutation sorting sigma descending), so
+    T_wush = H P^T diag(sigma)^-1/2 where (P^T)[k, j] = 1 iff j is the k-th largest."""
+    G = 8
+    sig = np.array([0.5, 2.0, 1.0, 3.0, 0.25, 1.5, 0.75, 4.0])
+    b = O.transforms_from_moments(np.eye(G)[None], np.diag(sig ** 2)[None])
+    order = np.argsort(-sig)
+    Pt = np.zeros((G, G))
+    Pt[np.arange(G), order] = 1.0
+    H = O.sylvester_hadamard(G)
+    assert np.allclose(b["T_wush"][0], H @ Pt @ np.diag(sig ** -0.5), atol=1e-12)
+    assert np.allclose(b["T_xvsh"][0], H @ Pt @ np.diag(sig ** 0.5), atol=1e-12)
+
+
+def test_wus_ablation_is_hadamard_free():
+    G = 8
+    sig = np.linspace(2, 1, G)
+    b = O.transforms_from_moments(np.eye(G)[None], np.diag(sig ** 2)[None], use_hadamard=False)
+    assert np.allclose(b["T_wush"][0], np.diag(sig ** -0.5), atol=1e-12)
+
+
+def test_damping_adds_scaled_identity():
+    S = np.array([[[4.0, 1.0], [1.0, 2.0]]])
+    D = O.damp(S, 0.5)
+    assert np.allclose(D[0], [[5.5, 1.0], [1.0, 3.5]])
+
+
+def test_second_moments_exact_on_basis_tokens():
+    """Tokens that are scaled basis vectors give a diagonal second moment whose entries
+    are the mean squared scale per channel; weights with one nonzero per row likewise."""
+    G, C = 4, 2
+    d = G * C
+    x = np.zeros((2 * d, d))
+    for j in range(d):
+        x[j, j] = 2.0
+        x[d + j, j] = -4.0
+    w = np.zeros((d, d))
+    w[np.arange(d), np.arange(d)] = np.arange(1, d + 1)
+    Sw, Sx = O.block_second_moments(w, x, G)
+    for i in range(C):
+        assert np.allclose(Sx[i], np.eye(G) * (4.0 + 16.0) / (2 * d))
+        assert np.allclose(Sw[i], np.diag(np.arange(i * G + 1, i * G + G + 1) ** 2 / d))
+
+
+def test_transformed_calibration_data_has_HSH_moment():
+    """End-to-end pin of second moments + construction + block_transform on data:
+    the empirical second moment of y = T_wush x over the calibration tokens is H S H^T,
+    and of T_xvsh w over the weight rows likewise (lam = 0, exact algebra)."""
+    inp, b = _tiny_build(lam=0.0)
+    xcal = O.bf16_to_f64(inp.xcal_bits)
+    y = O.block_transform(xcal, b["T_wush"])
+    wb = O.block_transform(inp.w.astype(np.float64), b["T_xvsh"])
+    G = 32
+    H = O.sylvester_hadamard(G)
+    for i in range(b["T_wush"].shape[0]):
+        HSH = H @ np.diag(b["s"][i]) @ H.T
+        yi = y[:, i * G:(i + 1) * G]
+        wi = wb[:, i * G:(i + 1) * G]
+        assert np.allclose(yi.T @ yi / yi.shape[0], HSH, atol=1e-9 * np.max(np.abs(HSH)))
+        assert np.allclose(wi.T @ wi / wi.shape[0], HSH, atol=1e-9 * np.max(np.abs(HSH)))
+
+
+def test_unquantised_product_preserved():
+    """W^T X is unchanged by the transform pair: sum over blocks of (T_xvsh w).(T_wush x) = w.x."""
+    inp, b = _tiny_build(lam=0.01)
+    x = O.bf16_to_f64(inp.x_bits)
+    w = inp.w.astype(np.float64)
+    ref = w @ x.T
+    got = O.block_transform(w, b["T_xvsh"]) @ O.block_transform(x, b["T_wush"]).T
+    assert np.max(np.abs(got - ref)) < 1e-9 * np.max(np.abs(ref))
+
+
+# ---------------------------------------------------------------- block_transform
+
+
+def test_block_transform_permutation_and_identity():
+    rng = np.random.default_rng(1)
+    G, C, n = 4, 3, 5
+    x = rng.standard_normal((n, C * G))
+    I = np.stack([np.eye(G)] * C)
+    assert np.array_equal(O.block_transform(x, I), x)
+    # T_i maps channel c to output r = (c + 1) mod G, i.e. T[r, c] = 1 iff r = c + 1 mod G.
+    P = np.zeros((G, G))
+    P[(np.arange(G) + 1) % G, np.arange(G)] = 1.0
+    Ts = np.stack([P, np.eye(G), 2 * np.eye(G)])
+    y = O.block_transform(x, Ts)
+    xb = x.reshape(n, C, G)
+    assert np.array_equal(y.reshape(n, C, G)[:, 0, (np.arange(G) + 1) % G], xb[:, 0, :])
+    assert np.array_equal(y.reshape(n, C, G)[:, 1], xb[:, 1])
+    assert np.array_equal(y.reshape(n, C, G)[:, 2], 2 * xb[:, 2])
+
+
+def test_block_transform_basis_vector_gives_column():
+    G = 8
+    T = np.arange(G * G, dtype=float).reshape(1, G, G)
+    for c in range(G):
+        e = np.zeros((1, G))
+        e[0, c] = 1.0
+        assert np.array_equal(O.block_transform(e, T)[0], T[0][:, c])
+
+
+# ---------------------------------------------------------------- grids, brute force
+
+
+def _e2m1_brute(v):
+    """Exhaustive nearest-grid search over the eight magnitudes; ties -> even index."""
+    grid = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+    a = abs(v)
+    best = None
+    for m, g in enumerate(grid):
+        d = abs(g - a)
+        if best is None or d < best[0] or (d == best[0] and m % 2 == 0):
+            best = (d, m)
+    return best[1] | (8 if math.copysign(1.0, v) < 0 else 0)
+
+
+def test_e2m1_matches_brute_force():
+    rng = np.random.default_rng(7)
+    vals = np.concatenate([rng.uniform(-8, 8, 4000),
+                           np.arange(-7.0, 7.01, 0.25),   # every tie point and grid point
+                           [6.0000001, -6.5, 100.0, 0.0, -0.0, 1e-30]])
+    got = O.e2m1_encode(vals)
+    for v, g in zip(vals, got):
+        assert int(g) == _e2m1_brute(float(v)), v
+
+
+def test_e2m1_decode_roundtrip():
+    codes = np.arange(16, dtype=np.uint8)
+    back = O.e2m1_encode(O.e2m1_decode(codes))
+    assert np.array_equal(back, codes)
+
+
+def _e4m3_value(b):
+    s = -1.0 if b & 0x80 else 1.0
+    e = (b >> 3) & 0xF
+    m = b & 7
+    if e == 0:
+        return s * m / 512.0
+    return s * (8 + m) / 8.0 * 2.0 ** (e - 7)
+
+
+def _e4m3_brute(r):
+    """Nearest over all 127 non-negative finite codes (0x00..0x7E); ties -> even code;
+    values beyond 448 saturate."""
+    a = abs(r)
+    best = None
+    for b in range(0x7F):
+        d = abs(_e4m3_value(b) - a)
+        if best is None or d < best[0] or (d == best[0] and b % 2 == 0):
+            best = (d, b)
+    return best[1] | (0x80 if r < 0 else 0)
+
+
+def test_e4m3_matches_brute_force_and_golden():
+    rng = np.random.default_rng(3)
+    vals = np.concatenate([rng.uniform(0, 460, 300), np.exp(rng.uniform(-9, 6, 700)),
+                           [_e4m3_value(b) for b in range(0x7F)],
+                           [(_e4m3_value(b) + _e4m3_value(b + 1)) / 2 for b in range(0x7E)]])
+    got = O.e4m3_encode(vals)
+    for v, g in zip(vals, got):
+        assert int(g) == _e4m3_brute(float(v)), v
+    with open(os.path.join(GOLDEN, "e4m3_examples.txt")) as f:
+        for line in f:
+            if line.startswith("#") or not line.strip():
+                continue
+            v, b = (t.strip() for t in line.split("|"))
+            assert int(O.e4m3_encode(np.array([float(v)]))[0]) == int(b, 16), line
+    for b in range(0x7F):
+        assert O.e4m3_decode(np.array([b], np.uint8))[0] == _e4m3_value(b)
+
+
+def _mx_exponent_brute(amax):
+    if amax == 0:
+        return -127
+    a = Fraction(amax)
+    for e in range(-400, 400):
+        if a <= 6 * Fraction(2) ** e:
+            return max(-127, min(127, e))
+    raise AssertionError
+
+
+def test_mxfp4_exponent_matches_search():
+    rng = np.random.default_rng(11)
+    vals = np.concatenate([np.exp(rng.uniform(-100, 80, 500)).astype(np.float32).astype(np.float64),
+                           [6.0 * 2.0 ** k for k in range(-20, 20)],
+                           [np.nextafter(np.float32(6.0 * 2.0 ** k), np.float32(np.inf)) for k in range(-5, 5)],
+                           [3.0, 0.0, 2.0 ** -140, 1e-45]])
+    got = O.mxfp4_exponent(vals)
+    for v, g in zip(vals, got):
+        assert int(g) == _mx_exponent_brute(float(v)), v
+
+
+def test_int4_rounding_matches_brute_force():
+    rng = np.random.default_rng(5)
+    y = rng.standard_normal((50, 32)) * rng.uniform(0.01, 10, (50, 1))
+    codes, s = O.quant_int4(y, 32)
+    q = O.int4_decode(codes)
+    for r in range(y.shape[0]):
+        sc = np.float32(np.max(np.abs(y[r])) / 7.0)
+        inv = np.float32(1.0 / np.float64(sc))
+        assert s[r, 0] == sc
+        for j in range(32):
+            v = float(np.float32(y[r, j] * np.float64(inv)))
+            best = min(range(-7, 8), key=lambda k: (abs(k - v), k % 2))
+            assert q[r, j] == best
+
+
+def _read_quant_examples():
+    rows = []
+    with open(os.path.join(GOLDEN, "quant_examples.txt")) as f:
+        for line in f:
+            if line.startswith("#") or not line.strip():
+                continue
+            fmt, ctx, vals, scale, codes = (t.strip() for t in line.split("|"))
+            rows.append((fmt, ctx, [float(v) for v in vals.split()], scale,
+                         [int(c, 16) for c in codes.split()]))
+    return rows
+
+
+@pytest.mark.parametrize("row", _read_quant_examples(), ids=lambda r: f"{r[0]}:{r[2][:2]}")
+def test_hand_worked_examples(row):
+    fmt, ctx, vals, scale, codes = row
+    g = {"mxfp4": 32, "nvfp4": 16, "int4": 32}[fmt]
+    y = np.zeros((1, g))
+    y[0, :len(vals)] = vals
+    want = np.zeros(g, dtype=np.uint8)
+    want[:len(codes)] = codes
+    if fmt == "mxfp4":
+        c, s = O.quant_mxfp4(y)
+        assert int(s[0, 0]) == int(scale, 16)
+    elif fmt == "nvfp4":
+        st = float(ctx.split("=")[1])
+        c, s, _ = O.quant_nvfp4(y, st)
+        assert int(s[0, 0]) == int(scale, 16)
+    else:
+        c, s = O.quant_int4(y, g)
+        assert float(s[0, 0]) == float(scale)
+    assert np.array_equal(c[0], want), (c[0][:len(codes)], codes)
+
+
+def test_ocp_floor_rule_differs_on_7():
+    """The alternative OCP exponent saturates 7 to 6 while the AbsMax rule keeps 8."""
+    y = np.zeros((1, 32))
+    y[0, 0] = 7.0
+    c_abs, s_abs = O.quant_mxfp4(y)
+    c_ocp, s_ocp = O.quant_mxfp4(y, rule="ocp_floor")
+    assert O.dequant(c_abs, s_abs, "mxfp4", 32)[0, 0] == 8.0
+    assert O.dequant(c_ocp, s_ocp, "mxfp4", 32)[0, 0] == 6.0
+
+
+def test_nvfp4_tensor_scale_definition():
+    assert O.nvfp4_tensor_scale(2688.0) == 1.0
+    assert O.nvfp4_tensor_scale(0.0) == 0.0
+    # amax / 2688 rounded to float32
+    assert O.nvfp4_tensor_scale(1.0) == float(np.float32(1.0 / 2688.0))
+
+
+def test_nvfp4_zero_and_underflow_groups():
+    y = np.zeros((1, 32))
+    y[0, 0] = 2688.0          # tensor amax -> s_t = 1
+    y[0, 16] = 1e-4           # r = 1e-4/6 < 2^-10 -> E4M3 0 -> whole group zero
+    c, s, st = O.quant_nvfp4(y)
+    assert st == 1.0 and s[0, 1] == 0 and np.all(c[0, 16:] & 7 == 0)
+
+
+# ---------------------------------------------------------------- packing
+
+
+def test_pack_low_nibble_is_even_element():
+    c = np.array([[1, 2, 3, 4, 0xF, 0]], dtype=np.uint8)
+    p = O.pack_nibbles(c)
+    assert p.tolist() == [[0x21, 0x43, 0x0F]]
+    assert np.array_equal(O.unpack_nibbles(p), c)
+
+
+# ---------------------------------------------------------------- composed path
+
+
+@pytest.mark.parametrize("fmt,G", [("mxfp4", 32), ("nvfp4", 16), ("int4", 32), ("int4", 16)])
+def test_quantiser_error_bound_and_amax_code(fmt, G):
+    """Every element dequantises to its nearest grid point at the group's scale, the
+    block maximum never saturates (MXFP4/INT4) and lands on the top binade."""
+    rng = np.random.default_rng(17)
+    y = rng.standard_t(3, (200, 4 * G)) * np.exp(rng.uniform(-6, 6, (200, 1)))
+    c, s, st = O.quantize(y, fmt, G)
+    deq = O.dequant(c, s, fmt, G, st)
+    g = y.reshape(200, 4, G)
+    dg = deq.reshape(200, 4, G)
+    if fmt == "mxfp4":
+        sc = np.exp2(s.astype(float) - 127)[:, :, None]
+        err = np.abs(dg - g) / sc
+        v = np.abs(g) / sc
+        half = np.where(v < 2, 0.25, np.where(v < 4, 0.5, 1.0))
+        assert np.all(err <= half + 1e-12)
+        top = np.abs(g).max(axis=2, keepdims=True) / sc
+        assert np.all((top > 3) & (top <= 6))
+    elif fmt == "int4":
+        sc = s.astype(float)[:, :, None]
+        assert np.all(np.abs(dg - g) <= 0.5 * sc * (1 + 1e-6))
+        q = O.int4_decode(c).reshape(200, 4, G)
+        amax_idx = np.argmax(np.abs(g), axis=2)
+        assert np.all(np.abs(np.take_along_axis(q, amax_idx[:, :, None], 2)) == 7)
+    else:
+        scd = (O.e4m3_decode(s) * st)[:, :, None]
+        zero = (s == 0)[:, :, None]                     # block scale underflowed: group is all zero
+        assert np.all(np.broadcast_to(zero, g.shape) <= (dg == 0))
+        with np.errstate(divide="ignore", invalid="ignore"):
+            v = np.where(zero, 0.0, np.abs(g) / np.where(zero, 1.0, scd))
+        half = np.where(v < 2, 0.25, np.where(v < 4, 0.5, 1.0)) * scd
+        ok = (np.abs(dg - g) <= half * (1 + 1e-6)) | zero
+        sat = v > 6.0
+        assert np.all(ok | sat)
+        # the 3-bit mantissa of a normal E4M3 scale rounds by at most 1/16, so a group
+        # maximum can exceed 6 only a little before it saturates
+        normal = np.broadcast_to((s >= 0x08)[:, :, None], g.shape)
+        assert np.all(v[sat & normal] < 6.0 * (1 + 2 ** -3))
+
+
+def test_quant_act_tiny_bit_patterns_and_shapes():
+    wl = workload("tiny_mxfp4")
+    inp = make_inputs(wl)
+    b = O.build_transforms(inp.w, inp.xcal_bits, 32)
+    codes, scales, st, y = O.quant_act(inp.x_bits, b["T_wush32"], 32, "mxfp4")
+    assert codes.shape == (64, 128) and scales.shape == (64, 8) and st is None
+    deq = O.dequant(O.unpack_nibbles(codes), scales, "mxfp4", 32)
+    # MXFP4 relative error on Gaussian-like data: a few percent, far below 1
+    rel = np.linalg.norm(deq - y) / np.linalg.norm(y)
+    assert 1e-3 < rel < 0.2
+
+
+def test_generator_bf16_rounding_is_rne():
+    v = np.array([1.0, 1.0 + 2 ** -8, 1.0 + 3 * 2 ** -9, -2.5, 1.0 + 2 ** -7 + 2 ** -8])
+    bits = bf16_bits_from_f64(v)
+    # 1 + 2^-8 is a tie between 1 and 1 + 2^-7 -> even (1.0); 1 + 3*2^-9 rounds up to 1 + 2^-7;
+    # 1 + 2^-7 + 2^-8 ties between 1+2^-7 (odd) and 1+2^-6 (even) -> 1 + 2^-6.
+    assert np.array_equal(O.bf16_to_f64(bits), [1.0, 1.0, 1.0 + 2 ** -7, -2.5, 1.0 + 2 ** -6])
