@@ -1,0 +1,378 @@
+#!/usr/bin/env python
+"""Throughput of the fused WUSH transform + MXFP4 quantisation on the Llama-8B-like
+attention-input workload: 4096 tokens x d_in = 4096, G = 32, bf16 activations.
+
+One step = one call of wush_quant_act over the whole 4096 x 4096 batch.  Inputs are
+resident in HBM; eight rotating input/output sets (8 x 43 MB > 126 MB L2) make every
+step read its activations from DRAM.  The timed region replays CUDA graphs of the
+launches, bracketed by a barrier + synchronize and CUDA events on the launching
+stream; under torchrun every rank runs its own batch (weak scaling) and the time is
+the maximum over ranks.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
+
+Prints one JSON line (rank 0).  ``--impl reference`` times the float64 CPU oracle on
+the host cores instead, on bounded samples of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "WUSH+quant GB/s & tokens/s at d=4096 G=32 MXFP4; % of HBM roofline"
+WORKLOAD = "attn_mxfp4_4096"
+N_SETS = 8
+GRAPH_LEN = 100
+FALLBACK_HBM_GBS = 6650.0
+PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "wush_fused_mxfp4_attn_4096.md")
+KERNEL_SOURCES = ("blockwise_adaptive_transforms_b200/csrc/wush_fused.cuh",
+                  "blockwise_adaptive_transforms_b200/csrc/wush_ptx.cuh")
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20000)
+    ap.add_argument("--warmup", type=int, default=2000)
+    ap.add_argument("--impl", choices=("native", "reference"), default="native")
+    ap.add_argument("--e2e-steps", type=int, default=30)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def algorithmic_bytes(n_tok: int, d_in: int, G: int) -> int:
+    """Bytes one step must move: read x (bf16) and T (fp32), write codes and E8M0 scales."""
+    C = d_in // G
+    return n_tok * d_in * 2 + n_tok * d_in // 2 + n_tok * C + C * G * G * 4
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic():
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on the
+    current kernel source; else None."""
+    try:
+        fields = {}
+        with open(PROFILE_SUMMARY) as f:
+            for line in f:
+                if ":" in line and line.strip().startswith("- "):
+                    k, v = line.strip()[2:].split(":", 1)
+                    fields[k.strip()] = v.strip().strip("`")
+        if fields.get("kernel_source_sha256_16") != kernel_source_hash():
+            return None
+        return int(fields["dram_bytes_per_launch"])
+    except (OSError, KeyError, ValueError):
+        return None
+
+
+def hbm_peak():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while running (read only)."""
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x2: "applications_clocks_setting"}
+
+    def __init__(self, device_index: int, period_s: float = 0.002):
+        self.samples, self.reasons, self.max_mhz = [], 0, None
+        self.period = period_s
+        self._stop = threading.Event()
+        self._h = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            try:
+                import torch
+                p = torch.cuda.get_device_properties(device_index)
+                bus = f"{p.pci_domain_id:08X}:{p.pci_bus_id:02X}:{p.pci_device_id:02X}.0"
+                self._h = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+            except Exception:
+                self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self._h = None
+
+    def _run(self):
+        nv = self._nv
+        get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                self.reasons |= int(get_reasons(self._h))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self._h is not None:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self._h is not None:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"], "samples": 0}
+        names = [n for bit, n in self.REASONS.items() if self.reasons & bit]
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz, "reasons": names,
+                "samples": len(self.samples)}
+
+
+def cpu_baseline(inp, wl, seconds: float):
+    """The float64 oracle, as it stands, on the host cores: repeated calls on 256-token
+    samples of the workload for about `seconds`, scaled to the metric's bytes."""
+    from oracle import wush_oracle as O
+    from threadpoolctl import threadpool_info
+    b = O.build_transforms(inp.w, inp.xcal_bits, wl.G)
+    T32 = b["T_wush32"]
+    rows = 256
+    O.quant_act(inp.x_bits[:rows], T32, wl.G, wl.fmt)
+    done, t0, i = 0, time.perf_counter(), 0
+    while time.perf_counter() - t0 < seconds:
+        r0 = (i * rows) % wl.n_tok
+        O.quant_act(inp.x_bits[r0:r0 + rows], T32, wl.G, wl.fmt)
+        done += rows
+        i += 1
+    dt = time.perf_counter() - t0
+    per_tok = algorithmic_bytes(wl.n_tok, wl.d_in, wl.G) / wl.n_tok
+    threads = max([p.get("num_threads", 1) for p in threadpool_info()] + [1])
+    return {"value": round(done / dt * per_tok / 1e9, 6), "unit": "GB/s", "cores": threads, "kind": "oracle",
+            "tokens_per_s": round(done / dt, 1),
+            "sample": f"{done} tokens in {rows}-token slices of the {wl.n_tok}x{wl.d_in} workload, "
+                      f"{dt:.1f} s; bytes scaled per token"}
+
+
+def run_reference(args):
+    """--impl reference: the float64 CPU oracle, on rank 0 only."""
+    if int(os.environ.get("RANK", "0")) != 0:
+        return
+    from workloads import make_inputs, workload
+    from oracle import wush_oracle as O
+    from threadpoolctl import threadpool_info
+    wl = workload(WORKLOAD)
+    inp = make_inputs(wl)
+    b = O.build_transforms(inp.w, inp.xcal_bits, wl.G)
+    T32 = b["T_wush32"]
+    total = max(1, args.steps + args.warmup)
+    rows = max(1, min(256, int(60.0 / (total * 2.5e-4))))
+    per_tok = algorithmic_bytes(wl.n_tok, wl.d_in, wl.G) / wl.n_tok
+    for i in range(args.warmup):
+        r0 = (i * rows) % wl.n_tok
+        O.quant_act(inp.x_bits[r0:r0 + rows], T32, wl.G, wl.fmt)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        r0 = (i * rows) % wl.n_tok
+        O.quant_act(inp.x_bits[r0:r0 + rows], T32, wl.G, wl.fmt)
+    dt = time.perf_counter() - t0
+    toks = rows * args.steps
+    value = toks / dt * per_tok / 1e9
+    threads = max([p.get("num_threads", 1) for p in threadpool_info()] + [1])
+    sample = f"{rows} tokens per step of the {wl.n_tok}x{wl.d_in} workload; bytes scaled per token"
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "GB/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(dt / args.steps * 1e3, 4), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "tokens_per_s": round(toks / dt, 1),
+            "config": {"workload": WORKLOAD, "tokens": wl.n_tok, "d_in": wl.d_in, "G": wl.G, "fmt": wl.fmt},
+            "cpu_baseline": {"value": round(value, 6), "unit": "GB/s", "cores": threads, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": round(value, 6), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_native(args):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+    import blockwise_adaptive_transforms_b200 as W
+    from workloads import make_inputs, workload
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    wl = workload(WORKLOAD)
+    inp = make_inputs(wl)
+    G, n, d = wl.G, wl.n_tok, wl.d_in
+    C = d // G
+    step_bytes = algorithmic_bytes(n, d, G)
+
+    # transforms: built on the device from the weights and calibration activations
+    w_dev = torch.from_numpy(inp.w).to(dev)
+    xcal_dev = torch.from_numpy(inp.xcal_bits.view(np.int16)).view(torch.bfloat16).to(dev)
+    tb0 = time.perf_counter()
+    T, _ = W.wush_build_transforms(w_dev, xcal_dev, G)
+    torch.cuda.synchronize()
+    build_ms = (time.perf_counter() - tb0) * 1e3
+    del w_dev, xcal_dev
+
+    x_host = torch.from_numpy(inp.x_bits.view(np.int16)).view(torch.bfloat16)
+    xs = [x_host.to(dev) for _ in range(N_SETS)]
+    codes = [torch.empty((n, d // 2), dtype=torch.uint8, device=dev) for _ in range(N_SETS)]
+    scales = [torch.empty((n, C), dtype=torch.uint8, device=dev) for _ in range(N_SETS)]
+    stream = torch.cuda.Stream(device=dev)
+
+    def launch(i):
+        k = i % N_SETS
+        W.wush_quant_act(xs[k], T, G, wl.fmt, codes=codes[k], scales=scales[k], stream=stream)
+
+    # warm-up: eager launches, then capture the graphs
+    with torch.cuda.stream(stream):
+        for i in range(min(args.warmup, 64)):
+            launch(i)
+        stream.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            for i in range(GRAPH_LEN):
+                launch(i)
+        rem = args.steps % GRAPH_LEN
+        tail = None
+        if rem:
+            tail = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(tail, stream=stream):
+                for i in range(rem):
+                    launch(i)
+        done = min(args.warmup, 64)
+        while done < args.warmup:
+            graph.replay()
+            done += GRAPH_LEN
+        stream.synchronize()
+    st, bits = W.wush_device_status(stream)
+    if st != 0:
+        raise RuntimeError(f"device error word {bits:#x} after warm-up")
+
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clocks:
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for _ in range(args.steps // GRAPH_LEN):
+                graph.replay()
+            if tail is not None:
+                tail.replay()
+            e1.record(stream)
+        e1.synchronize()
+    torch.cuda.synchronize()
+    elapsed_s = e0.elapsed_time(e1) / 1e3
+    if world > 1:
+        t = torch.tensor([elapsed_s], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_s = float(t.item())
+        dist.barrier()
+    st, bits = W.wush_device_status(stream)
+    if st != 0:
+        raise RuntimeError(f"device error word {bits:#x} after the timed region")
+
+    per_launch_s = elapsed_s / args.steps
+    value = world * args.steps * step_bytes / elapsed_s / 1e9
+    tokens_s = world * args.steps * n / elapsed_s
+    achieved = step_bytes / per_launch_s / 1e9
+    peak, peak_kind = hbm_peak()
+
+    # end to end through the public API: pinned host x -> device, kernel, codes + scales -> pinned host
+    x_pin = x_host.pin_memory()
+    c_pin = torch.empty((n, d // 2), dtype=torch.uint8).pin_memory()
+    s_pin = torch.empty((n, C), dtype=torch.uint8).pin_memory()
+    with torch.cuda.stream(stream):
+        def e2e_step():
+            xs[0].copy_(x_pin, non_blocking=True)
+            W.wush_quant_act(xs[0], T, G, wl.fmt, codes=codes[0], scales=scales[0], stream=stream)
+            c_pin.copy_(codes[0], non_blocking=True)
+            s_pin.copy_(scales[0], non_blocking=True)
+        for _ in range(3):
+            e2e_step()
+        stream.synchronize()
+        if world > 1:
+            dist.barrier()
+        f0 = torch.cuda.Event(enable_timing=True)
+        f1 = torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        f1.record(stream)
+        f1.synchronize()
+    e2e_s = f0.elapsed_time(f1) / 1e3
+    if world > 1:
+        t = torch.tensor([e2e_s], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_s = float(t.item())
+    e2e_value = world * args.e2e_steps * step_bytes / e2e_s / 1e9
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(inp, wl, args.cpu_seconds)
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    clk = clocks.summary()
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(per_launch_s * 1e3, 6),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "tokens_per_s": round(tokens_s, 1),
+        "hbm_roofline_frac": round(achieved / peak, 4),
+        "config": {"workload": WORKLOAD, "tokens": n, "d_in": d, "G": G, "fmt": wl.fmt,
+                   "l2": f"{N_SETS} rotating input/output sets ({N_SETS * step_bytes / 1e6:.0f} MB > 126 MB L2)",
+                   "launch": f"CUDA graphs of {GRAPH_LEN} launches", "transform_build_ms": round(build_ms, 2)},
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                     "frac": round(achieved / peak, 4), "traffic": measured_traffic(),
+                     "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
+                     else "fallback", "algorithmic_bytes_per_launch": step_bytes},
+        "cpu_baseline": cpu,
+        "e2e": {"value": round(e2e_value, 3), "unit": "GB/s", "h2d_bytes_per_step": n * d * 2,
+                "d2h_bytes_per_step": n * d // 2 + n * C, "steps": args.e2e_steps},
+        "gpu_launches": args.steps,
+        "clocks": clk,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_native(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,234 @@
+"""B200-native fused WUSH blockwise transform + 4-bit quantisation.
+
+Thin Python binding of the C ABI in ``include/wush.h`` (``libwush.so``, built in-tree
+for sm_100a).  The functions carry the C names; they only marshal arguments: torch
+tensors supply device memory and the current CUDA stream, every step of the
+computation runs in the library's kernels.  There is no CPU fallback: if the library
+is missing or cannot be loaded, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+from ._build import LIB_PATH, build as build_library  # noqa: F401
+
+__all__ = ["FMT", "WushError", "wush_quant_act", "wush_quant_weight", "wush_quant_act_debug",
+           "wush_quant_weight_debug", "wush_build_transforms", "wush_device_status", "wush_set_wait_limit_ns",
+           "wush_selftest_wait_timeout", "wush_status_string", "wush_version", "load_library",
+           "EXPORTED_SYMBOLS", "output_shapes"]
+
+FMT = {"mxfp4": 0, "nvfp4": 1, "int4": 2}
+STATUS = {0: "WUSH_OK", 1: "WUSH_ERR_INVALID_ARG", 2: "WUSH_ERR_UNSUPPORTED", 3: "WUSH_ERR_MISALIGNED",
+          4: "WUSH_ERR_CUDA", 5: "WUSH_ERR_DEVICE_TIMEOUT"}
+EXPORTED_SYMBOLS = ("wush_quant_act", "wush_quant_weight", "wush_quant_act_debug",
+                    "wush_quant_weight_debug", "wush_build_transforms", "wush_device_status",
+                    "wush_set_wait_limit_ns",
+                    "wush_selftest_wait_timeout", "wush_status_string", "wush_version")
+
+
+class WushError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {wush_status_string(status)} (status {status})")
+
+
+_LIB = None
+_P, _I64, _I32, _U64 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_uint64
+
+
+def load_library(path: str | None = None) -> ctypes.CDLL:
+    """Load libwush.so (once) and declare the C signatures."""
+    global _LIB
+    if _LIB is not None and path is None:
+        return _LIB
+    p = path or LIB_PATH
+    if not os.path.exists(p):
+        raise OSError(f"{p} is missing: build it with `python -m blockwise_adaptive_transforms_b200._build`")
+    lib = ctypes.CDLL(p)
+    quant = [_P, _P, _I64, _I64, _I32, _I32, _P, _P, _P, _P]
+    lib.wush_quant_act.argtypes = quant
+    lib.wush_quant_weight.argtypes = quant
+    dbg = [_P, _P, _I64, _I64, _I32, _I32, _P, _P, _P, _P, _P]
+    lib.wush_quant_act_debug.argtypes = dbg
+    lib.wush_quant_weight_debug.argtypes = dbg
+    for f in ("wush_quant_act", "wush_quant_weight", "wush_quant_act_debug", "wush_quant_weight_debug"):
+        getattr(lib, f).restype = ctypes.c_int
+    lib.wush_build_transforms.argtypes = [_P, _P, _I64, _I64, _I64, _I32, ctypes.c_double, _I32,
+                                          _P, _P, _P, _P, _P, _P]
+    lib.wush_build_transforms.restype = ctypes.c_int
+    lib.wush_device_status.argtypes = [_P, ctypes.POINTER(ctypes.c_uint32)]
+    lib.wush_device_status.restype = ctypes.c_int
+    lib.wush_set_wait_limit_ns.argtypes = [_U64]
+    lib.wush_set_wait_limit_ns.restype = ctypes.c_int
+    lib.wush_selftest_wait_timeout.argtypes = [_U64, _P, ctypes.POINTER(ctypes.c_uint32)]
+    lib.wush_selftest_wait_timeout.restype = ctypes.c_int
+    lib.wush_status_string.argtypes = [ctypes.c_int]
+    lib.wush_status_string.restype = ctypes.c_char_p
+    lib.wush_version.argtypes = []
+    lib.wush_version.restype = ctypes.c_int
+    if path is None:
+        _LIB = lib
+    return lib
+
+
+def wush_status_string(status: int) -> str:
+    return load_library().wush_status_string(int(status)).decode()
+
+
+def wush_version() -> int:
+    return int(load_library().wush_version())
+
+
+def _stream_handle(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return int(stream.cuda_stream) if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _fmt_code(fmt) -> int:
+    return FMT[fmt] if isinstance(fmt, str) else int(fmt)
+
+
+def output_shapes(rows: int, d_in: int, G: int, fmt):
+    """(codes shape, scales shape, scales dtype) of a call."""
+    f = _fmt_code(fmt)
+    return (rows, d_in // 2), (rows, d_in // G), (torch.float32 if f == FMT["int4"] else torch.uint8)
+
+
+def _check_dev(t: torch.Tensor, name: str, dtype=None):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _alloc_outputs(ref: torch.Tensor, rows: int, d_in: int, G: int, fmt, codes, scales, tensor_scale):
+    cs, ss, sdt = output_shapes(rows, d_in, G, fmt)
+    if codes is None:
+        codes = torch.empty(cs, dtype=torch.uint8, device=ref.device)
+    if scales is None:
+        scales = torch.empty(ss, dtype=sdt, device=ref.device)
+    if tensor_scale is None and _fmt_code(fmt) == FMT["nvfp4"]:
+        tensor_scale = torch.empty(1, dtype=torch.float32, device=ref.device)
+    _check_dev(codes, "codes", torch.uint8)
+    _check_dev(scales, "scales", sdt)
+    if tuple(codes.shape) != cs or tuple(scales.shape) != ss:
+        raise ValueError(f"output shapes must be codes {cs} and scales {ss}")
+    if tensor_scale is not None:
+        _check_dev(tensor_scale, "tensor_scale", torch.float32)
+    return codes, scales, tensor_scale
+
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def _call(fn_name, inp, in_dtype, T, G, fmt, codes, scales, tensor_scale, y, stream):
+    lib = load_library()
+    _check_dev(inp, "input", in_dtype)
+    _check_dev(T, "T", torch.float32)
+    if inp.dim() != 2:
+        raise ValueError("input must be 2-D [rows][d_in]")
+    rows, d_in = int(inp.shape[0]), int(inp.shape[1])
+    if d_in % G:
+        raise ValueError("d_in must be a multiple of G")
+    if tuple(T.shape) != (d_in // G, G, G):
+        raise ValueError(f"T must have shape {(d_in // G, G, G)}")
+    codes, scales, tensor_scale = _alloc_outputs(inp, rows, d_in, G, fmt, codes, scales, tensor_scale)
+    args = [_ptr(inp), _ptr(T), rows, d_in, int(G), _fmt_code(fmt), _ptr(codes), _ptr(scales),
+            _ptr(tensor_scale)]
+    if y is not None:
+        args.append(_ptr(y))
+    args.append(_stream_handle(stream))
+    with torch.cuda.device(inp.device):
+        st = getattr(lib, fn_name)(*args)
+    if st != 0:
+        raise WushError(st, fn_name)
+    return codes, scales, tensor_scale
+
+
+def wush_quant_act(x, T, G, fmt, codes=None, scales=None, tensor_scale=None, stream=None):
+    """Activations x (bf16 [n_tok][d_in]) -> (codes u8 [n_tok][d_in/2], scales, tensor_scale)."""
+    return _call("wush_quant_act", x, torch.bfloat16, T, G, fmt, codes, scales, tensor_scale, None, stream)
+
+
+def wush_quant_weight(w, T, G, fmt, codes=None, scales=None, tensor_scale=None, stream=None):
+    """Weights w (fp32 [d_out][d_in]) -> (codes, scales, tensor_scale)."""
+    return _call("wush_quant_weight", w, torch.float32, T, G, fmt, codes, scales, tensor_scale, None, stream)
+
+
+def _y_buffer(inp, y):
+    if y is None:
+        y = torch.empty(inp.shape, dtype=torch.float32, device=inp.device)
+    _check_dev(y, "y_out", torch.float32)
+    if tuple(y.shape) != tuple(inp.shape):
+        raise ValueError("y_out must have the input's shape")
+    return y
+
+
+def wush_quant_act_debug(x, T, G, fmt, y_out=None, stream=None):
+    """As wush_quant_act, also returning the fp32 transformed values y the kernel quantised."""
+    y = _y_buffer(x, y_out)
+    c, s, ts = _call("wush_quant_act_debug", x, torch.bfloat16, T, G, fmt, None, None, None, y, stream)
+    return c, s, ts, y
+
+
+def wush_quant_weight_debug(w, T, G, fmt, y_out=None, stream=None):
+    y = _y_buffer(w, y_out)
+    c, s, ts = _call("wush_quant_weight_debug", w, torch.float32, T, G, fmt, None, None, None, y, stream)
+    return c, s, ts, y
+
+
+def wush_build_transforms(w, xcal, G, lam=0.01, use_hadamard=True, want_f64=False, stream=None):
+    """Per-block WUSH transforms of one layer, built on the device in fp64.
+
+    w: fp32 [d_out][d_in] weights; xcal: bf16 [n_cal][d_in] calibration activations.
+    Returns (T_wush, T_xvsh) as fp32 [C][G][G]; with ``want_f64`` also the fp64
+    transforms and the singular values: (T_wush, T_xvsh, T_wush64, T_xvsh64, s64)."""
+    lib = load_library()
+    _check_dev(w, "w", torch.float32)
+    _check_dev(xcal, "xcal", torch.bfloat16)
+    if w.dim() != 2 or xcal.dim() != 2 or w.shape[1] != xcal.shape[1]:
+        raise ValueError("w [d_out][d_in] and xcal [n_cal][d_in] must share d_in")
+    d_out, d_in = int(w.shape[0]), int(w.shape[1])
+    n_cal = int(xcal.shape[0])
+    if d_in % G:
+        raise ValueError("d_in must be a multiple of G")
+    C = d_in // G
+    dev = w.device
+    Tw = torch.empty((C, G, G), dtype=torch.float32, device=dev)
+    Tx = torch.empty_like(Tw)
+    Tw64 = Tx64 = s64 = None
+    if want_f64:
+        Tw64 = torch.empty((C, G, G), dtype=torch.float64, device=dev)
+        Tx64 = torch.empty_like(Tw64)
+        s64 = torch.empty((C, G), dtype=torch.float64, device=dev)
+    with torch.cuda.device(dev):
+        st = lib.wush_build_transforms(_ptr(w), _ptr(xcal), d_out, n_cal, d_in, int(G), float(lam),
+                                       1 if use_hadamard else 0, _ptr(Tw), _ptr(Tx), _ptr(Tw64),
+                                       _ptr(Tx64), _ptr(s64), _stream_handle(stream))
+    if st != 0:
+        raise WushError(st, "wush_build_transforms")
+    return (Tw, Tx, Tw64, Tx64, s64) if want_f64 else (Tw, Tx)
+
+
+def wush_device_status(stream=None):
+    """Synchronise the stream, read and clear the device error word: (status, bits)."""
+    bits = ctypes.c_uint32(0)
+    st = load_library().wush_device_status(_stream_handle(stream), ctypes.byref(bits))
+    return int(st), int(bits.value)
+
+
+def wush_set_wait_limit_ns(ns: int) -> None:
+    load_library().wush_set_wait_limit_ns(int(ns))
+
+
+def wush_selftest_wait_timeout(limit_ns: int, stream=None):
+    bits = ctypes.c_uint32(0)
+    st = load_library().wush_selftest_wait_timeout(int(limit_ns), _stream_handle(stream), ctypes.byref(bits))
+    return int(st), int(bits.value)

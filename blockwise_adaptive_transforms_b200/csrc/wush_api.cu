@@ -1,0 +1,267 @@
+// Host side of the C ABI declared in include/wush.h: argument validation, TMA
+// descriptor encoding, kernel selection and launch.  No allocation, no host
+// synchronisation on the quantisation calls.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <climits>
+#include <cstdint>
+#include <mutex>
+
+#include "wush.h"
+#include "wush_fused.cuh"
+#include "wush_build.cuh"
+
+namespace wush {
+// Waits on an mbarrier that no thread ever arrives on; the bounded wait must give up.
+__global__ void wush_selftest_wait_kernel(unsigned long long limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_word;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_addr(&bar), 1);
+    abort_word = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) wait_bounded(smem_addr(&bar), 0u, &abort_word, 32u, limit_ns);
+}
+}  // namespace wush
+
+namespace {
+
+constexpr unsigned long long kDefaultWaitLimitNs = 2000000000ull;
+std::atomic<unsigned long long> g_wait_limit_ns{kDefaultWaitLimitNs};
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return static_cast<PFN_cuTensorMapEncodeTiled_v12000>(nullptr);
+    return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }();
+  return fn;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+// 2-D row-major [rows][cols] tensor, box {box_cols, 128 rows}.
+int encode_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dt, int elem_bytes, int64_t rows,
+              int64_t cols, int box_cols, CUtensorMapSwizzle swz) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return WUSH_ERR_CUDA;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * static_cast<cuuint64_t>(elem_bytes)};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(box_cols), 128u};
+  cuuint32_t estr[2] = {1u, 1u};
+  CUresult r = enc(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? WUSH_OK : WUSH_ERR_CUDA;
+}
+
+template <class Cfg>
+int launch_fused(const CUtensorMap& map, wush::FusedParams p, cudaStream_t stream) {
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return WUSH_ERR_CUDA;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return WUSH_ERR_CUDA;
+  static std::atomic<unsigned long long> configured{0ull};   // one bit per device ordinal
+  const unsigned long long bit = 1ull << (dev & 63);
+  if (!(configured.load(std::memory_order_acquire) & bit)) {
+    if (cudaFuncSetAttribute(wush::wush_fused_kernel<Cfg>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             Cfg::SMEM_BYTES) != cudaSuccess)
+      return WUSH_ERR_CUDA;
+    configured.fetch_or(bit, std::memory_order_acq_rel);
+  }
+  const int grid = p.total_tiles < sms ? p.total_tiles : sms;
+  wush::wush_fused_kernel<Cfg><<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(map, p);
+  return cudaGetLastError() == cudaSuccess ? WUSH_OK : WUSH_ERR_CUDA;
+}
+
+template <int G, int FMT, bool IN_F32, bool AMAX_ONLY>
+int launch_pick_y(const CUtensorMap& map, const wush::FusedParams& p, bool emit_y, cudaStream_t s) {
+  if (emit_y) return launch_fused<wush::FusedCfg<G, FMT, IN_F32, AMAX_ONLY, true>>(map, p, s);
+  return launch_fused<wush::FusedCfg<G, FMT, IN_F32, AMAX_ONLY, false>>(map, p, s);
+}
+
+template <bool IN_F32>
+int dispatch(const CUtensorMap& map, wush::FusedParams p, int G, int fmt, bool emit_y, float* tensor_scale,
+             cudaStream_t s) {
+  if (fmt == WUSH_MXFP4) return launch_pick_y<32, wush::kMXFP4, IN_F32, false>(map, p, emit_y, s);
+  if (fmt == WUSH_INT4) {
+    if (G == 32) return launch_pick_y<32, wush::kINT4, IN_F32, false>(map, p, emit_y, s);
+    return launch_pick_y<16, wush::kINT4, IN_F32, false>(map, p, emit_y, s);
+  }
+  // NVFP4: pass 1 finds amax|y| (float bits, running max in *tensor_scale), a one-thread
+  // kernel turns it into s_t in place, pass 2 quantises with s_t.
+  if (cudaMemsetAsync(tensor_scale, 0, sizeof(float), s) != cudaSuccess) return WUSH_ERR_CUDA;
+  p.amax_word = reinterpret_cast<unsigned int*>(tensor_scale);
+  int st = launch_fused<wush::FusedCfg<16, wush::kNVFP4, IN_F32, true, false>>(map, p, s);
+  if (st != WUSH_OK) return st;
+  wush::wush_nvfp4_tensor_scale_kernel<<<1, 32, 0, s>>>(tensor_scale);
+  if (cudaGetLastError() != cudaSuccess) return WUSH_ERR_CUDA;
+  p.amax_word = nullptr;
+  p.tensor_scale = tensor_scale;
+  return launch_pick_y<16, wush::kNVFP4, IN_F32, false>(map, p, emit_y, s);
+}
+
+int quant_common(const void* in, bool in_f32, const float* T, int64_t rows, int64_t d_in, int G, int fmt,
+                 uint8_t* codes, void* scales, float* tensor_scale, float* y_out, bool debug,
+                 wush_stream_t stream) {
+  if (fmt != WUSH_MXFP4 && fmt != WUSH_NVFP4 && fmt != WUSH_INT4) return WUSH_ERR_UNSUPPORTED;
+  const bool g_ok = (fmt == WUSH_MXFP4 && G == 32) || (fmt == WUSH_NVFP4 && G == 16) ||
+                    (fmt == WUSH_INT4 && (G == 16 || G == 32));
+  if (!g_ok) return WUSH_ERR_UNSUPPORTED;
+  if (rows < 0 || d_in <= 0 || d_in % G != 0) return WUSH_ERR_INVALID_ARG;
+  if (rows > INT_MAX || d_in > INT_MAX) return WUSH_ERR_INVALID_ARG;
+  if (rows == 0) return WUSH_OK;   // empty batch: nothing to read or write, pointers unused
+  if (!in || !T || !codes || !scales) return WUSH_ERR_INVALID_ARG;
+  if (fmt == WUSH_NVFP4 && !tensor_scale) return WUSH_ERR_INVALID_ARG;
+  if (debug && !y_out) return WUSH_ERR_INVALID_ARG;
+  if (!aligned(in, 16) || !aligned(T, 16) || !aligned(codes, 16)) return WUSH_ERR_MISALIGNED;
+  if (fmt == WUSH_INT4 && !aligned(scales, 4)) return WUSH_ERR_MISALIGNED;
+  if (tensor_scale && !aligned(tensor_scale, 4)) return WUSH_ERR_MISALIGNED;
+  if (debug && !aligned(y_out, 16)) return WUSH_ERR_MISALIGNED;
+
+  const int ch = in_f32 ? 64 : 128;   // channels per tile, as in FusedCfg
+  const long long n_row_tiles = (rows + 127) / 128;
+  const long long n_col_tiles = (d_in + ch - 1) / ch;
+  if (n_row_tiles * n_col_tiles > INT_MAX) return WUSH_ERR_INVALID_ARG;
+
+  CUtensorMap map;
+  int st = in_f32 ? encode_2d(&map, in, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, rows, d_in, 64,
+                              CU_TENSOR_MAP_SWIZZLE_NONE)
+                  : encode_2d(&map, in, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, d_in, 64,
+                              CU_TENSOR_MAP_SWIZZLE_128B);
+  if (st != WUSH_OK) return st;
+
+  wush::FusedParams p{};
+  p.T = T;
+  p.codes = codes;
+  p.scales = scales;
+  p.y_out = y_out;
+  p.amax_word = nullptr;
+  p.tensor_scale = nullptr;
+  p.n_rows = rows;
+  p.d_in = static_cast<int>(d_in);
+  p.C = static_cast<int>(d_in / G);
+  p.n_row_tiles = static_cast<int>(n_row_tiles);
+  p.total_tiles = static_cast<int>(n_row_tiles * n_col_tiles);
+  p.wait_limit_ns = g_wait_limit_ns.load(std::memory_order_relaxed);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  return in_f32 ? dispatch<true>(map, p, G, fmt, debug, tensor_scale, s)
+                : dispatch<false>(map, p, G, fmt, debug, tensor_scale, s);
+}
+
+}  // namespace
+
+extern "C" {
+
+int wush_quant_act(const void* x_bf16, const float* T_blocks, int64_t n_tok, int64_t d_in, int G, int fmt,
+                   uint8_t* codes, void* scales, float* tensor_scale, wush_stream_t stream) {
+  return quant_common(x_bf16, false, T_blocks, n_tok, d_in, G, fmt, codes, scales, tensor_scale, nullptr, false,
+                      stream);
+}
+
+int wush_quant_weight(const float* w_f32, const float* T_blocks, int64_t d_out, int64_t d_in, int G, int fmt,
+                      uint8_t* codes, void* scales, float* tensor_scale, wush_stream_t stream) {
+  return quant_common(w_f32, true, T_blocks, d_out, d_in, G, fmt, codes, scales, tensor_scale, nullptr, false,
+                      stream);
+}
+
+int wush_quant_act_debug(const void* x_bf16, const float* T_blocks, int64_t n_tok, int64_t d_in, int G, int fmt,
+                         uint8_t* codes, void* scales, float* tensor_scale, float* y_out, wush_stream_t stream) {
+  return quant_common(x_bf16, false, T_blocks, n_tok, d_in, G, fmt, codes, scales, tensor_scale, y_out, true,
+                      stream);
+}
+
+int wush_quant_weight_debug(const float* w_f32, const float* T_blocks, int64_t d_out, int64_t d_in, int G,
+                            int fmt, uint8_t* codes, void* scales, float* tensor_scale, float* y_out,
+                            wush_stream_t stream) {
+  return quant_common(w_f32, true, T_blocks, d_out, d_in, G, fmt, codes, scales, tensor_scale, y_out, true,
+                      stream);
+}
+
+int wush_build_transforms(const float* w_f32, const void* xcal_bf16, int64_t d_out, int64_t n_cal, int64_t d_in,
+                          int G, double lambda, int use_hadamard, float* T_wush, float* T_xvsh, double* T_wush64,
+                          double* T_xvsh64, double* s_out, wush_stream_t stream) {
+  if (G != 16 && G != 32) return WUSH_ERR_UNSUPPORTED;
+  if (d_out <= 0 || n_cal <= 0 || d_in <= 0 || d_in % G != 0 || d_in > INT_MAX) return WUSH_ERR_INVALID_ARG;
+  if (!(lambda >= 0.0) || lambda > 1e30) return WUSH_ERR_INVALID_ARG;
+  if (!w_f32 || !xcal_bf16 || !T_wush || !T_xvsh) return WUSH_ERR_INVALID_ARG;
+  if (!aligned(w_f32, 4) || !aligned(xcal_bf16, 2) || !aligned(T_wush, 4) || !aligned(T_xvsh, 4) ||
+      !aligned(T_wush64, 8) || !aligned(T_xvsh64, 8) || !aligned(s_out, 8))
+    return WUSH_ERR_MISALIGNED;
+  wush::BuildParams p{};
+  p.w = w_f32;
+  p.xcal = static_cast<const __nv_bfloat16*>(xcal_bf16);
+  p.d_out = d_out;
+  p.n_cal = n_cal;
+  p.d_in = static_cast<int>(d_in);
+  p.C = static_cast<int>(d_in / G);
+  p.lambda = lambda;
+  p.use_hadamard = use_hadamard ? 1 : 0;
+  p.T_wush = T_wush;
+  p.T_xvsh = T_xvsh;
+  p.T_wush64 = T_wush64;
+  p.T_xvsh64 = T_xvsh64;
+  p.s_out = s_out;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (G == 32) {
+    constexpr int bytes = wush::BuildSmem<32>::BYTES;
+    if (cudaFuncSetAttribute(wush::wush_build_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) !=
+        cudaSuccess)
+      return WUSH_ERR_CUDA;
+    wush::wush_build_kernel<32><<<p.C, wush::kBuildThreads, bytes, s>>>(p);
+  } else {
+    constexpr int bytes = wush::BuildSmem<16>::BYTES;
+    if (cudaFuncSetAttribute(wush::wush_build_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) !=
+        cudaSuccess)
+      return WUSH_ERR_CUDA;
+    wush::wush_build_kernel<16><<<p.C, wush::kBuildThreads, bytes, s>>>(p);
+  }
+  return cudaGetLastError() == cudaSuccess ? WUSH_OK : WUSH_ERR_CUDA;
+}
+
+int wush_device_status(wush_stream_t stream, uint32_t* bits) {
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return WUSH_ERR_CUDA;
+  unsigned int word = 0u, zero = 0u;
+  if (cudaMemcpyFromSymbol(&word, wush::g_wush_device_error, sizeof(word)) != cudaSuccess) return WUSH_ERR_CUDA;
+  if (word && cudaMemcpyToSymbol(wush::g_wush_device_error, &zero, sizeof(zero)) != cudaSuccess)
+    return WUSH_ERR_CUDA;
+  if (bits) *bits = word;
+  return word ? WUSH_ERR_DEVICE_TIMEOUT : WUSH_OK;
+}
+
+int wush_set_wait_limit_ns(uint64_t ns) {
+  g_wait_limit_ns.store(ns ? ns : kDefaultWaitLimitNs, std::memory_order_relaxed);
+  return WUSH_OK;
+}
+
+int wush_selftest_wait_timeout(uint64_t limit_ns, wush_stream_t stream, uint32_t* bits) {
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  wush::wush_selftest_wait_kernel<<<1, 32, 0, s>>>(limit_ns);
+  if (cudaGetLastError() != cudaSuccess) return WUSH_ERR_CUDA;
+  uint32_t word = 0;
+  const int st = wush_device_status(stream, &word);
+  if (bits) *bits = word;
+  return st;
+}
+
+const char* wush_status_string(int status) {
+  switch (status) {
+    case WUSH_OK: return "WUSH_OK";
+    case WUSH_ERR_INVALID_ARG: return "WUSH_ERR_INVALID_ARG: null pointer or bad size";
+    case WUSH_ERR_UNSUPPORTED: return "WUSH_ERR_UNSUPPORTED: format or group size not supported";
+    case WUSH_ERR_MISALIGNED: return "WUSH_ERR_MISALIGNED: pointer alignment requirement not met";
+    case WUSH_ERR_CUDA: return "WUSH_ERR_CUDA: CUDA runtime error";
+    case WUSH_ERR_DEVICE_TIMEOUT: return "WUSH_ERR_DEVICE_TIMEOUT: an in-kernel wait expired";
+    default: return "unknown wush status";
+  }
+}
+
+int wush_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,163 @@
+/*
+ * wush.h - C ABI of the B200 (sm_100a) fused WUSH transform + 4-bit quantisation library.
+ *
+ * What the library computes.  Sources are pages describing arXiv 2512.00956, "WUSH:
+ * Near-Optimal Adaptive Transforms for LLM Quantization":
+ *   - paper-graph-ui analysis, section 3.2 "Big-Picture Architecture": the "Online
+ *     Activation Transform + Quantize Kernel" multiplies each incoming activation block
+ *     by its own T_wush,i and quantises it on the fly; the "Weight Pre-Quantizer"
+ *     applies the weight-side transform to the weight block and quantises it with RTN.
+ *   - same page, section 3.4.7 "GPU Kernel Design": tokens x d_in activations; C = d_in/G
+ *     independent (M x G) x (G x G) products, one G x G matrix per block.
+ *   - same page, section 3.4.1: block size G = quantisation group size (32 for MXFP4,
+ *     16 for NVFP4); G is a power of two dividing d_in.
+ *   - ai.info summary, authors' abstract: "RTN AbsMax-scaled block quantizers".
+ *   - papernotes.org summary, section "整体框架": activations use T_wush, weights use
+ *     T_xvsh = T_wush^-T.
+ *
+ * Layouts (all row-major, no padding):
+ *   x          bf16  [n_tok][d_in]            activations, one row per token
+ *   w          fp32  [d_out][d_in]            weights, one row per output channel
+ *   T_blocks   fp32  [C][G][G]                element (i, r, c) at (i*G + r)*G + c is
+ *                                             (T_i)_{r,c}; y_r = sum_c (T_i)_{r,c} x_c
+ *   codes      u8    [rows][d_in/2]           4-bit codes, byte j holds element 2j in the
+ *                                             low nibble and element 2j+1 in the high one
+ *   scales     MXFP4: u8 [rows][C]            E8M0 byte e + 127, group value = code * 2^e
+ *              NVFP4: u8 [rows][C]            E4M3 block scale, value = code * dec * s_t
+ *              INT4 : fp32 [rows][C]          value = signed nibble * scale
+ *   tensor_scale fp32 [1]                     NVFP4 only: s_t = amax|y| / (6 * 448)
+ * with rows = n_tok (activations) or d_out (weights).
+ *
+ * Codes.  E2M1 (MXFP4, NVFP4): bit 3 is the sign, bits 0-2 index the grid
+ * {0, 0.5, 1, 1.5, 2, 3, 4, 6}; rounding is to nearest with ties to the even code and
+ * saturation at 6; 0x0 and 0x8 both encode zero.  INT4: two's-complement nibble in
+ * [-7, 7], round to nearest even.  Scale rules:
+ *   MXFP4  e = least integer with amax <= 6 * 2^e, clamped to [-127, 127]
+ *   NVFP4  sb = E4M3(amax / (6 s_t)); y is multiplied by the fp32 reciprocal of dec(sb)*s_t
+ *   INT4   s = amax / 7; y is multiplied by the fp32 reciprocal of s
+ * A group whose scale reciprocal is not a finite fp32 encodes as all zero.
+ *
+ * Supported (fmt, G): (MXFP4, 32), (NVFP4, 16), (INT4, 16), (INT4, 32).
+ *
+ * Ownership and execution.  Every pointer argument of the quantisation calls is
+ * caller-owned DEVICE memory on the current CUDA device.  Calls are asynchronous on
+ * `stream` (0 = legacy default stream), never synchronise the host, allocate nothing
+ * and keep no state between calls except the device error word described at
+ * wush_device_status().  Inputs must be finite; NaN or Inf gives unspecified codes.
+ *
+ * Errors.  Arguments are checked on the host before any launch:
+ *   WUSH_ERR_INVALID_ARG   NULL pointer, n_tok/d_out < 0, d_in <= 0, d_in % G != 0,
+ *                          a size beyond 2^31 - 1 rows or 2^31 - 1 channels
+ *   WUSH_ERR_UNSUPPORTED   unknown fmt or an unsupported (fmt, G) pair
+ *   WUSH_ERR_MISALIGNED    x, w, T_blocks, codes, y_out not 16-byte aligned; INT4 scales
+ *                          or tensor_scale not 4-byte aligned
+ *   WUSH_ERR_CUDA          a CUDA runtime error while launching (including a missing or
+ *                          non-sm_100 device)
+ * Bits of the device error word (wush_device_status): 1/2/4/8/16 a wait of the TMA
+ * producer / MMA issuer / converter / epilogue / final drain expired, 32 the wait
+ * self-test expired (expected), 64 a Cholesky pivot was not positive.
+ * rows == 0 (with a supported fmt/G and a valid d_in) returns WUSH_OK without launching
+ * anything; its pointers are then not checked and may be NULL.
+ */
+#ifndef WUSH_H_
+#define WUSH_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same object as cudaStream_t / CUstream. */
+typedef struct CUstream_st* wush_stream_t;
+
+typedef enum { WUSH_MXFP4 = 0, WUSH_NVFP4 = 1, WUSH_INT4 = 2 } wush_fmt;
+
+typedef enum {
+  WUSH_OK = 0,
+  WUSH_ERR_INVALID_ARG = 1,
+  WUSH_ERR_UNSUPPORTED = 2,
+  WUSH_ERR_MISALIGNED = 3,
+  WUSH_ERR_CUDA = 4,
+  WUSH_ERR_DEVICE_TIMEOUT = 5
+} wush_status;
+
+/* Online activation path: y = T_wush,i x per token and block, then AbsMax quantise.
+ * For NVFP4 the call makes two passes over x (the first finds amax|y| for s_t) and
+ * writes s_t to *tensor_scale, which also serves as the running-max word of the first
+ * pass; tensor_scale may be NULL for the other formats. */
+int wush_quant_act(const void* x_bf16, const float* T_blocks, int64_t n_tok, int64_t d_in, int G,
+                   int fmt, uint8_t* codes, void* scales, float* tensor_scale, wush_stream_t stream);
+
+/* Weight pre-quantisation: W_bar = T_xvsh,i w per output channel and block, then AbsMax
+ * quantise; w is fp32 [d_out][d_in].  Same outputs and rules as wush_quant_act. */
+int wush_quant_weight(const float* w_f32, const float* T_blocks, int64_t d_out, int64_t d_in, int G,
+                      int fmt, uint8_t* codes, void* scales, float* tensor_scale,
+                      wush_stream_t stream);
+
+/* Test variants: identical kernels that additionally write the fp32 transformed values
+ * y [rows][d_in] they quantised (device memory, 16-byte aligned), so that the
+ * quantiser can be checked bit for bit against an independent implementation fed the
+ * same y. */
+int wush_quant_act_debug(const void* x_bf16, const float* T_blocks, int64_t n_tok, int64_t d_in,
+                         int G, int fmt, uint8_t* codes, void* scales, float* tensor_scale,
+                         float* y_out, wush_stream_t stream);
+int wush_quant_weight_debug(const float* w_f32, const float* T_blocks, int64_t d_out, int64_t d_in,
+                            int G, int fmt, uint8_t* codes, void* scales, float* tensor_scale,
+                            float* y_out, wush_stream_t stream);
+
+/* Transform construction for one layer, on the device, in fp64 (one CTA per block).
+ * Sources: paper-graph-ui analysis, section 3.2 "Second-Moment Computer" and "Transform
+ * Constructor", sections 3.4.2 and 3.4.4 (Eq. 8); papernotes.org summary, "关键设计";
+ * ai.info summary, "Methodology in Plain English" (damping of the diagonals).
+ *   Sigma_w = d_out^-1 W_(i) W_(i)^T, Sigma_x = n_cal^-1 X_(i) X_(i)^T          per block i
+ *   Sigma  += lambda * mean(diag Sigma) * I                                   (both sides)
+ *   W' = chol(Sigma_w), X' = chol(Sigma_x)  (lower);  W'^T X' = U S V^T
+ *   T_wush = H S^-1/2 U^T W'^T,  T_xvsh = H S^-1/2 V^T X'^T = T_wush^-T
+ * H is the normalised Sylvester Hadamard matrix (use_hadamard = 0 replaces it by I).
+ * Singular values are sorted descending; each pair (u_k, v_k) is flipped so that the
+ * largest-magnitude entry of u_k is positive.
+ * Inputs (device): w_f32 [d_out][d_in], xcal_bf16 [n_cal][d_in] calibration activations.
+ * Outputs (device): T_wush, T_xvsh fp32 [C][G][G] (the fp64 results rounded once);
+ * optional (may be NULL) T_wush64, T_xvsh64 fp64 [C][G][G] and s_out fp64 [C][G].
+ * G in {16, 32}.  A Cholesky pivot at or below 1e-12 of the mean (damped) diagonal
+ * (e.g. lambda = 0 on rank-deficient data) sets bit 64 of the device error word (see
+ * wush_device_status) and yields unusable T.
+ * Errors: WUSH_ERR_UNSUPPORTED (G), WUSH_ERR_INVALID_ARG (NULL input/output, sizes,
+ * lambda < 0 or not finite), WUSH_ERR_MISALIGNED (fp32 pointers not 4-byte, bf16 not
+ * 2-byte, fp64 not 8-byte aligned), WUSH_ERR_CUDA.  Asynchronous on `stream`, allocates
+ * nothing. */
+int wush_build_transforms(const float* w_f32, const void* xcal_bf16, int64_t d_out, int64_t n_cal,
+                          int64_t d_in, int G, double lambda, int use_hadamard, float* T_wush,
+                          float* T_xvsh, double* T_wush64, double* T_xvsh64, double* s_out,
+                          wush_stream_t stream);
+
+/* Every wait inside the kernels is bounded in time (default 2 s).  When one expires
+ * the kernel records a bit in a per-device error word and returns early; outputs of
+ * that call are then unspecified.  wush_device_status() synchronises `stream`, reads
+ * and clears the word of the current device and returns WUSH_OK or
+ * WUSH_ERR_DEVICE_TIMEOUT (WUSH_ERR_CUDA if the runtime reports an error).  If
+ * `bits` is not NULL it receives the raw word. */
+int wush_device_status(wush_stream_t stream, uint32_t* bits);
+
+/* Sets the bound of every in-kernel wait for later launches, in nanoseconds
+ * (0 restores the default of 2 s).  Returns WUSH_OK. */
+int wush_set_wait_limit_ns(uint64_t ns);
+
+/* Self-test of the bounded-wait path: launches one CTA that waits on an mbarrier no
+ * thread ever arrives on, with a limit of `limit_ns`; the wait must give up, record
+ * its bit and return.  Synchronises `stream` and returns the error word it produced
+ * (expected: 32).  Does not fault or hang the device. */
+int wush_selftest_wait_timeout(uint64_t limit_ns, wush_stream_t stream, uint32_t* bits);
+
+/* Human-readable name of a wush_status value (static string, never NULL). */
+const char* wush_status_string(int status);
+
+/* Library ABI version (major * 10000 + minor * 100 + patch). */
+int wush_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* WUSH_H_ */

@@ -37,6 +37,8 @@ design notes of the repository):
       stored as a two's-complement nibble with an fp32 scale.  ([graph] §3.4.5 writes
       the scale as 2^(1-b) * amax, i.e. amax / 8, which would need the code +8.)
   R8  Packing: byte j holds element 2j in its low nibble and 2j+1 in its high nibble.
+  R9  A group whose scale reciprocal fl32(1/S) is not a finite float32 (S = 0, or S so
+      small that 1/S overflows) encodes as all zero codes (the pages are silent).
 fl32(.) marks a float32 rounding point: the oracle computes in float64 and rounds
 to float32 there, which equals the IEEE float32 result of a single +, -, *, /.
 """
@@ -303,6 +305,16 @@ def quant_mxfp4(y: np.ndarray, rule: str = "absmax"):
     return codes, (e + 127).astype(np.uint8)
 
 
+def _recip32(S: np.ndarray) -> np.ndarray:
+    """fl32(1 / S) for S > 0; 0 where S is 0 or where the float32 reciprocal overflows
+    (reading R9: such a group encodes as all zero)."""
+    S = np.asarray(S, dtype=np.float64)
+    with np.errstate(divide="ignore", over="ignore"):
+        inv = np.where(S > 0, np.float32(1.0) / np.where(S > 0, S, 1.0).astype(np.float32), 0.0)
+    inv = np.asarray(inv, dtype=np.float64)
+    return np.where(np.isfinite(inv), inv, 0.0)
+
+
 def nvfp4_tensor_scale(amax_tensor: float) -> float:
     """Reading R6: s_t = fl32(amax_tensor / 2688), 2688 = 6 * 448."""
     return float(fl32(np.float64(amax_tensor) / 2688.0))
@@ -320,8 +332,7 @@ def quant_nvfp4(y: np.ndarray, s_t: float | None = None):
         r = np.where(d6 > 0, fl32(amax / d6), 0.0)
     sb = e4m3_encode(r)
     S = fl32(e4m3_decode(sb) * s_t)
-    with np.errstate(divide="ignore"):
-        inv = np.where(S > 0, fl32(1.0 / np.where(S > 0, S, 1.0)), 0.0)
+    inv = _recip32(S)
     v = fl32(g * inv[:, :, None])
     codes = e2m1_encode(v).reshape(y.shape)
     return codes, sb, s_t
@@ -332,7 +343,7 @@ def quant_int4(y: np.ndarray, G: int):
     g = _groups(y, G)
     amax = np.max(np.abs(g), axis=2)
     s = fl32(amax / 7.0)
-    inv = np.where(s > 0, fl32(1.0 / np.where(s > 0, s, 1.0)), 0.0)
+    inv = _recip32(s)
     v = fl32(g * inv[:, :, None])
     q = np.clip(np.rint(v), -7, 7).astype(np.int64)
     codes = (q & 0xF).astype(np.uint8).reshape(y.shape)

@@ -1,0 +1,141 @@
+"""The C ABI boundary without a GPU: the library loads, exports every symbol that
+include/wush.h declares, and rejects bad arguments on the host before any launch."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import blockwise_adaptive_transforms_b200 as W
+from blockwise_adaptive_transforms_b200 import _build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "wush.h")
+
+OK, INVALID, UNSUPPORTED, MISALIGNED = 0, 1, 2, 3
+
+
+@pytest.fixture(scope="module")
+def lib():
+    _build.build()
+    return W.load_library()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(wush_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_documented_entry_points():
+    names = declared_functions()
+    for required in ("wush_quant_act", "wush_quant_weight", "wush_status_string"):
+        assert required in names
+    assert set(names) == set(W.EXPORTED_SYMBOLS)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+    # and they are C symbols (no C++ mangling)
+    nm = os.popen(f"nm -D --defined-only {W.LIB_PATH}").read()
+    for name in declared_functions():
+        assert re.search(rf"\bT {name}$", nm, re.M), name
+
+
+def test_status_strings_and_version(lib):
+    assert W.wush_status_string(0) == "WUSH_OK"
+    for s in range(1, 6):
+        assert W.wush_status_string(s).startswith(W.STATUS[s])
+    assert "unknown" in W.wush_status_string(99)
+    assert W.wush_version() == 100
+
+
+# fake, never-dereferenced addresses: every call below returns before touching CUDA
+A16 = 0x10000
+A4 = 0x20004
+A1 = 0x30001
+
+
+def call_act(lib, x=A16, T=A16, n=128, d=256, G=32, fmt=0, codes=A16, scales=A16, ts=None):
+    return lib.wush_quant_act(x, T, n, d, G, fmt, codes, scales, ts, None)
+
+
+def test_null_pointers_rejected(lib):
+    assert call_act(lib, x=None) == INVALID
+    assert call_act(lib, T=None) == INVALID
+    assert call_act(lib, codes=None) == INVALID
+    assert call_act(lib, scales=None) == INVALID
+    assert call_act(lib, fmt=1, G=16, ts=None) == INVALID            # NVFP4 needs tensor_scale
+    assert lib.wush_quant_weight(None, A16, 8, 64, 32, 0, A16, A16, None, None) == INVALID
+    assert lib.wush_quant_act_debug(A16, A16, 8, 64, 32, 0, A16, A16, None, None, None) == INVALID
+
+
+def test_sizes_rejected(lib):
+    assert call_act(lib, n=-1) == INVALID
+    assert call_act(lib, d=0) == INVALID
+    assert call_act(lib, d=-32) == INVALID
+    assert call_act(lib, d=48) == INVALID                # not a multiple of G = 32
+    assert call_act(lib, d=40, G=16, fmt=2) == INVALID
+    assert call_act(lib, n=2 ** 31) == INVALID
+    assert call_act(lib, d=2 ** 31 + 32) == INVALID
+
+
+def test_unsupported_format_and_group(lib):
+    assert call_act(lib, fmt=3) == UNSUPPORTED
+    assert call_act(lib, fmt=-1) == UNSUPPORTED
+    assert call_act(lib, fmt=0, G=16) == UNSUPPORTED     # MXFP4 groups are 32
+    assert call_act(lib, fmt=1, G=32, ts=A16) == UNSUPPORTED  # NVFP4 groups are 16
+    assert call_act(lib, fmt=2, G=64) == UNSUPPORTED
+    assert call_act(lib, fmt=2, G=8) == UNSUPPORTED
+
+
+def test_misaligned_pointers(lib):
+    assert call_act(lib, x=A16 + 2) == MISALIGNED
+    assert call_act(lib, T=A4) == MISALIGNED
+    assert call_act(lib, codes=A16 + 8) == MISALIGNED
+    assert call_act(lib, fmt=2, scales=A1) == MISALIGNED       # INT4 scales are fp32
+    assert call_act(lib, fmt=0, scales=A1, n=0) == OK          # byte scales need no alignment
+    assert call_act(lib, fmt=1, G=16, ts=A1) == MISALIGNED
+    assert lib.wush_quant_act_debug(A16, A16, 8, 64, 32, 0, A16, A16, None, A4, None) == MISALIGNED
+
+
+def test_empty_batch_is_ok_without_launch(lib):
+    assert call_act(lib, n=0) == OK
+    assert call_act(lib, n=0, x=None, codes=None, scales=None) == OK   # empty tensors have no storage
+    assert call_act(lib, n=0, fmt=0, G=16) == UNSUPPORTED
+    assert lib.wush_quant_weight(A16, A16, 0, 64, 32, 0, A16, A16, None, None) == OK
+    assert call_act(lib, n=0, fmt=1, G=16, ts=A16) == OK
+
+
+def test_wait_limit_setter(lib):
+    assert lib.wush_set_wait_limit_ns(0) == OK
+    assert lib.wush_set_wait_limit_ns(5_000_000_000) == OK
+    assert lib.wush_set_wait_limit_ns(0) == OK
+
+
+def test_python_binding_refuses_cpu_tensors():
+    import torch
+    x = torch.zeros(4, 64, dtype=torch.bfloat16)
+    T = torch.zeros(2, 32, 32)
+    with pytest.raises(TypeError):
+        W.wush_quant_act(x, T, 32, "mxfp4")
+
+
+def test_build_flags_target_sm100a_only():
+    assert _build.ARCH_FLAGS == ["-gencode", "arch=compute_100a,code=sm_100a"]
+
+
+def test_builder_argument_checks(lib):
+    b = lib.wush_build_transforms
+    assert b(A16, A16, 64, 64, 256, 8, 0.01, 1, A16, A16, None, None, None, None) == UNSUPPORTED
+    assert b(A16, A16, 0, 64, 256, 32, 0.01, 1, A16, A16, None, None, None, None) == INVALID
+    assert b(A16, A16, 64, 0, 256, 32, 0.01, 1, A16, A16, None, None, None, None) == INVALID
+    assert b(A16, A16, 64, 64, 250, 32, 0.01, 1, A16, A16, None, None, None, None) == INVALID
+    assert b(A16, A16, 64, 64, 256, 32, -1.0, 1, A16, A16, None, None, None, None) == INVALID
+    assert b(A16, A16, 64, 64, 256, 32, float("nan"), 1, A16, A16, None, None, None, None) == INVALID
+    assert b(None, A16, 64, 64, 256, 32, 0.01, 1, A16, A16, None, None, None, None) == INVALID
+    assert b(A16, A16, 64, 64, 256, 32, 0.01, 1, None, A16, None, None, None, None) == INVALID
+    assert b(A16 + 2, A16, 64, 64, 256, 32, 0.01, 1, A16, A16, None, None, None, None) == MISALIGNED
+    assert b(A16, A1, 64, 64, 256, 32, 0.01, 1, A16, A16, None, None, None, None) == MISALIGNED
+    assert b(A16, A16, 64, 64, 256, 32, 0.01, 1, A16, A16, A4, None, None, None) == MISALIGNED
