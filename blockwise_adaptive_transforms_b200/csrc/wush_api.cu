@@ -63,7 +63,7 @@ int encode_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dt, int el
 }
 
 template <class Cfg>
-int launch_fused(const CUtensorMap& map, wush::FusedParams p, cudaStream_t stream) {
+int launch_fused(const CUtensorMap& map, const CUtensorMap& cmap, wush::FusedParams p, cudaStream_t stream) {
   int dev = 0, sms = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return WUSH_ERR_CUDA;
   if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return WUSH_ERR_CUDA;
@@ -76,35 +76,37 @@ int launch_fused(const CUtensorMap& map, wush::FusedParams p, cudaStream_t strea
     configured.fetch_or(bit, std::memory_order_acq_rel);
   }
   const int grid = p.total_tiles < sms ? p.total_tiles : sms;
-  wush::wush_fused_kernel<Cfg><<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(map, p);
+  wush::wush_fused_kernel<Cfg><<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(map, cmap, p);
   return cudaGetLastError() == cudaSuccess ? WUSH_OK : WUSH_ERR_CUDA;
 }
 
 template <int G, int FMT, bool IN_F32, bool AMAX_ONLY>
-int launch_pick_y(const CUtensorMap& map, const wush::FusedParams& p, bool emit_y, cudaStream_t s) {
-  if (emit_y) return launch_fused<wush::FusedCfg<G, FMT, IN_F32, AMAX_ONLY, true>>(map, p, s);
-  return launch_fused<wush::FusedCfg<G, FMT, IN_F32, AMAX_ONLY, false>>(map, p, s);
+int launch_pick_y(const CUtensorMap& map, const CUtensorMap& cmap, const wush::FusedParams& p, bool emit_y,
+                  cudaStream_t s) {
+  if (emit_y) return launch_fused<wush::FusedCfg<G, FMT, IN_F32, AMAX_ONLY, true>>(map, cmap, p, s);
+  return launch_fused<wush::FusedCfg<G, FMT, IN_F32, AMAX_ONLY, false>>(map, cmap, p, s);
 }
 
 template <bool IN_F32>
-int dispatch(const CUtensorMap& map, wush::FusedParams p, int G, int fmt, bool emit_y, float* tensor_scale,
-             cudaStream_t s) {
-  if (fmt == WUSH_MXFP4) return launch_pick_y<32, wush::kMXFP4, IN_F32, false>(map, p, emit_y, s);
+int dispatch(const CUtensorMap& map, const CUtensorMap& cmap, wush::FusedParams p, int G, int fmt, bool emit_y,
+             float* tensor_scale, cudaStream_t s) {
+  if (fmt == WUSH_MXFP4) return launch_pick_y<32, wush::kMXFP4, IN_F32, false>(map, cmap, p, emit_y, s);
   if (fmt == WUSH_INT4) {
-    if (G == 32) return launch_pick_y<32, wush::kINT4, IN_F32, false>(map, p, emit_y, s);
-    return launch_pick_y<16, wush::kINT4, IN_F32, false>(map, p, emit_y, s);
+    if (G == 32) return launch_pick_y<32, wush::kINT4, IN_F32, false>(map, cmap, p, emit_y, s);
+    return launch_pick_y<16, wush::kINT4, IN_F32, false>(map, cmap, p, emit_y, s);
   }
   // NVFP4: pass 1 finds amax|y| (float bits, running max in *tensor_scale), a one-thread
   // kernel turns it into s_t in place, pass 2 quantises with s_t.
   if (cudaMemsetAsync(tensor_scale, 0, sizeof(float), s) != cudaSuccess) return WUSH_ERR_CUDA;
-  p.amax_word = reinterpret_cast<unsigned int*>(tensor_scale);
-  int st = launch_fused<wush::FusedCfg<16, wush::kNVFP4, IN_F32, true, false>>(map, p, s);
+  wush::FusedParams p1 = p;
+  p1.amax_word = reinterpret_cast<unsigned int*>(tensor_scale);
+  p1.codes_via_tma = 0;
+  int st = launch_fused<wush::FusedCfg<16, wush::kNVFP4, IN_F32, true, false>>(map, cmap, p1, s);
   if (st != WUSH_OK) return st;
   wush::wush_nvfp4_tensor_scale_kernel<<<1, 32, 0, s>>>(tensor_scale);
   if (cudaGetLastError() != cudaSuccess) return WUSH_ERR_CUDA;
-  p.amax_word = nullptr;
   p.tensor_scale = tensor_scale;
-  return launch_pick_y<16, wush::kNVFP4, IN_F32, false>(map, p, emit_y, s);
+  return launch_pick_y<16, wush::kNVFP4, IN_F32, false>(map, cmap, p, emit_y, s);
 }
 
 int quant_common(const void* in, bool in_f32, const float* T, int64_t rows, int64_t d_in, int G, int fmt,
@@ -136,8 +138,19 @@ int quant_common(const void* in, bool in_f32, const float* T, int64_t rows, int6
                   : encode_2d(&map, in, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, d_in, 64,
                               CU_TENSOR_MAP_SWIZZLE_128B);
   if (st != WUSH_OK) return st;
+  // codes leave through a TMA store when the row pitch allows it (a multiple of 16 bytes);
+  // the store map's swizzle matches the kernel's staging layout (64-byte rows: 64B
+  // swizzle, 32-byte rows: 32B swizzle)
+  CUtensorMap cmap = map;
+  const bool codes_tma = ((d_in / 2) % 16) == 0;
+  if (codes_tma) {
+    st = encode_2d(&cmap, codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, rows, d_in / 2, ch / 2,
+                   in_f32 ? CU_TENSOR_MAP_SWIZZLE_32B : CU_TENSOR_MAP_SWIZZLE_64B);
+    if (st != WUSH_OK) return st;
+  }
 
   wush::FusedParams p{};
+  p.codes_via_tma = codes_tma ? 1 : 0;
   p.T = T;
   p.codes = codes;
   p.scales = scales;
@@ -151,8 +164,8 @@ int quant_common(const void* in, bool in_f32, const float* T, int64_t rows, int6
   p.total_tiles = static_cast<int>(n_row_tiles * n_col_tiles);
   p.wait_limit_ns = g_wait_limit_ns.load(std::memory_order_relaxed);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  return in_f32 ? dispatch<true>(map, p, G, fmt, debug, tensor_scale, s)
-                : dispatch<false>(map, p, G, fmt, debug, tensor_scale, s);
+  return in_f32 ? dispatch<true>(map, cmap, p, G, fmt, debug, tensor_scale, s)
+                : dispatch<false>(map, cmap, p, G, fmt, debug, tensor_scale, s);
 }
 
 }  // namespace

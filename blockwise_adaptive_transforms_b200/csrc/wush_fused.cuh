@@ -10,14 +10,19 @@
 //  * persistent CTAs, one per SM, each owning a contiguous run of 128-row x CH-channel
 //    tiles, column-tile major so consecutive tiles share their transforms;
 //  * warp 0 streams the input tiles with TMA (128-byte swizzle) through a STAGES-deep
-//    mbarrier ring; warps 2-5 split each fp32 T_i into bf16 hi + lo panels in shared
-//    memory (and, for fp32 weights, split the weight tile into bf16 hi + lo operands);
-//  * warp 1 issues tcgen05.mma (M=128, N=G, K=16) with fp32 accumulators in TMEM:
-//    X*T_hi^T + X*T_lo^T for bf16 activations, W_hi*T_hi^T + W_hi*T_lo^T + W_lo*T_hi^T
-//    for fp32 weights, double-buffered in TMEM;
-//  * warps 6-13 read the accumulators with tcgen05.ld (one token row per thread, a
-//    whole group in registers), compute the AbsMax scale, round and pack, and store
-//    16-byte vectors directly to global memory.
+//    mbarrier ring; warps 2-3 split each fp32 T_i into bf16 hi and lo and stack them
+//    along N in shared memory (for fp32 weights they also split each staged weight
+//    tile into bf16 hi + lo operands);
+//  * warp 1 issues tcgen05.mma (M=128, N=2G, K=16) into fp32 TMEM accumulators,
+//    double-buffered: one MMA per block and K-step yields X*T_hi^T and X*T_lo^T side
+//    by side (fp32 weights add W_lo*T_hi^T into the first half; the dropped W_lo*T_lo
+//    term is below 2^-16 relative).  Each tcgen05.mma costs the issuing thread ~50
+//    cycles whatever N is, so stacking hi|lo halves the issue work of the tile;
+//  * warps 4-11 read the accumulators with tcgen05.ld (one token row per thread),
+//    add the hi and lo halves, compute the AbsMax scale, round and pack, stage the
+//    tile's codes in shared memory for one TMA store and write one scale word per row.
+//  * every wait is an mbarrier try_wait with a suspend-time hint, so waiting warps do
+//    not take issue slots from the working ones.
 #pragma once
 #include <cstdint>
 #include <cuda_bf16.h>
@@ -39,6 +44,7 @@ struct FusedParams {
   int C;
   int n_row_tiles;
   int total_tiles;
+  int codes_via_tma;        // 1: codes leave through the TMA store map (needs d_in % 32 == 0)
   unsigned long long wait_limit_ns;
 };
 
@@ -56,26 +62,35 @@ struct FusedCfg {
   static constexpr int STAGES = IN_F32 ? 3 : 5;
   static constexpr int STAGE_BYTES = IN_F32 ? BM * CH * 4 : BM * CH * 2;  // 32 KiB
   static constexpr int OPER_BYTES = BM * CH * 2;       // one bf16 operand tile (hi or lo)
-  static constexpr int BLK_PER_PANEL = 32 / G;         // blocks whose hi|lo rows share a 128 B row
-  static constexpr int PANEL_BYTES = G * 128;
-  static constexpr int N_PANELS = BPT / BLK_PER_PANEL;
+  // transform panels: 2G rows (hi rows then lo rows) x 128 bytes of K; a 128-byte row
+  // holds the K = G values of BPP = 64/G blocks side by side
+  static constexpr int BPP = 64 / G;
+  static constexpr int PANEL_BYTES = 2 * G * 128;
+  static constexpr int N_PANELS = BPT / BPP;
   static constexpr int TSLOT_BYTES = N_PANELS * PANEL_BYTES;
-  static constexpr int TMEM_COLS = 2 * CH;             // two accumulator buffers
-  static constexpr int N_EPI_WARPS = 8;
+  static constexpr int ACC_COLS = 2 * CH;              // hi|lo of every block of a tile
+  static constexpr int TMEM_COLS = 2 * ACC_COLS;       // two accumulator buffers
   static constexpr int BPW = BPT / 2;                  // blocks per epilogue warp
-  static constexpr int THREADS = 14 * 32;
+  static constexpr int N_EPI_WARPS = 8;
+  static constexpr int THREADS = 12 * 32;
+  static constexpr int CODE_STAGE = 128 * CH / 2;      // one tile of packed codes
+  static constexpr int SCALE_STAGE = 128 * BPT * (FMT == kINT4 ? 4 : 1);
   // shared memory carve-up (offsets from a 1024-byte aligned base)
   static constexpr int OFF_STAGE = 0;
   static constexpr int OFF_OPER = OFF_STAGE + STAGES * STAGE_BYTES;
   static constexpr int OFF_T = OFF_OPER + (IN_F32 ? 2 * 2 * OPER_BYTES : 0);
-  static constexpr int OFF_BAR = OFF_T + 2 * TSLOT_BYTES;
+  static constexpr int OFF_CODES = OFF_T + 2 * TSLOT_BYTES;
+  static constexpr int OFF_SCALES = OFF_CODES + 2 * CODE_STAGE;
+  static constexpr int OFF_BAR = OFF_SCALES + 2 * SCALE_STAGE;
   // barriers: full[S], empty[S], ofull[2], oempty[2], tfull[2], tempty[2], afull[2], aempty[2], drain
   static constexpr int N_BARS = 2 * STAGES + 13;
   static constexpr int OFF_MISC = OFF_BAR + 8 * N_BARS;
   static constexpr int SMEM_BYTES = OFF_MISC + 64 + 1024;   // + alignment slack
   static_assert(G == 16 || G == 32, "G must be 16 or 32");
   static_assert(!(FMT == kMXFP4 && G != 32) && !(FMT == kNVFP4 && G != 16), "format/group mismatch");
+  static_assert(TMEM_COLS <= 512, "TMEM columns");
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+  static_assert(OFF_CODES % 1024 == 0 && CODE_STAGE % 1024 == 0, "swizzled staging alignment");
 };
 
 // byte offset of logical 16-byte chunk `chunk` of row `row` in a 128-byte-swizzled tile
@@ -103,6 +118,19 @@ __device__ __forceinline__ void split8(const float* v, uint4& hi, uint4& lo) {
   lo = make_uint4(l[0], l[1], l[2], l[3]);
 }
 
+// Largest |v_j| of a group, as a balanced tree (max is exact, so the order is free).
+template <int NV>
+__device__ __forceinline__ float group_absmax(const float* v) {
+  float m[NV / 2];
+#pragma unroll
+  for (int j = 0; j < NV / 2; ++j) m[j] = fmaxf(fabsf(v[2 * j]), fabsf(v[2 * j + 1]));
+#pragma unroll
+  for (int w = NV / 4; w >= 1; w >>= 1)
+#pragma unroll
+    for (int j = 0; j < w; ++j) m[j] = fmaxf(m[j], m[j + w]);
+  return m[0];
+}
+
 // ---------------------------------------------------------------- group quantisers
 // Each consumes the G transformed values of one (row, block) group held in registers
 // and produces G/8 packed code words plus the group's scale.
@@ -112,9 +140,7 @@ __device__ __forceinline__ void split8(const float* v, uint4& hi, uint4& lo) {
 // e = E - 2 when m <= 1.5 and E - 1 otherwise, read off the float's bits.
 template <int NV>
 __device__ __forceinline__ uint32_t quant_mx(const float* v, uint32_t* words) {
-  float amax = 0.0f;
-#pragma unroll
-  for (int j = 0; j < NV; ++j) amax = fmaxf(amax, fabsf(v[j]));
+  const float amax = group_absmax<NV>(v);
   const uint32_t ab = __float_as_uint(amax);
   int sb = static_cast<int>(ab >> 23) - 2 + ((ab & 0x7FFFFFu) > 0x400000u ? 1 : 0);
   sb = max(sb, 0);
@@ -132,9 +158,7 @@ __device__ __forceinline__ uint32_t quant_mx(const float* v, uint32_t* words) {
 // codes = E2M1(y * (1/S)); every step rounded to fp32 (IEEE division / reciprocal).
 template <int NV>
 __device__ __forceinline__ uint32_t quant_nv(const float* v, float s_t, float d6, uint32_t* words) {
-  float amax = 0.0f;
-#pragma unroll
-  for (int j = 0; j < NV; ++j) amax = fmaxf(amax, fabsf(v[j]));
+  const float amax = group_absmax<NV>(v);
   const float r = d6 > 0.0f ? __fdiv_rn(amax, d6) : 0.0f;
   const uint32_t sb = e4m3_byte(r);
   const float S = __fmul_rn(e4m3_value(sb), s_t);
@@ -151,9 +175,7 @@ __device__ __forceinline__ uint32_t quant_nv(const float* v, float s_t, float d6
 // INT4 symmetric: s = amax / 7, q = clamp(rne(y * (1/s)), -7, 7), two's-complement nibbles.
 template <int NV>
 __device__ __forceinline__ float quant_int4(const float* v, uint32_t* words) {
-  float amax = 0.0f;
-#pragma unroll
-  for (int j = 0; j < NV; ++j) amax = fmaxf(amax, fabsf(v[j]));
+  const float amax = group_absmax<NV>(v);
   const float s = __fdiv_rn(amax, 7.0f);
   float inv = s > 0.0f ? __frcp_rn(s) : 0.0f;
   if (isinf(inv)) inv = 0.0f;
@@ -179,13 +201,16 @@ __device__ __forceinline__ T* offset_ptr(void* base, long long bytes) {
 // ---------------------------------------------------------------- the kernel
 template <class Cfg>
 __global__ void __launch_bounds__(Cfg::THREADS, 1)
-    wush_fused_kernel(const __grid_constant__ CUtensorMap tmap_in, const FusedParams p) {
-  constexpr int G = Cfg::G, CH = Cfg::CH, BPT = Cfg::BPT, STAGES = Cfg::STAGES;
+    wush_fused_kernel(const __grid_constant__ CUtensorMap tmap_in, const __grid_constant__ CUtensorMap tmap_codes,
+                      const FusedParams p) {
+  constexpr int G = Cfg::G, CH = Cfg::CH, BPT = Cfg::BPT, STAGES = Cfg::STAGES, BPW = Cfg::BPW;
+  constexpr int NCH = CH / 32;                 // 16-byte code chunks per staged row
+  constexpr int CPT = NCH / 2;                 // code chunks produced per epilogue thread
+  constexpr int SW_SHIFT = NCH == 4 ? 1 : 2;   // staging swizzle = TMA 64B / 32B swizzle pattern
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_addr(smem);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::OFF_BAR);
-  const uint32_t bar0 = smem_addr(bars);
+  const uint32_t bar0 = sbase + Cfg::OFF_BAR;
   auto BAR = [&](int i) -> uint32_t { return bar0 + 8u * static_cast<uint32_t>(i); };
   const int B_FULL = 0, B_EMPTY = STAGES, B_OFULL = 2 * STAGES, B_OEMPTY = 2 * STAGES + 2,
             B_TFULL = 2 * STAGES + 4, B_TEMPTY = 2 * STAGES + 6, B_AFULL = 2 * STAGES + 8,
@@ -202,12 +227,12 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(BAR(B_FULL + s), 1);
-      mbar_init(BAR(B_EMPTY + s), Cfg::IN_F32 ? 128 : 1);
+      mbar_init(BAR(B_EMPTY + s), Cfg::IN_F32 ? 64 : 1);
     }
     for (int k = 0; k < 2; ++k) {
-      mbar_init(BAR(B_OFULL + k), 128);
+      mbar_init(BAR(B_OFULL + k), 64);
       mbar_init(BAR(B_OEMPTY + k), 1);
-      mbar_init(BAR(B_TFULL + k), 128);
+      mbar_init(BAR(B_TFULL + k), 64);
       mbar_init(BAR(B_TEMPTY + k), 1);
       mbar_init(BAR(B_AFULL + k), 1);
       mbar_init(BAR(B_AEMPTY + k), Cfg::N_EPI_WARPS);
@@ -216,8 +241,9 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
     *abort_flag = 0;
     fence_barrier_init();
     tma_prefetch_desc(&tmap_in);
+    if (p.codes_via_tma) tma_prefetch_desc(&tmap_codes);
   }
-  if (warp == 1) {
+  if (warp == 0) {
     tmem_alloc(smem_addr(const_cast<uint32_t*>(tmem_slot)), Cfg::TMEM_COLS);
     tmem_relinquish();
   }
@@ -230,12 +256,8 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       const uint64_t pol = l2_policy_evict_first();
-      int stage = 0;
+      int stage = 0, n_loaded = 0;
       uint32_t phase = 0;
-      int issued_parity[STAGES];
-      bool issued[STAGES];
-#pragma unroll
-      for (int s = 0; s < STAGES; ++s) issued[s] = false, issued_parity[s] = 0;
       for (int t = t_begin; t < t_end; ++t) {
         if (!wait_bounded(BAR(B_EMPTY + stage), phase ^ 1u, abort_flag, 1u, lim)) break;
         const int ct = t / nrt, rt = t - ct * nrt;
@@ -248,67 +270,57 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
           for (int s = 0; s < Cfg::SUB; ++s)
             tma_load_2d(dst + s * 16384, &tmap_in, BAR(B_FULL + stage), ct * CH + 64 * s, rt * 128, pol);
         }
-        issued[stage] = true;
-        issued_parity[stage] = static_cast<int>(phase);
+        ++n_loaded;
         if (++stage == STAGES) stage = 0, phase ^= 1u;
       }
-      if (*abort_flag) {  // let every copy still in flight land before the CTA exits
-        for (int s = 0; s < STAGES; ++s)
-          if (issued[s]) {
-            volatile int no_abort = 0;
-            wait_bounded(BAR(B_FULL + s), static_cast<uint32_t>(issued_parity[s]), &no_abort, 16u, lim);
-          }
+      if (*abort_flag) {  // let the copies still in flight land before the CTA exits
+        volatile int no_abort = 0;
+        for (int k = (n_loaded > STAGES ? n_loaded - STAGES : 0); k < n_loaded; ++k)
+          wait_bounded(BAR(B_FULL + k % STAGES), static_cast<uint32_t>((k / STAGES) & 1), &no_abort, 16u, lim);
       }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16_f32(128, G);
+      constexpr uint32_t idesc_hl = idesc_bf16_f32(128, 2 * G);   // hi|lo stacked along N
+      constexpr uint32_t idesc_h = idesc_bf16_f32(128, G);        // hi only
       int stage = 0, obuf = 0;
       uint32_t phase = 0, ophase = 0;
       int epoch = -1, prev_ct = -1;
       int it = 0;
-      bool ok = true;
-      for (int t = t_begin; t < t_end && ok; ++t, ++it) {
+      for (int t = t_begin; t < t_end; ++t, ++it) {
         const int ct = t / nrt;
         if (ct != prev_ct) {
           ++epoch;
           prev_ct = ct;
-          if (!wait_bounded(BAR(B_TFULL + (epoch & 1)), static_cast<uint32_t>((epoch >> 1) & 1), abort_flag, 2u, lim)) { ok = false; break; }
+          if (!wait_bounded(BAR(B_TFULL + (epoch & 1)), static_cast<uint32_t>((epoch >> 1) & 1), abort_flag, 2u, lim)) break;
         }
         const int tslot = epoch & 1;
         uint32_t a_hi, a_lo = 0;
         if (Cfg::IN_F32) {
-          if (!wait_bounded(BAR(B_OFULL + obuf), ophase, abort_flag, 2u, lim)) { ok = false; break; }
+          if (!wait_bounded(BAR(B_OFULL + obuf), ophase, abort_flag, 2u, lim)) break;
           a_hi = sbase + Cfg::OFF_OPER + obuf * 2 * Cfg::OPER_BYTES;
           a_lo = a_hi + Cfg::OPER_BYTES;
         } else {
-          if (!wait_bounded(BAR(B_FULL + stage), phase, abort_flag, 2u, lim)) { ok = false; break; }
+          if (!wait_bounded(BAR(B_FULL + stage), phase, abort_flag, 2u, lim)) break;
           a_hi = sbase + Cfg::OFF_STAGE + stage * Cfg::STAGE_BYTES;
         }
         const int acc = it & 1;
-        if (!wait_bounded(BAR(B_AEMPTY + acc), static_cast<uint32_t>(((it >> 1) & 1) ^ 1), abort_flag, 2u, lim)) { ok = false; break; }
+        if (!wait_bounded(BAR(B_AEMPTY + acc), static_cast<uint32_t>(((it >> 1) & 1) ^ 1), abort_flag, 2u, lim)) break;
         tc_fence_after();
         const uint32_t tbase = sbase + Cfg::OFF_T + tslot * Cfg::TSLOT_BYTES;
 #pragma unroll
         for (int b = 0; b < BPT; ++b) {
-          const uint32_t d = tmem_base + static_cast<uint32_t>(acc * CH + b * G);
+          const uint32_t d = tmem_base + static_cast<uint32_t>(acc * Cfg::ACC_COLS + b * 2 * G);
           // A: block b occupies bytes [b*2G, b*2G + 2G) of the 128-byte rows of sub-tile (b*G)/64
           const uint32_t a_off = static_cast<uint32_t>(((b * G) / 64) * 16384 + ((b * G) % 64) * 2);
-          // B: panel b / BLK_PER_PANEL; hi at byte (b % BLK_PER_PANEL) * 4G, lo 2G further
-          const uint32_t p_off = static_cast<uint32_t>((b / Cfg::BLK_PER_PANEL) * Cfg::PANEL_BYTES +
-                                                        (b % Cfg::BLK_PER_PANEL) * 4 * G);
+          // B: panel b / BPP, K bytes [(b % BPP) * 2G, +2G) of its 2G rows (hi rows, then lo rows)
+          const uint32_t p_off = static_cast<uint32_t>((b / Cfg::BPP) * Cfg::PANEL_BYTES + (b % Cfg::BPP) * 2 * G);
 #pragma unroll
           for (int kk = 0; kk < G / 16; ++kk) {
-            const uint64_t ah = desc_k_sw128(a_hi + a_off + kk * 32);
-            const uint64_t bh = desc_k_sw128(tbase + p_off + kk * 32);
-            const uint64_t bl = desc_k_sw128(tbase + p_off + 2 * G + kk * 32);
-            umma_bf16(d, ah, bh, idesc, kk > 0 ? 1u : 0u);
-            umma_bf16(d, ah, bl, idesc, 1u);
-            if (Cfg::IN_F32) {
-              const uint64_t al = desc_k_sw128(a_lo + a_off + kk * 32);
-              umma_bf16(d, al, bh, idesc, 1u);
-            }
+            const uint64_t bd = desc_k_sw128(tbase + p_off + kk * 32);
+            umma_bf16(d, desc_k_sw128(a_hi + a_off + kk * 32), bd, idesc_hl, kk > 0 ? 1u : 0u);
+            if (Cfg::IN_F32) umma_bf16(d, desc_k_sw128(a_lo + a_off + kk * 32), bd, idesc_h, 1u);
           }
         }
         if (Cfg::IN_F32) {
@@ -326,8 +338,8 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
       volatile int no_abort = 0;
       wait_bounded(BAR(B_DRAIN), 0u, &no_abort, 16u, lim);
     }
-  } else if (warp < 6) {
-    // ------------------------------------------------------------ converters (128 threads)
+  } else if (warp < 4) {
+    // ------------------------------------------------------------ converters (64 threads)
     const int ct_id = threadIdx.x - 64;
     int epoch = -1, prev_ct = -1;
     int stage = 0, obuf = 0;
@@ -340,30 +352,41 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
         const int slot = epoch & 1;
         if (!wait_bounded(BAR(B_TEMPTY + slot), static_cast<uint32_t>(((epoch >> 1) & 1) ^ 1), abort_flag, 4u, lim)) break;
         uint8_t* tdst = smem + Cfg::OFF_T + slot * Cfg::TSLOT_BYTES;
-        // BPT blocks x G rows x (G/8) chunks of 8 values
+        // BPT blocks x G rows x (G/8) chunks of 8 values; each thread first issues all of
+        // its loads (one memory latency), then splits and stores them
         constexpr int CHUNKS = BPT * G * (G / 8);
-        for (int q = ct_id; q < CHUNKS; q += 128) {
+        constexpr int PER_THREAD = (CHUNKS + 63) / 64;
+        float4 u[PER_THREAD][2];
+#pragma unroll
+        for (int k = 0; k < PER_THREAD; ++k) {
+          const int q = ct_id + 64 * k;
           const int b = q / (G * (G / 8));
           const int rem = q - b * (G * (G / 8));
           const int r = rem / (G / 8), j = rem - r * (G / 8);
           const int blk = ct * BPT + b;
-          float v[8];
-          if (blk < p.C) {
+          if (q < CHUNKS && blk < p.C) {
             const float4* src = reinterpret_cast<const float4*>(p.T + (static_cast<long long>(blk) * G + r) * G + 8 * j);
-            const float4 u0 = __ldg(src), u1 = __ldg(src + 1);
-            v[0] = u0.x; v[1] = u0.y; v[2] = u0.z; v[3] = u0.w;
-            v[4] = u1.x; v[5] = u1.y; v[6] = u1.z; v[7] = u1.w;
+            u[k][0] = __ldg(src);
+            u[k][1] = __ldg(src + 1);
           } else {
-#pragma unroll
-            for (int e = 0; e < 8; ++e) v[e] = 0.0f;
+            u[k][0] = u[k][1] = make_float4(0.f, 0.f, 0.f, 0.f);
           }
+        }
+#pragma unroll
+        for (int k = 0; k < PER_THREAD; ++k) {
+          const int q = ct_id + 64 * k;
+          if (q >= CHUNKS) break;
+          const int b = q / (G * (G / 8));
+          const int rem = q - b * (G * (G / 8));
+          const int r = rem / (G / 8), j = rem - r * (G / 8);
+          const float v[8] = {u[k][0].x, u[k][0].y, u[k][0].z, u[k][0].w,
+                              u[k][1].x, u[k][1].y, u[k][1].z, u[k][1].w};
           uint4 hi, lo;
           split8(v, hi, lo);
-          uint8_t* panel = tdst + (b / Cfg::BLK_PER_PANEL) * Cfg::PANEL_BYTES;
-          // a block's hi|lo row span is 4G bytes = G/4 chunks; hi first, lo G/8 chunks later
-          const int c0 = (b % Cfg::BLK_PER_PANEL) * (G / 4);
-          *reinterpret_cast<uint4*>(panel + sw128_off(r, c0 + j)) = hi;
-          *reinterpret_cast<uint4*>(panel + sw128_off(r, c0 + G / 8 + j)) = lo;
+          uint8_t* panel = tdst + (b / Cfg::BPP) * Cfg::PANEL_BYTES;
+          const int c = (b % Cfg::BPP) * (G / 8) + j;     // 16-byte chunk along K
+          *reinterpret_cast<uint4*>(panel + sw128_off(r, c)) = hi;
+          *reinterpret_cast<uint4*>(panel + sw128_off(G + r, c)) = lo;
         }
         fence_proxy_async_smem();
         mbar_arrive(BAR(B_TFULL + slot));
@@ -375,7 +398,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
         uint8_t* dhi = smem + Cfg::OFF_OPER + obuf * 2 * Cfg::OPER_BYTES;
         uint8_t* dlo = dhi + Cfg::OPER_BYTES;
         constexpr int CPR = CH / 8;    // 16-byte output chunks per row
-        for (int q = ct_id; q < 128 * CPR; q += 128) {
+        for (int q = ct_id; q < 128 * CPR; q += 64) {
           const int r = q / CPR, j = q - r * CPR;
           const float4* s4 = reinterpret_cast<const float4*>(src + r * CH * 4 + j * 32);
           const float4 u0 = s4[0], u1 = s4[1];
@@ -395,70 +418,146 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue (8 warps)
+    const int e = warp - 4;                    // epilogue warp index 0..7
     const int quad = warp & 3;                 // TMEM lanes this warp may read
-    const int half = (warp - 6) >> 2;          // which half of the tile's blocks
+    const int half = e >> 2;                   // which half of the tile's blocks it quantises
+    const int etid = e * 32 + lane;            // 0..255
+    const bool store_leader = (e == 0) && lane == 0;
     const int C = p.C;
+    const int code_row_bytes = p.d_in / 2;
+    const bool vec16 = (code_row_bytes % 16) == 0;
     float s_t = 0.0f, d6 = 0.0f;
     if (Cfg::FMT == kNVFP4 && !Cfg::AMAX_ONLY) {
       s_t = *p.tensor_scale;
       d6 = __fmul_rn(6.0f, s_t);
     }
+    bool live = true;
     float run_max = 0.0f;
     int it = 0;
     for (int t = t_begin; t < t_end; ++t, ++it) {
-      const int acc = it & 1;
-      if (!wait_bounded(BAR(B_AFULL + acc), static_cast<uint32_t>((it >> 1) & 1), abort_flag, 8u, lim)) break;
-      tc_fence_after();
       const int ct = t / nrt, rt = t - ct * nrt;
-      float v[Cfg::BPW][G];
-      const uint32_t tq = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(acc * CH);
+      const int acc = it & 1;
+      if (live && !wait_bounded(BAR(B_AFULL + acc), static_cast<uint32_t>((it >> 1) & 1), abort_flag, 8u, lim))
+        live = false;
+      const bool warp_live = __all_sync(0xffffffffu, live) && !*abort_flag;
+      float v[BPW][G];
+      if (warp_live) {
+        tc_fence_after();
+        const uint32_t tq = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(acc * Cfg::ACC_COLS);
 #pragma unroll
-      for (int bb = 0; bb < Cfg::BPW; ++bb) {
-        const uint32_t ta = tq + static_cast<uint32_t>((half * Cfg::BPW + bb) * G);
-        if (G == 32) tmem_ld_x32(ta, v[bb]); else tmem_ld_x16(ta, v[bb]);
+        for (int bb = 0; bb < BPW; ++bb) {
+          float hl[2 * G];
+          const uint32_t ta = tq + static_cast<uint32_t>((half * BPW + bb) * 2 * G);
+          if (G == 32) tmem_ld_x64(ta, hl); else tmem_ld_x32(ta, hl);
+          tmem_ld_wait();
+#pragma unroll
+          for (int jj = 0; jj < G; ++jj) v[bb][jj] = hl[jj] + hl[G + jj];   // X*T_hi^T + X*T_lo^T
+        }
       }
-      tmem_ld_wait();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(BAR(B_AEMPTY + acc));
 
-      const long long row = static_cast<long long>(rt) * 128 + quad * 32 + lane;
-      const bool row_ok = row < p.n_rows;
-      const int blk0 = ct * BPT + half * Cfg::BPW;
+      const int row = quad * 32 + lane;                       // row within the tile
+      const long long grow = static_cast<long long>(rt) * 128 + row;
+      const bool row_ok = grow < p.n_rows;
+      const int blk0 = ct * BPT + half * BPW;
       if (Cfg::AMAX_ONLY) {
+        if (warp_live) {
 #pragma unroll
-        for (int bb = 0; bb < Cfg::BPW; ++bb)
-          if (row_ok && blk0 + bb < C)
-#pragma unroll
-            for (int j = 0; j < G; ++j) run_max = fmaxf(run_max, fabsf(v[bb][j]));
+          for (int bb = 0; bb < BPW; ++bb)
+            if (row_ok && blk0 + bb < C) run_max = fmaxf(run_max, group_absmax<G>(v[bb]));
+        }
         continue;
       }
+      const int buf = it & 1;
+      uint8_t* cstage = smem + Cfg::OFF_CODES + buf * Cfg::CODE_STAGE;
+      uint8_t* sstage = smem + Cfg::OFF_SCALES + buf * Cfg::SCALE_STAGE;
+      if (warp_live) {
+        uint32_t cw[CPT * 4];
 #pragma unroll
-      for (int bb = 0; bb < Cfg::BPW; ++bb) {
-        const int blk = blk0 + bb;
-        if (!row_ok || blk >= C) continue;
-        uint32_t words[G / 8];
-        const long long cbyte = row * (p.d_in / 2) + static_cast<long long>(blk) * (G / 2);
-        if (Cfg::FMT == kMXFP4) {
-          const uint32_t sb = quant_mx<G>(v[bb], words);
-          offset_ptr<uint8_t>(p.scales, row * C + blk)[0] = static_cast<uint8_t>(sb);
-        } else if (Cfg::FMT == kNVFP4) {
-          const uint32_t sb = quant_nv<G>(v[bb], s_t, d6, words);
-          offset_ptr<uint8_t>(p.scales, row * C + blk)[0] = static_cast<uint8_t>(sb);
-        } else {
-          const float s = quant_int4<G>(v[bb], words);
-          offset_ptr<float>(p.scales, (row * C + blk) * 4)[0] = s;
-        }
-        if (G == 32) {
-          *offset_ptr<uint4>(p.codes, cbyte) = make_uint4(words[0], words[1], words[2], words[3]);
-        } else {
-          *offset_ptr<uint2>(p.codes, cbyte) = make_uint2(words[0], words[1]);
-        }
-        if (Cfg::EMIT_Y) {
-          float4* yd = reinterpret_cast<float4*>(p.y_out + row * p.d_in + static_cast<long long>(blk) * G);
+        for (int bb = 0; bb < BPW; ++bb) {
+          uint32_t* words = cw + bb * (G / 8);
+          if (Cfg::FMT == kMXFP4) {
+            sstage[row * BPT + half * BPW + bb] = static_cast<uint8_t>(quant_mx<G>(v[bb], words));
+          } else if (Cfg::FMT == kNVFP4) {
+            sstage[row * BPT + half * BPW + bb] = static_cast<uint8_t>(quant_nv<G>(v[bb], s_t, d6, words));
+          } else {
+            reinterpret_cast<float*>(sstage)[row * BPT + half * BPW + bb] = quant_int4<G>(v[bb], words);
+          }
+          if (Cfg::EMIT_Y && row_ok && blk0 + bb < C) {
+            float4* yd = reinterpret_cast<float4*>(p.y_out + grow * p.d_in + static_cast<long long>(blk0 + bb) * G);
 #pragma unroll
-          for (int k = 0; k < G / 4; ++k)
-            yd[k] = make_float4(v[bb][4 * k], v[bb][4 * k + 1], v[bb][4 * k + 2], v[bb][4 * k + 3]);
+            for (int k = 0; k < G / 4; ++k)
+              yd[k] = make_float4(v[bb][4 * k], v[bb][4 * k + 1], v[bb][4 * k + 2], v[bb][4 * k + 3]);
+          }
+        }
+#pragma unroll
+        for (int k = 0; k < CPT; ++k) {
+          const int c = half * CPT + k;
+          const int pc = c ^ ((row >> SW_SHIFT) & (NCH - 1));
+          *reinterpret_cast<uint4*>(cstage + row * (CH / 2) + pc * 16) =
+              make_uint4(cw[4 * k], cw[4 * k + 1], cw[4 * k + 2], cw[4 * k + 3]);
+        }
+        if (p.codes_via_tma) fence_proxy_async_smem();
+      }
+      // the staging buffer written two tiles from now is the one stored at the previous
+      // tile: make sure that store has read it before anyone moves past this barrier
+      if (store_leader && p.codes_via_tma) bulk_wait_read_all();
+      named_bar_sync(1, 256);      // the tile's codes and scales are staged
+      if (warp_live) {
+        if (p.codes_via_tma) {
+          if (store_leader) {
+            tma_store_2d(&tmap_codes, smem_addr(cstage), ct * (CH / 2), rt * 128);
+            bulk_commit_group();
+          }
+        } else {
+          // consecutive threads write consecutive 16-byte chunks of a row
+          const long long col0 = static_cast<long long>(ct) * (CH / 2);
+#pragma unroll
+          for (int c = etid; c < 128 * NCH; c += 256) {
+            const int r = c / NCH, q = c - r * NCH;
+            const long long gr = static_cast<long long>(rt) * 128 + r;
+            const long long gc = col0 + q * 16;
+            if (gr >= p.n_rows || gc >= code_row_bytes) continue;
+            const uint4 val = *reinterpret_cast<const uint4*>(cstage + r * (CH / 2) + ((q ^ ((r >> SW_SHIFT) & (NCH - 1))) << 4));
+            uint8_t* dst = p.codes + gr * code_row_bytes + gc;
+            if (vec16 && gc + 16 <= code_row_bytes) {
+              *reinterpret_cast<uint4*>(dst) = val;
+            } else {
+              *reinterpret_cast<uint2*>(dst) = make_uint2(val.x, val.y);
+              if (gc + 8 < code_row_bytes) *reinterpret_cast<uint2*>(dst + 8) = make_uint2(val.z, val.w);
+            }
+          }
+        }
+        // scales: one thread per row writes the tile's BPT scales of that row
+        if (etid < 128) {
+          const int r = etid;
+          const long long gr = static_cast<long long>(rt) * 128 + r;
+          const int nb = min(BPT, C - ct * BPT);
+          if (gr < p.n_rows && nb > 0) {
+            constexpr int ES = Cfg::FMT == kINT4 ? 4 : 1;
+            constexpr int RB = BPT * ES;   // bytes of one row's scales in this tile: 2..32
+            constexpr int VA = RB >= 16 ? 16 : RB;
+            const uint8_t* src = sstage + r * RB;
+            uint8_t* dst = offset_ptr<uint8_t>(p.scales, (gr * C + static_cast<long long>(ct) * BPT) * ES);
+            if (nb == BPT && (reinterpret_cast<uintptr_t>(dst) % VA) == 0) {
+              if constexpr (RB == 2) {
+                *reinterpret_cast<uint16_t*>(dst) = *reinterpret_cast<const uint16_t*>(src);
+              } else if constexpr (RB == 4) {
+                *reinterpret_cast<uint32_t*>(dst) = *reinterpret_cast<const uint32_t*>(src);
+              } else if constexpr (RB == 8) {
+                *reinterpret_cast<uint2*>(dst) = *reinterpret_cast<const uint2*>(src);
+              } else {
+                static_assert(RB % 16 == 0, "row scale bytes");
+#pragma unroll
+                for (int k = 0; k < RB / 16; ++k)
+                  reinterpret_cast<uint4*>(dst)[k] = reinterpret_cast<const uint4*>(src)[k];
+              }
+            } else {
+              for (int k = 0; k < nb * ES; ++k) dst[k] = src[k];
+            }
+          }
         }
       }
     }
@@ -467,11 +566,12 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
       for (int o = 16; o > 0; o >>= 1) run_max = fmaxf(run_max, __shfl_xor_sync(0xffffffffu, run_max, o));
       if (lane == 0 && run_max > 0.0f) atomicMax(p.amax_word, __float_as_uint(run_max));
     }
+    if (store_leader && p.codes_via_tma) bulk_wait_all();
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == 0) {
     tc_fence_after();
     tmem_dealloc(tmem_base, Cfg::TMEM_COLS);
   }
