@@ -29,6 +29,10 @@ __global__ void wush_selftest_wait_kernel(unsigned long long limit_ns) {
 }
 }  // namespace wush
 
+#ifndef WUSH_USE_PDL
+#define WUSH_USE_PDL 1
+#endif
+
 namespace {
 
 constexpr unsigned long long kDefaultWaitLimitNs = 2000000000ull;
@@ -76,7 +80,20 @@ int launch_fused(const CUtensorMap& map, const CUtensorMap& cmap, wush::FusedPar
     configured.fetch_or(bit, std::memory_order_acq_rel);
   }
   const int grid = p.total_tiles < sms ? p.total_tiles : sms;
-  wush::wush_fused_kernel<Cfg><<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(map, cmap, p);
+  // programmatic stream serialisation: the CTAs may be scheduled while the previous kernel
+  // in the stream drains; they do their set-up and then wait (griddepcontrol.wait) for it
+  // to complete before reading any input
+  cudaLaunchConfig_t lc = {};
+  lc.gridDim = dim3(static_cast<unsigned>(grid));
+  lc.blockDim = dim3(Cfg::THREADS);
+  lc.dynamicSmemBytes = Cfg::SMEM_BYTES;
+  lc.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  lc.attrs = attr;
+  lc.numAttrs = WUSH_USE_PDL ? 1 : 0;
+  if (cudaLaunchKernelEx(&lc, wush::wush_fused_kernel<Cfg>, map, cmap, p) != cudaSuccess) return WUSH_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? WUSH_OK : WUSH_ERR_CUDA;
 }
 
@@ -127,7 +144,7 @@ int quant_common(const void* in, bool in_f32, const float* T, int64_t rows, int6
   if (tensor_scale && !aligned(tensor_scale, 4)) return WUSH_ERR_MISALIGNED;
   if (debug && !aligned(y_out, 16)) return WUSH_ERR_MISALIGNED;
 
-  const int ch = in_f32 ? 64 : 128;   // channels per tile, as in FusedCfg
+  const int ch = in_f32 ? 64 : WUSH_ACT_TILE_CH;   // channels per tile, as in FusedCfg
   const long long n_row_tiles = (rows + 127) / 128;
   const long long n_col_tiles = (d_in + ch - 1) / ch;
   if (n_row_tiles * n_col_tiles > INT_MAX) return WUSH_ERR_INVALID_ARG;
@@ -145,7 +162,7 @@ int quant_common(const void* in, bool in_f32, const float* T, int64_t rows, int6
   const bool codes_tma = ((d_in / 2) % 16) == 0;
   if (codes_tma) {
     st = encode_2d(&cmap, codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, rows, d_in / 2, ch / 2,
-                   in_f32 ? CU_TENSOR_MAP_SWIZZLE_32B : CU_TENSOR_MAP_SWIZZLE_64B);
+                   ch == 128 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B);
     if (st != WUSH_OK) return st;
   }
 

@@ -26,7 +26,16 @@
 #pragma once
 #include <cstdint>
 #include <cuda_bf16.h>
+#include <type_traits>
 #include "wush_ptx.cuh"
+
+// Tuning of the bf16 activation path (channels per tile, input stages in flight).
+#ifndef WUSH_ACT_TILE_CH
+#define WUSH_ACT_TILE_CH 128
+#endif
+#ifndef WUSH_ACT_STAGES
+#define WUSH_ACT_STAGES 5
+#endif
 
 namespace wush {
 
@@ -56,11 +65,11 @@ struct FusedCfg {
   static constexpr bool AMAX_ONLY = AMAX_ONLY_;
   static constexpr bool EMIT_Y = EMIT_Y_;
   static constexpr int BM = 128;                       // rows per tile = UMMA M
-  static constexpr int CH = IN_F32 ? 64 : 128;         // channels per tile
+  static constexpr int CH = IN_F32 ? 64 : WUSH_ACT_TILE_CH;   // channels per tile
   static constexpr int BPT = CH / G;                   // blocks per tile
   static constexpr int SUB = CH / 64;                  // 128-byte-wide bf16 operand sub-tiles
-  static constexpr int STAGES = IN_F32 ? 3 : 5;
-  static constexpr int STAGE_BYTES = IN_F32 ? BM * CH * 4 : BM * CH * 2;  // 32 KiB
+  static constexpr int STAGES = IN_F32 ? 3 : WUSH_ACT_STAGES;
+  static constexpr int STAGE_BYTES = IN_F32 ? BM * CH * 4 : BM * CH * 2;  // 32 KiB fp32, 16 KiB bf16
   static constexpr int OPER_BYTES = BM * CH * 2;       // one bf16 operand tile (hi or lo)
   // transform panels: 2G rows (hi rows then lo rows) x 128 bytes of K; a 128-byte row
   // holds the K = G values of BPP = 64/G blocks side by side
@@ -69,21 +78,21 @@ struct FusedCfg {
   static constexpr int N_PANELS = BPT / BPP;
   static constexpr int TSLOT_BYTES = N_PANELS * PANEL_BYTES;
   static constexpr int ACC_COLS = 2 * CH;              // hi|lo of every block of a tile
-  static constexpr int TMEM_COLS = 2 * ACC_COLS;       // two accumulator buffers
-  static constexpr int BPW = BPT / 2;                  // blocks per epilogue warp
-  static constexpr int N_EPI_WARPS = 8;
+  static constexpr int NACC = 512 / ACC_COLS;          // accumulator buffers in TMEM
+  static constexpr int TMEM_COLS = NACC * ACC_COLS;
+  static constexpr int N_GROUPS = 2;                   // epilogue groups, alternate tiles
+  static constexpr int GROUP_WARPS = 4;                // one warp per TMEM lane quadrant
   static constexpr int THREADS = 12 * 32;
   static constexpr int CODE_STAGE = 128 * CH / 2;      // one tile of packed codes
-  static constexpr int SCALE_STAGE = 128 * BPT * (FMT == kINT4 ? 4 : 1);
+  static_assert(NACC % N_GROUPS == 0, "each group owns whole accumulator buffers");
   // shared memory carve-up (offsets from a 1024-byte aligned base)
   static constexpr int OFF_STAGE = 0;
   static constexpr int OFF_OPER = OFF_STAGE + STAGES * STAGE_BYTES;
   static constexpr int OFF_T = OFF_OPER + (IN_F32 ? 2 * 2 * OPER_BYTES : 0);
-  static constexpr int OFF_CODES = OFF_T + 2 * TSLOT_BYTES;
-  static constexpr int OFF_SCALES = OFF_CODES + 2 * CODE_STAGE;
-  static constexpr int OFF_BAR = OFF_SCALES + 2 * SCALE_STAGE;
-  // barriers: full[S], empty[S], ofull[2], oempty[2], tfull[2], tempty[2], afull[2], aempty[2], drain
-  static constexpr int N_BARS = 2 * STAGES + 13;
+  static constexpr int OFF_CODES = OFF_T + 2 * TSLOT_BYTES;   // [group][2] code staging buffers
+  static constexpr int OFF_BAR = OFF_CODES + N_GROUPS * 2 * CODE_STAGE;
+  // barriers: full[S], empty[S], ofull[2], oempty[2], tfull[2], tempty[2], afull[NACC], aempty[NACC], drain
+  static constexpr int N_BARS = 2 * STAGES + 9 + 2 * NACC;
   static constexpr int OFF_MISC = OFF_BAR + 8 * N_BARS;
   static constexpr int SMEM_BYTES = OFF_MISC + 64 + 1024;   // + alignment slack
   static_assert(G == 16 || G == 32, "G must be 16 or 32");
@@ -118,6 +127,27 @@ __device__ __forceinline__ void split8(const float* v, uint4& hi, uint4& lo) {
   lo = make_uint4(l[0], l[1], l[2], l[3]);
 }
 
+// Packed fp32 pair arithmetic (sm_100a add/mul .f32x2): each is the IEEE round-to-nearest
+// result of the two scalar operations.
+__device__ __forceinline__ void add2_rn(float& a0, float& a1, float b0, float b1) {
+  asm("{\n\t.reg .b64 ra, rb;\n\t"
+      "mov.b64 ra, {%0, %1};\n\t"
+      "mov.b64 rb, {%2, %3};\n\t"
+      "add.rn.f32x2 ra, ra, rb;\n\t"
+      "mov.b64 {%0, %1}, ra;\n\t}"
+      : "+f"(a0), "+f"(a1)
+      : "f"(b0), "f"(b1));
+}
+__device__ __forceinline__ void mul2_rn(float& a0, float& a1, float m) {
+  asm("{\n\t.reg .b64 ra, rb;\n\t"
+      "mov.b64 ra, {%0, %1};\n\t"
+      "mov.b64 rb, {%2, %2};\n\t"
+      "mul.rn.f32x2 ra, ra, rb;\n\t"
+      "mov.b64 {%0, %1}, ra;\n\t}"
+      : "+f"(a0), "+f"(a1)
+      : "f"(m));
+}
+
 // Largest |v_j| of a group, as a balanced tree (max is exact, so the order is free).
 template <int NV>
 __device__ __forceinline__ float group_absmax(const float* v) {
@@ -148,7 +178,11 @@ __device__ __forceinline__ uint32_t quant_mx(const float* v, uint32_t* words) {
   const float mul = __uint_as_float(sb < 254 ? static_cast<uint32_t>(254 - sb) << 23 : 0x00400000u);
   float w[NV];
 #pragma unroll
-  for (int j = 0; j < NV; ++j) w[j] = v[j] * mul;   // exact: multiplication by a power of two
+  for (int j = 0; j < NV; j += 2) {   // exact: multiplication by a power of two
+    w[j] = v[j];
+    w[j + 1] = v[j + 1];
+    mul2_rn(w[j], w[j + 1], mul);
+  }
 #pragma unroll
   for (int k = 0; k < NV / 8; ++k) words[k] = e2m1_pack8(w + 8 * k);
   return static_cast<uint32_t>(sb);
@@ -166,7 +200,11 @@ __device__ __forceinline__ uint32_t quant_nv(const float* v, float s_t, float d6
   if (isinf(inv)) inv = 0.0f;       // scale below the fp32 reciprocal range: group encodes as zero
   float w[NV];
 #pragma unroll
-  for (int j = 0; j < NV; ++j) w[j] = __fmul_rn(v[j], inv);
+  for (int j = 0; j < NV; j += 2) {   // each product rounded to fp32
+    w[j] = v[j];
+    w[j + 1] = v[j + 1];
+    mul2_rn(w[j], w[j + 1], inv);
+  }
 #pragma unroll
   for (int k = 0; k < NV / 8; ++k) words[k] = e2m1_pack8(w + 8 * k);
   return sb;
@@ -203,9 +241,8 @@ template <class Cfg>
 __global__ void __launch_bounds__(Cfg::THREADS, 1)
     wush_fused_kernel(const __grid_constant__ CUtensorMap tmap_in, const __grid_constant__ CUtensorMap tmap_codes,
                       const FusedParams p) {
-  constexpr int G = Cfg::G, CH = Cfg::CH, BPT = Cfg::BPT, STAGES = Cfg::STAGES, BPW = Cfg::BPW;
+  constexpr int G = Cfg::G, CH = Cfg::CH, BPT = Cfg::BPT, STAGES = Cfg::STAGES;
   constexpr int NCH = CH / 32;                 // 16-byte code chunks per staged row
-  constexpr int CPT = NCH / 2;                 // code chunks produced per epilogue thread
   constexpr int SW_SHIFT = NCH == 4 ? 1 : 2;   // staging swizzle = TMA 64B / 32B swizzle pattern
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -214,7 +251,8 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
   auto BAR = [&](int i) -> uint32_t { return bar0 + 8u * static_cast<uint32_t>(i); };
   const int B_FULL = 0, B_EMPTY = STAGES, B_OFULL = 2 * STAGES, B_OEMPTY = 2 * STAGES + 2,
             B_TFULL = 2 * STAGES + 4, B_TEMPTY = 2 * STAGES + 6, B_AFULL = 2 * STAGES + 8,
-            B_AEMPTY = 2 * STAGES + 10, B_DRAIN = 2 * STAGES + 12;
+            B_AEMPTY = 2 * STAGES + 8 + Cfg::NACC, B_DRAIN = 2 * STAGES + 8 + 2 * Cfg::NACC;
+  constexpr int NACC = Cfg::NACC;
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + Cfg::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::OFF_MISC + 4);
 
@@ -234,8 +272,10 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
       mbar_init(BAR(B_OEMPTY + k), 1);
       mbar_init(BAR(B_TFULL + k), 64);
       mbar_init(BAR(B_TEMPTY + k), 1);
+    }
+    for (int k = 0; k < NACC; ++k) {
       mbar_init(BAR(B_AFULL + k), 1);
-      mbar_init(BAR(B_AEMPTY + k), Cfg::N_EPI_WARPS);
+      mbar_init(BAR(B_AEMPTY + k), Cfg::GROUP_WARPS);
     }
     mbar_init(BAR(B_DRAIN), 1);
     *abort_flag = 0;
@@ -243,6 +283,25 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
     tma_prefetch_desc(&tmap_in);
     if (p.codes_via_tma) tma_prefetch_desc(&tmap_codes);
   }
+  // Launched with programmatic stream serialisation: everything above overlapped the end
+  // of the previous kernel in the stream; its results are visible only after this wait.
+  grid_dependency_wait();
+  grid_launch_dependents();
+  // the producer starts streaming before the rest of the CTA is set up
+  const uint64_t l2_pol = l2_policy_evict_first();
+  int n_preloaded = 0;
+  if (threadIdx.x == 0) {
+    for (; n_preloaded < STAGES && t_begin + n_preloaded < t_end; ++n_preloaded) {
+      const int t = t_begin + n_preloaded;
+      const int ct = t / nrt, rt = t - ct * nrt;
+      const uint32_t dst = sbase + Cfg::OFF_STAGE + n_preloaded * Cfg::STAGE_BYTES;
+      mbar_arrive_expect_tx(BAR(B_FULL + n_preloaded), Cfg::STAGE_BYTES);
+#pragma unroll
+      for (int s = 0; s < Cfg::SUB; ++s)
+        tma_load_2d(dst + s * 16384, &tmap_in, BAR(B_FULL + n_preloaded), ct * CH + 64 * s, rt * 128, l2_pol);
+    }
+  }
+  __syncwarp();
   if (warp == 0) {
     tmem_alloc(smem_addr(const_cast<uint32_t*>(tmem_slot)), Cfg::TMEM_COLS);
     tmem_relinquish();
@@ -255,10 +314,11 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      const uint64_t pol = l2_policy_evict_first();
-      int stage = 0, n_loaded = 0;
-      uint32_t phase = 0;
-      for (int t = t_begin; t < t_end; ++t) {
+      const uint64_t pol = l2_pol;
+      int n_loaded = n_preloaded;
+      int stage = n_preloaded % STAGES;
+      uint32_t phase = n_preloaded == STAGES ? 1u : 0u;
+      for (int t = t_begin + n_preloaded; t < t_end; ++t) {
         if (!wait_bounded(BAR(B_EMPTY + stage), phase ^ 1u, abort_flag, 1u, lim)) break;
         const int ct = t / nrt, rt = t - ct * nrt;
         const uint32_t dst = sbase + Cfg::OFF_STAGE + stage * Cfg::STAGE_BYTES;
@@ -305,8 +365,8 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
           if (!wait_bounded(BAR(B_FULL + stage), phase, abort_flag, 2u, lim)) break;
           a_hi = sbase + Cfg::OFF_STAGE + stage * Cfg::STAGE_BYTES;
         }
-        const int acc = it & 1;
-        if (!wait_bounded(BAR(B_AEMPTY + acc), static_cast<uint32_t>(((it >> 1) & 1) ^ 1), abort_flag, 2u, lim)) break;
+        const int acc = it % NACC;
+        if (!wait_bounded(BAR(B_AEMPTY + acc), static_cast<uint32_t>(((it / NACC) & 1) ^ 1), abort_flag, 2u, lim)) break;
         tc_fence_after();
         const uint32_t tbase = sbase + Cfg::OFF_T + tslot * Cfg::TSLOT_BYTES;
 #pragma unroll
@@ -417,15 +477,19 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
       }
     }
   } else {
-    // ------------------------------------------------------------ epilogue (8 warps)
-    const int e = warp - 4;                    // epilogue warp index 0..7
+    // ------------------------------------------------------------ epilogue: 2 groups x 4 warps
+    // Group g takes the tiles with local index = g (mod 2) and the accumulator buffers of
+    // those tiles; the groups run independently, so one group's TMEM loads, barrier and
+    // store overlap the other group's arithmetic.  Thread = token row of the tile; it
+    // handles the tile's blocks one after the other.
+    const int grp = (warp - 4) >> 2;           // epilogue group
     const int quad = warp & 3;                 // TMEM lanes this warp may read
-    const int half = e >> 2;                   // which half of the tile's blocks it quantises
-    const int etid = e * 32 + lane;            // 0..255
-    const bool store_leader = (e == 0) && lane == 0;
+    const int row = quad * 32 + lane;          // row within the tile
+    const bool store_leader = (quad == 0) && lane == 0;
     const int C = p.C;
     const int code_row_bytes = p.d_in / 2;
     const bool vec16 = (code_row_bytes % 16) == 0;
+    using ScaleT = typename std::conditional<Cfg::FMT == kINT4, float, uint8_t>::type;
     float s_t = 0.0f, d6 = 0.0f;
     if (Cfg::FMT == kNVFP4 && !Cfg::AMAX_ONLY) {
       s_t = *p.tensor_scale;
@@ -433,130 +497,114 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
     }
     bool live = true;
     float run_max = 0.0f;
-    int it = 0;
-    for (int t = t_begin; t < t_end; ++t, ++it) {
+    int m = 0;                                  // tiles handled by this group so far
+    for (int it = grp; t_begin + it < t_end; it += Cfg::N_GROUPS, ++m) {
+      const int t = t_begin + it;
       const int ct = t / nrt, rt = t - ct * nrt;
-      const int acc = it & 1;
-      if (live && !wait_bounded(BAR(B_AFULL + acc), static_cast<uint32_t>((it >> 1) & 1), abort_flag, 8u, lim))
+      const int acc = it % NACC;
+      if (live && !wait_bounded(BAR(B_AFULL + acc), static_cast<uint32_t>((it / NACC) & 1), abort_flag, 8u, lim))
         live = false;
       const bool warp_live = __all_sync(0xffffffffu, live) && !*abort_flag;
-      float v[BPW][G];
-      if (warp_live) {
-        tc_fence_after();
-        const uint32_t tq = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(acc * Cfg::ACC_COLS);
-#pragma unroll
-        for (int bb = 0; bb < BPW; ++bb) {
-          float hl[2 * G];
-          const uint32_t ta = tq + static_cast<uint32_t>((half * BPW + bb) * 2 * G);
-          if (G == 32) tmem_ld_x64(ta, hl); else tmem_ld_x32(ta, hl);
-          tmem_ld_wait();
-#pragma unroll
-          for (int jj = 0; jj < G; ++jj) v[bb][jj] = hl[jj] + hl[G + jj];   // X*T_hi^T + X*T_lo^T
-        }
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(BAR(B_AEMPTY + acc));
-
-      const int row = quad * 32 + lane;                       // row within the tile
       const long long grow = static_cast<long long>(rt) * 128 + row;
       const bool row_ok = grow < p.n_rows;
-      const int blk0 = ct * BPT + half * BPW;
-      if (Cfg::AMAX_ONLY) {
+      uint8_t* cstage = smem + Cfg::OFF_CODES + (grp * 2 + (m & 1)) * Cfg::CODE_STAGE;
+      const uint32_t tq = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(acc * Cfg::ACC_COLS);
+      ScaleT sc[BPT];
+      if (warp_live) tc_fence_after();
+#pragma unroll
+      for (int b = 0; b < BPT; ++b) {
+        float hl[2 * G];
         if (warp_live) {
-#pragma unroll
-          for (int bb = 0; bb < BPW; ++bb)
-            if (row_ok && blk0 + bb < C) run_max = fmaxf(run_max, group_absmax<G>(v[bb]));
+          if constexpr (G == 32) tmem_ld64_sync(tq + static_cast<uint32_t>(b * 2 * G), hl);
+          else tmem_ld32_sync(tq + static_cast<uint32_t>(b * 2 * G), hl);
         }
-        continue;
-      }
-      const int buf = it & 1;
-      uint8_t* cstage = smem + Cfg::OFF_CODES + buf * Cfg::CODE_STAGE;
-      uint8_t* sstage = smem + Cfg::OFF_SCALES + buf * Cfg::SCALE_STAGE;
-      if (warp_live) {
-        uint32_t cw[CPT * 4];
+        if (b == BPT - 1) {             // the whole accumulator buffer has been read
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(BAR(B_AEMPTY + acc));
+        }
+        if (!warp_live) continue;
 #pragma unroll
-        for (int bb = 0; bb < BPW; ++bb) {
-          uint32_t* words = cw + bb * (G / 8);
-          if (Cfg::FMT == kMXFP4) {
-            sstage[row * BPT + half * BPW + bb] = static_cast<uint8_t>(quant_mx<G>(v[bb], words));
-          } else if (Cfg::FMT == kNVFP4) {
-            sstage[row * BPT + half * BPW + bb] = static_cast<uint8_t>(quant_nv<G>(v[bb], s_t, d6, words));
+        for (int jj = 0; jj < G; jj += 2) add2_rn(hl[jj], hl[jj + 1], hl[G + jj], hl[G + jj + 1]);  // hi + lo
+        const int blk = ct * BPT + b;
+        if (Cfg::AMAX_ONLY) {
+          if (row_ok && blk < C) run_max = fmaxf(run_max, group_absmax<G>(hl));
+          continue;
+        }
+        if (Cfg::EMIT_Y && row_ok && blk < C) {
+          float4* yd = reinterpret_cast<float4*>(p.y_out + grow * p.d_in + static_cast<long long>(blk) * G);
+#pragma unroll
+          for (int k = 0; k < G / 4; ++k) yd[k] = make_float4(hl[4 * k], hl[4 * k + 1], hl[4 * k + 2], hl[4 * k + 3]);
+        }
+        uint32_t words[G / 8];
+        if (Cfg::FMT == kMXFP4) sc[b] = static_cast<ScaleT>(quant_mx<G>(hl, words));
+        else if (Cfg::FMT == kNVFP4) sc[b] = static_cast<ScaleT>(quant_nv<G>(hl, s_t, d6, words));
+        else sc[b] = static_cast<ScaleT>(quant_int4<G>(hl, words));
+        const int c = (b * G) / 32;       // 16-byte chunk of this row's codes
+        const int pc = c ^ ((row >> SW_SHIFT) & (NCH - 1));
+        if constexpr (G == 32) {
+          *reinterpret_cast<uint4*>(cstage + row * (CH / 2) + pc * 16) = make_uint4(words[0], words[1], words[2], words[3]);
+        } else {                          // a G=16 block fills one 8-byte half of the chunk
+          *reinterpret_cast<uint2*>(cstage + row * (CH / 2) + pc * 16 + (b & 1) * 8) = make_uint2(words[0], words[1]);
+        }
+      }
+      if (Cfg::AMAX_ONLY) continue;
+      // scales: this thread's row of the tile, straight from registers
+      if (warp_live && row_ok) {
+        const int nb = min(BPT, C - ct * BPT);
+        ScaleT* dst = reinterpret_cast<ScaleT*>(p.scales) + grow * C + static_cast<long long>(ct) * BPT;
+        constexpr int RB = BPT * static_cast<int>(sizeof(ScaleT));   // 2..32 bytes
+        if (nb == BPT && (reinterpret_cast<uintptr_t>(dst) % (RB >= 16 ? 16 : RB)) == 0) {
+          if constexpr (RB == 2) {
+            *reinterpret_cast<uint16_t*>(dst) = static_cast<uint16_t>(sc[0] | (sc[1] << 8));
+          } else if constexpr (RB == 4 && sizeof(ScaleT) == 1) {
+            *reinterpret_cast<uint32_t*>(dst) = static_cast<uint32_t>(sc[0]) | (static_cast<uint32_t>(sc[1]) << 8) |
+                                                (static_cast<uint32_t>(sc[2]) << 16) | (static_cast<uint32_t>(sc[3]) << 24);
+          } else if constexpr (RB == 8 && sizeof(ScaleT) == 1) {
+            uint32_t lo = 0, hi = 0;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) lo |= static_cast<uint32_t>(sc[k]) << (8 * k), hi |= static_cast<uint32_t>(sc[4 + k]) << (8 * k);
+            *reinterpret_cast<uint2*>(dst) = make_uint2(lo, hi);
+          } else if constexpr (sizeof(ScaleT) == 4 && RB % 16 == 0) {
+#pragma unroll
+            for (int k = 0; k < BPT / 4; ++k)
+              reinterpret_cast<float4*>(dst)[k] = make_float4(sc[4 * k], sc[4 * k + 1], sc[4 * k + 2], sc[4 * k + 3]);
           } else {
-            reinterpret_cast<float*>(sstage)[row * BPT + half * BPW + bb] = quant_int4<G>(v[bb], words);
-          }
-          if (Cfg::EMIT_Y && row_ok && blk0 + bb < C) {
-            float4* yd = reinterpret_cast<float4*>(p.y_out + grow * p.d_in + static_cast<long long>(blk0 + bb) * G);
 #pragma unroll
-            for (int k = 0; k < G / 4; ++k)
-              yd[k] = make_float4(v[bb][4 * k], v[bb][4 * k + 1], v[bb][4 * k + 2], v[bb][4 * k + 3]);
-          }
-        }
-#pragma unroll
-        for (int k = 0; k < CPT; ++k) {
-          const int c = half * CPT + k;
-          const int pc = c ^ ((row >> SW_SHIFT) & (NCH - 1));
-          *reinterpret_cast<uint4*>(cstage + row * (CH / 2) + pc * 16) =
-              make_uint4(cw[4 * k], cw[4 * k + 1], cw[4 * k + 2], cw[4 * k + 3]);
-        }
-        if (p.codes_via_tma) fence_proxy_async_smem();
-      }
-      // the staging buffer written two tiles from now is the one stored at the previous
-      // tile: make sure that store has read it before anyone moves past this barrier
-      if (store_leader && p.codes_via_tma) bulk_wait_read_all();
-      named_bar_sync(1, 256);      // the tile's codes and scales are staged
-      if (warp_live) {
-        if (p.codes_via_tma) {
-          if (store_leader) {
-            tma_store_2d(&tmap_codes, smem_addr(cstage), ct * (CH / 2), rt * 128);
-            bulk_commit_group();
+            for (int k = 0; k < BPT; ++k) dst[k] = sc[k];
           }
         } else {
-          // consecutive threads write consecutive 16-byte chunks of a row
-          const long long col0 = static_cast<long long>(ct) * (CH / 2);
-#pragma unroll
-          for (int c = etid; c < 128 * NCH; c += 256) {
-            const int r = c / NCH, q = c - r * NCH;
-            const long long gr = static_cast<long long>(rt) * 128 + r;
-            const long long gc = col0 + q * 16;
-            if (gr >= p.n_rows || gc >= code_row_bytes) continue;
-            const uint4 val = *reinterpret_cast<const uint4*>(cstage + r * (CH / 2) + ((q ^ ((r >> SW_SHIFT) & (NCH - 1))) << 4));
-            uint8_t* dst = p.codes + gr * code_row_bytes + gc;
-            if (vec16 && gc + 16 <= code_row_bytes) {
-              *reinterpret_cast<uint4*>(dst) = val;
-            } else {
-              *reinterpret_cast<uint2*>(dst) = make_uint2(val.x, val.y);
-              if (gc + 8 < code_row_bytes) *reinterpret_cast<uint2*>(dst + 8) = make_uint2(val.z, val.w);
-            }
-          }
+          for (int k = 0; k < nb; ++k) dst[k] = sc[k];
         }
-        // scales: one thread per row writes the tile's BPT scales of that row
-        if (etid < 128) {
-          const int r = etid;
-          const long long gr = static_cast<long long>(rt) * 128 + r;
-          const int nb = min(BPT, C - ct * BPT);
-          if (gr < p.n_rows && nb > 0) {
-            constexpr int ES = Cfg::FMT == kINT4 ? 4 : 1;
-            constexpr int RB = BPT * ES;   // bytes of one row's scales in this tile: 2..32
-            constexpr int VA = RB >= 16 ? 16 : RB;
-            const uint8_t* src = sstage + r * RB;
-            uint8_t* dst = offset_ptr<uint8_t>(p.scales, (gr * C + static_cast<long long>(ct) * BPT) * ES);
-            if (nb == BPT && (reinterpret_cast<uintptr_t>(dst) % VA) == 0) {
-              if constexpr (RB == 2) {
-                *reinterpret_cast<uint16_t*>(dst) = *reinterpret_cast<const uint16_t*>(src);
-              } else if constexpr (RB == 4) {
-                *reinterpret_cast<uint32_t*>(dst) = *reinterpret_cast<const uint32_t*>(src);
-              } else if constexpr (RB == 8) {
-                *reinterpret_cast<uint2*>(dst) = *reinterpret_cast<const uint2*>(src);
-              } else {
-                static_assert(RB % 16 == 0, "row scale bytes");
+      }
+      if (warp_live && p.codes_via_tma) fence_proxy_async_smem();
+      // the buffer this group writes next time was stored one group-tile ago: make sure
+      // that store has read it before anyone of the group moves past this barrier
+      if (store_leader && p.codes_via_tma) bulk_wait_read_all();
+      named_bar_sync(1 + grp, 128);  // the tile's codes are staged
+      if (!warp_live) continue;
+      if (p.codes_via_tma) {
+        if (store_leader) {
+          tma_store_2d(&tmap_codes, smem_addr(cstage), ct * (CH / 2), rt * 128);
+          bulk_commit_group();
+        }
+      } else {
+        // consecutive threads of the group write consecutive 16-byte chunks of a row
+        const int gtid = quad * 32 + lane;
+        const long long col0 = static_cast<long long>(ct) * (CH / 2);
 #pragma unroll
-                for (int k = 0; k < RB / 16; ++k)
-                  reinterpret_cast<uint4*>(dst)[k] = reinterpret_cast<const uint4*>(src)[k];
-              }
-            } else {
-              for (int k = 0; k < nb * ES; ++k) dst[k] = src[k];
-            }
+        for (int c = gtid; c < 128 * NCH; c += 128) {
+          const int r = c / NCH, q = c - r * NCH;
+          const long long gr = static_cast<long long>(rt) * 128 + r;
+          const long long gc = col0 + q * 16;
+          if (gr >= p.n_rows || gc >= code_row_bytes) continue;
+          const uint4 val = *reinterpret_cast<const uint4*>(cstage + r * (CH / 2) + ((q ^ ((r >> SW_SHIFT) & (NCH - 1))) << 4));
+          uint8_t* dst = p.codes + gr * code_row_bytes + gc;
+          if (vec16 && gc + 16 <= code_row_bytes) {
+            *reinterpret_cast<uint4*>(dst) = val;
+          } else {
+            *reinterpret_cast<uint2*>(dst) = make_uint2(val.x, val.y);
+            if (gc + 8 < code_row_bytes) *reinterpret_cast<uint2*>(dst + 8) = make_uint2(val.z, val.w);
           }
         }
       }
