@@ -56,6 +56,22 @@ def algorithmic_bytes(n_tok: int, d_in: int, G: int) -> int:
     return n_tok * d_in * 2 + n_tok * d_in // 2 + n_tok * C + C * G * G * 4
 
 
+def max_over_ranks(x: float, device=None) -> float:
+    """Largest value of x over all ranks (the timing rule: the slowest rank decides)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world: int, steps: int, bytes_per_step: int, elapsed_s: float) -> float:
+    """Whole-job GB/s: every rank processes its own batch per step (weak scaling)."""
+    return world * steps * bytes_per_step / elapsed_s / 1e9
+
+
 def kernel_source_hash() -> str:
     h = hashlib.sha256()
     for rel in KERNEL_SOURCES:
@@ -288,18 +304,15 @@ def run_native(args):
             e1.record(stream)
         e1.synchronize()
     torch.cuda.synchronize()
-    elapsed_s = e0.elapsed_time(e1) / 1e3
+    elapsed_s = max_over_ranks(e0.elapsed_time(e1) / 1e3, dev)
     if world > 1:
-        t = torch.tensor([elapsed_s], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_s = float(t.item())
         dist.barrier()
     st, bits = W.wush_device_status(stream)
     if st != 0:
         raise RuntimeError(f"device error word {bits:#x} after the timed region")
 
     per_launch_s = elapsed_s / args.steps
-    value = world * args.steps * step_bytes / elapsed_s / 1e9
+    value = job_throughput(world, args.steps, step_bytes, elapsed_s)
     tokens_s = world * args.steps * n / elapsed_s
     achieved = step_bytes / per_launch_s / 1e9
     peak, peak_kind = hbm_peak()
@@ -326,12 +339,8 @@ def run_native(args):
             e2e_step()
         f1.record(stream)
         f1.synchronize()
-    e2e_s = f0.elapsed_time(f1) / 1e3
-    if world > 1:
-        t = torch.tensor([e2e_s], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_s = float(t.item())
-    e2e_value = world * args.e2e_steps * step_bytes / e2e_s / 1e9
+    e2e_s = max_over_ranks(f0.elapsed_time(f1) / 1e3, dev)
+    e2e_value = job_throughput(world, args.e2e_steps, step_bytes, e2e_s)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
