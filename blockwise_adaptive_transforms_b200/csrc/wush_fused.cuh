@@ -287,7 +287,52 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
   // of the previous kernel in the stream; its results are visible only after this wait.
   grid_dependency_wait();
   grid_launch_dependents();
-  // the producer starts streaming before the rest of the CTA is set up
+  // The converter warps issue the loads of the first column tile's transforms before any
+  // input tile is requested (behind the input burst they would wait microseconds), then
+  // the producer starts streaming before the rest of the CTA is set up.
+  // One column tile's transforms: BPT blocks x G rows x (G/8) chunks of 8 values;
+  // converter id v (0..63) takes chunks v, v + 64, ...
+  constexpr int T_CHUNKS = BPT * G * (G / 8);
+  constexpr int T_PER_THREAD = (T_CHUNKS + 63) / 64;
+  float4 tpre[T_PER_THREAD][2];
+  auto load_T = [&](int ct, int v, float4 (&u)[T_PER_THREAD][2]) {
+#pragma unroll
+    for (int k = 0; k < T_PER_THREAD; ++k) {
+      const int q = v + 64 * k;
+      const int b = q / (G * (G / 8));
+      const int rem = q - b * (G * (G / 8));
+      const int r = rem / (G / 8), j = rem - r * (G / 8);
+      const int blk = ct * BPT + b;
+      if (q < T_CHUNKS && blk < p.C) {
+        const float4* src = reinterpret_cast<const float4*>(p.T + (static_cast<long long>(blk) * G + r) * G + 8 * j);
+        u[k][0] = __ldg(src);
+        u[k][1] = __ldg(src + 1);
+      } else {
+        u[k][0] = u[k][1] = make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    }
+  };
+  // hi/lo split of loaded chunks into the K-major SW128 panels of a transform slot
+  auto store_T = [&](int v, const float4 (&u)[T_PER_THREAD][2], uint8_t* tdst) {
+#pragma unroll
+    for (int k = 0; k < T_PER_THREAD; ++k) {
+      const int q = v + 64 * k;
+      if (q >= T_CHUNKS) break;
+      const int b = q / (G * (G / 8));
+      const int rem = q - b * (G * (G / 8));
+      const int r = rem / (G / 8), j = rem - r * (G / 8);
+      const float vals[8] = {u[k][0].x, u[k][0].y, u[k][0].z, u[k][0].w,
+                             u[k][1].x, u[k][1].y, u[k][1].z, u[k][1].w};
+      uint4 hi, lo;
+      split8(vals, hi, lo);
+      uint8_t* panel = tdst + (b / Cfg::BPP) * Cfg::PANEL_BYTES;
+      const int c = (b % Cfg::BPP) * (G / 8) + j;     // 16-byte chunk along K
+      *reinterpret_cast<uint4*>(panel + sw128_off(r, c)) = hi;
+      *reinterpret_cast<uint4*>(panel + sw128_off(G + r, c)) = lo;
+    }
+  };
+  if ((warp == 2 || warp == 3) && t_begin < t_end) load_T(t_begin / nrt, threadIdx.x - 64, tpre);
+  if (warp == 0 || warp == 2 || warp == 3) named_bar_sync(3, 96);
   const uint64_t l2_pol = l2_policy_evict_first();
   int n_preloaded = 0;
   if (threadIdx.x == 0) {
@@ -302,7 +347,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
     }
   }
   __syncwarp();
-  if (warp == 0) {
+  if (warp == 1) {
     tmem_alloc(smem_addr(const_cast<uint32_t*>(tmem_slot)), Cfg::TMEM_COLS);
     tmem_relinquish();
   }
@@ -341,57 +386,63 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
+    // This thread's wait -> issue -> commit chain bounds the tile rate, so it carries as
+    // little arithmetic as possible: operand descriptors, barrier addresses and the
+    // accumulator column advance incrementally, and on the bf16 path the epilogue (not
+    // this thread) frees the input stage once it has seen the tile's accumulator land.
     if (lane == 0) {
       constexpr uint32_t idesc_hl = idesc_bf16_f32(128, 2 * G);   // hi|lo stacked along N
       constexpr uint32_t idesc_h = idesc_bf16_f32(128, G);        // hi only
-      int stage = 0, obuf = 0;
-      uint32_t phase = 0, ophase = 0;
+      constexpr int NBUF = Cfg::IN_F32 ? 2 : STAGES;                // operand buffers cycled through
+      constexpr uint32_t A_STEP = (Cfg::IN_F32 ? 2 * Cfg::OPER_BYTES : Cfg::STAGE_BYTES) >> 4;
+      const uint64_t da_first = desc_k_sw128(sbase + (Cfg::IN_F32 ? Cfg::OFF_OPER : Cfg::OFF_STAGE));
+      const uint64_t db_slot0 = desc_k_sw128(sbase + Cfg::OFF_T);
+      const uint32_t full_first = BAR(Cfg::IN_F32 ? B_OFULL : B_FULL);
+      int buf = 0;
+      uint32_t phase = 0;
+      uint64_t da_hi = da_first;
+      uint32_t full_bar = full_first;
       int epoch = -1, prev_ct = -1;
       int it = 0;
+      int ct = t_begin / nrt, rt = t_begin - (t_begin / nrt) * nrt;
+      uint64_t db = db_slot0;
       for (int t = t_begin; t < t_end; ++t, ++it) {
-        const int ct = t / nrt;
         if (ct != prev_ct) {
           ++epoch;
           prev_ct = ct;
+          db = db_slot0 + ((epoch & 1) ? static_cast<uint64_t>(Cfg::TSLOT_BYTES >> 4) : 0ull);
           if (!wait_bounded(BAR(B_TFULL + (epoch & 1)), static_cast<uint32_t>((epoch >> 1) & 1), abort_flag, 2u, lim)) break;
         }
-        const int tslot = epoch & 1;
-        uint32_t a_hi, a_lo = 0;
-        if (Cfg::IN_F32) {
-          if (!wait_bounded(BAR(B_OFULL + obuf), ophase, abort_flag, 2u, lim)) break;
-          a_hi = sbase + Cfg::OFF_OPER + obuf * 2 * Cfg::OPER_BYTES;
-          a_lo = a_hi + Cfg::OPER_BYTES;
-        } else {
-          if (!wait_bounded(BAR(B_FULL + stage), phase, abort_flag, 2u, lim)) break;
-          a_hi = sbase + Cfg::OFF_STAGE + stage * Cfg::STAGE_BYTES;
-        }
-        const int acc = it % NACC;
+        const int acc = it & (NACC - 1);
+        if (!wait_bounded(full_bar, phase, abort_flag, 2u, lim)) break;
         if (!wait_bounded(BAR(B_AEMPTY + acc), static_cast<uint32_t>(((it / NACC) & 1) ^ 1), abort_flag, 2u, lim)) break;
         tc_fence_after();
-        const uint32_t tbase = sbase + Cfg::OFF_T + tslot * Cfg::TSLOT_BYTES;
+        const uint64_t da_lo = da_hi + (Cfg::OPER_BYTES >> 4);
+        const uint32_t d0 = tmem_base + static_cast<uint32_t>(acc * Cfg::ACC_COLS);
 #pragma unroll
         for (int b = 0; b < BPT; ++b) {
-          const uint32_t d = tmem_base + static_cast<uint32_t>(acc * Cfg::ACC_COLS + b * 2 * G);
           // A: block b occupies bytes [b*2G, b*2G + 2G) of the 128-byte rows of sub-tile (b*G)/64
           const uint32_t a_off = static_cast<uint32_t>(((b * G) / 64) * 16384 + ((b * G) % 64) * 2);
           // B: panel b / BPP, K bytes [(b % BPP) * 2G, +2G) of its 2G rows (hi rows, then lo rows)
           const uint32_t p_off = static_cast<uint32_t>((b / Cfg::BPP) * Cfg::PANEL_BYTES + (b % Cfg::BPP) * 2 * G);
 #pragma unroll
           for (int kk = 0; kk < G / 16; ++kk) {
-            const uint64_t bd = desc_k_sw128(tbase + p_off + kk * 32);
-            umma_bf16(d, desc_k_sw128(a_hi + a_off + kk * 32), bd, idesc_hl, kk > 0 ? 1u : 0u);
-            if (Cfg::IN_F32) umma_bf16(d, desc_k_sw128(a_lo + a_off + kk * 32), bd, idesc_h, 1u);
+            const uint64_t bd = db + ((p_off + kk * 32) >> 4);
+            umma_bf16(d0 + static_cast<uint32_t>(b * 2 * G), da_hi + ((a_off + kk * 32) >> 4), bd, idesc_hl,
+                      kk > 0 ? 1u : 0u);
+            if (Cfg::IN_F32)
+              umma_bf16(d0 + static_cast<uint32_t>(b * 2 * G), da_lo + ((a_off + kk * 32) >> 4), bd, idesc_h, 1u);
           }
         }
-        if (Cfg::IN_F32) {
-          umma_commit(BAR(B_OEMPTY + obuf));
-          if (++obuf == 2) obuf = 0, ophase ^= 1u;
-        } else {
-          umma_commit(BAR(B_EMPTY + stage));
-          if (++stage == STAGES) stage = 0, phase ^= 1u;
-        }
         umma_commit(BAR(B_AFULL + acc));
-        if (t + 1 == t_end || (t + 1) / nrt != ct) umma_commit(BAR(B_TEMPTY + tslot));
+        if (Cfg::IN_F32) umma_commit(BAR(B_OEMPTY + buf));
+        if (t + 1 == t_end || rt + 1 == nrt) umma_commit(BAR(B_TEMPTY + (epoch & 1)));
+        if (++rt == nrt) rt = 0, ++ct;
+        if (++buf == NBUF) {
+          buf = 0, phase ^= 1u, da_hi = da_first, full_bar = full_first;
+        } else {
+          da_hi += A_STEP, full_bar += 8u;
+        }
       }
       // every MMA issued above has finished before TMEM can be released
       umma_commit(BAR(B_DRAIN));
@@ -400,7 +451,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
     }
   } else if (warp < 4) {
     // ------------------------------------------------------------ converters (64 threads)
-    const int ct_id = threadIdx.x - 64;
+    const int v0 = threadIdx.x - 64;
     int epoch = -1, prev_ct = -1;
     int stage = 0, obuf = 0;
     uint32_t phase = 0, ophase = 0;
@@ -412,42 +463,15 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
         const int slot = epoch & 1;
         if (!wait_bounded(BAR(B_TEMPTY + slot), static_cast<uint32_t>(((epoch >> 1) & 1) ^ 1), abort_flag, 4u, lim)) break;
         uint8_t* tdst = smem + Cfg::OFF_T + slot * Cfg::TSLOT_BYTES;
-        // BPT blocks x G rows x (G/8) chunks of 8 values; each thread first issues all of
-        // its loads (one memory latency), then splits and stores them
-        constexpr int CHUNKS = BPT * G * (G / 8);
-        constexpr int PER_THREAD = (CHUNKS + 63) / 64;
-        float4 u[PER_THREAD][2];
+        // the first column tile's values were loaded before the set-up, later ones here
+        float4 u[T_PER_THREAD][2];
+        if (epoch == 0) {
 #pragma unroll
-        for (int k = 0; k < PER_THREAD; ++k) {
-          const int q = ct_id + 64 * k;
-          const int b = q / (G * (G / 8));
-          const int rem = q - b * (G * (G / 8));
-          const int r = rem / (G / 8), j = rem - r * (G / 8);
-          const int blk = ct * BPT + b;
-          if (q < CHUNKS && blk < p.C) {
-            const float4* src = reinterpret_cast<const float4*>(p.T + (static_cast<long long>(blk) * G + r) * G + 8 * j);
-            u[k][0] = __ldg(src);
-            u[k][1] = __ldg(src + 1);
-          } else {
-            u[k][0] = u[k][1] = make_float4(0.f, 0.f, 0.f, 0.f);
-          }
+          for (int k = 0; k < T_PER_THREAD; ++k) u[k][0] = tpre[k][0], u[k][1] = tpre[k][1];
+        } else {
+          load_T(ct, v0, u);
         }
-#pragma unroll
-        for (int k = 0; k < PER_THREAD; ++k) {
-          const int q = ct_id + 64 * k;
-          if (q >= CHUNKS) break;
-          const int b = q / (G * (G / 8));
-          const int rem = q - b * (G * (G / 8));
-          const int r = rem / (G / 8), j = rem - r * (G / 8);
-          const float v[8] = {u[k][0].x, u[k][0].y, u[k][0].z, u[k][0].w,
-                              u[k][1].x, u[k][1].y, u[k][1].z, u[k][1].w};
-          uint4 hi, lo;
-          split8(v, hi, lo);
-          uint8_t* panel = tdst + (b / Cfg::BPP) * Cfg::PANEL_BYTES;
-          const int c = (b % Cfg::BPP) * (G / 8) + j;     // 16-byte chunk along K
-          *reinterpret_cast<uint4*>(panel + sw128_off(r, c)) = hi;
-          *reinterpret_cast<uint4*>(panel + sw128_off(G + r, c)) = lo;
-        }
+        store_T(v0, u, tdst);
         fence_proxy_async_smem();
         mbar_arrive(BAR(B_TFULL + slot));
       }
@@ -458,7 +482,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
         uint8_t* dhi = smem + Cfg::OFF_OPER + obuf * 2 * Cfg::OPER_BYTES;
         uint8_t* dlo = dhi + Cfg::OPER_BYTES;
         constexpr int CPR = CH / 8;    // 16-byte output chunks per row
-        for (int q = ct_id; q < 128 * CPR; q += 64) {
+        for (int q = v0; q < 128 * CPR; q += 64) {
           const int r = q / CPR, j = q - r * CPR;
           const float4* s4 = reinterpret_cast<const float4*>(src + r * CH * 4 + j * 32);
           const float4 u0 = s4[0], u1 = s4[1];
@@ -504,6 +528,9 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
       const int acc = it % NACC;
       if (live && !wait_bounded(BAR(B_AFULL + acc), static_cast<uint32_t>((it / NACC) & 1), abort_flag, 8u, lim))
         live = false;
+      // bf16 path: the accumulator has landed, so the MMAs that read this tile's input
+      // stage are done; hand the stage back to the producer
+      if (!Cfg::IN_F32 && quad == 0 && lane == 0 && live) mbar_arrive(BAR(B_EMPTY + it % STAGES));
       const bool warp_live = __all_sync(0xffffffffu, live) && !*abort_flag;
       const long long grow = static_cast<long long>(rt) * 128 + row;
       const bool row_ok = grow < p.n_rows;
@@ -619,7 +646,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) {
+  if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem_base, Cfg::TMEM_COLS);
   }
