@@ -185,6 +185,14 @@ def block_transform(x: np.ndarray, T: np.ndarray) -> np.ndarray:
     return y.reshape(n, d)
 
 
+def transform_groups(x_groups: np.ndarray, T: np.ndarray, blocks: np.ndarray) -> np.ndarray:
+    """The same y = T_i x for a list of single (token, block) groups: row k of
+    ``x_groups`` ([k][G]) is the input group of block ``blocks[k]``; float64."""
+    xg = np.asarray(x_groups, dtype=np.float64)
+    Tb = np.asarray(T, dtype=np.float64)[np.asarray(blocks)]
+    return np.einsum("krc,kc->kr", Tb, xg)
+
+
 # ---------------------------------------------------------------------------
 # 4-bit grids and scale encodings
 # ---------------------------------------------------------------------------

@@ -30,9 +30,18 @@ def canon_codes(codes: np.ndarray, fmt: str, packed: bool = False) -> np.ndarray
     return c
 
 
-def assert_bit_exact(codes_gpu, scales_gpu, ts_gpu, y_gpu, fmt, G):
-    """Rule 1."""
-    c_o, s_o, ts_o = O.quantize(np.asarray(y_gpu, dtype=np.float64), fmt, G)
+def oracle_quantize(y, fmt, G, s_t=None):
+    """The oracle quantiser; for NVFP4 an explicit tensor scale replaces the one taken
+    from max |y| (used when y holds only sampled groups of a larger tensor)."""
+    y = np.asarray(y, dtype=np.float64)
+    if fmt == "nvfp4" and s_t is not None:
+        return O.quant_nvfp4(y, float(s_t))
+    return O.quantize(y, fmt, G)
+
+
+def assert_bit_exact(codes_gpu, scales_gpu, ts_gpu, y_gpu, fmt, G, s_t=None):
+    """Rule 1.  ``s_t``: the oracle's NVFP4 tensor scale when y is a sample."""
+    c_o, s_o, ts_o = oracle_quantize(y_gpu, fmt, G, s_t)
     c_g = canon_codes(codes_gpu, fmt, packed=True)
     c_o = canon_codes(c_o, fmt)
     if fmt == "nvfp4":
@@ -54,9 +63,10 @@ def group_scale_values(scales, fmt, G, ts):
     return s.astype(np.float64)
 
 
-def end_to_end_report(codes_gpu, scales_gpu, ts_gpu, y_ref, fmt, G):
-    """Rule 2 statistics: (rel_frob, flip_fraction, n_scale_groups_differing, max_steps)."""
-    c_o, s_o, ts_o = O.quantize(np.asarray(y_ref, dtype=np.float64), fmt, G)
+def end_to_end_report(codes_gpu, scales_gpu, ts_gpu, y_ref, fmt, G, s_t_ref=None):
+    """Rule 2 statistics: (rel_frob, flip_fraction, n_scale_groups_differing, max_steps).
+    ``s_t_ref``: the oracle's NVFP4 tensor scale when y_ref is a sample."""
+    c_o, s_o, ts_o = oracle_quantize(y_ref, fmt, G, s_t_ref)
     c_g = O.unpack_nibbles(codes_gpu)
     n, d = c_g.shape
     deq_g = O.dequant(c_g, scales_gpu, fmt, G, ts_gpu)
@@ -88,8 +98,8 @@ def end_to_end_report(codes_gpu, scales_gpu, ts_gpu, y_ref, fmt, G):
     return rel, flips / float(n * d), n_scale_diff, max_steps_same
 
 
-def assert_end_to_end(codes_gpu, scales_gpu, ts_gpu, y_ref, fmt, G):
-    rel, frac, nsd, mx = end_to_end_report(codes_gpu, scales_gpu, ts_gpu, y_ref, fmt, G)
+def assert_end_to_end(codes_gpu, scales_gpu, ts_gpu, y_ref, fmt, G, s_t_ref=None):
+    rel, frac, nsd, mx = end_to_end_report(codes_gpu, scales_gpu, ts_gpu, y_ref, fmt, G, s_t_ref)
     assert mx <= 1, f"a code differs by {mx} grid steps"
     assert rel <= REL_FROB_TOL, f"relative Frobenius error {rel:.3e} > {REL_FROB_TOL}"
     assert frac <= FLIP_FRAC_TOL, f"{frac:.3e} of codes differ (> {FLIP_FRAC_TOL}); {nsd} groups differ in scale"

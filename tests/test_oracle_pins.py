@@ -216,6 +216,21 @@ def test_block_transform_basis_vector_gives_column():
         assert np.array_equal(O.block_transform(e, T)[0], T[0][:, c])
 
 
+def test_transform_groups_basis_vectors_and_block_choice():
+    """Each sampled group uses its own block's matrix: basis vectors pick its columns,
+    and a group of ones gives that block's row sums (exact in float64 for small ints)."""
+    G, C = 4, 3
+    T = np.arange(C * G * G, dtype=float).reshape(C, G, G)
+    for blk in range(C):
+        for c in range(G):
+            e = np.zeros((1, G))
+            e[0, c] = 1.0
+            assert np.array_equal(O.transform_groups(e, T, np.array([blk]))[0], T[blk][:, c])
+    ones = np.ones((C, G))
+    y = O.transform_groups(ones, T, np.array([2, 0, 1]))
+    assert np.array_equal(y, np.stack([T[2].sum(axis=1), T[0].sum(axis=1), T[1].sum(axis=1)]))
+
+
 # ---------------------------------------------------------------- grids, brute force
 
 

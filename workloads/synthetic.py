@@ -111,7 +111,7 @@ def _activations(rng, wl: Workload, n: int, L: np.ndarray, chan: np.ndarray,
     for r0 in range(0, n, chunk):
         r1 = min(n, r0 + chunk)
         z = _base_draw(rng, wl.base, (r1 - r0, C, G))
-        u = np.einsum("cij,ncj->nci", L, z, optimize=True).reshape(r1 - r0, wl.d_in)
+        u = np.einsum("cij,ncj->nci", L, z).reshape(r1 - r0, wl.d_in)
         out[r0:r1] = bf16_bits_from_f64(u * chan[None, :])
     return out
 
