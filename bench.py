@@ -32,6 +32,7 @@ METRIC = "WUSH+quant GB/s & tokens/s at d=4096 G=32 MXFP4; % of HBM roofline"
 WORKLOAD = "attn_mxfp4_4096"
 N_SETS = 8
 GRAPH_LEN = 100
+H_STEPS = 5000       # launches of the H+Quant comparator timed after the main region
 FALLBACK_HBM_GBS = 6650.0
 PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "wush_fused_mxfp4_attn_4096.md")
 KERNEL_SOURCES = ("blockwise_adaptive_transforms_b200/csrc/wush_fused.cuh",
@@ -313,6 +314,42 @@ def run_native(args):
 
     per_launch_s = elapsed_s / args.steps
     value = job_throughput(world, args.steps, step_bytes, elapsed_s)
+
+    # H+Quant comparator: the same kernel with one shared G x G Hadamard matrix, same
+    # inputs, outputs and timing method (the pages compare the two fused kernels)
+    H = W.hadamard_matrix(G, dev)
+
+    def launch_h(i):
+        k = i % N_SETS
+        W.wush_quant_act_shared(xs[k], H, G, wl.fmt, codes=codes[k], scales=scales[k], stream=stream)
+
+    h_reps = max(1, min(args.steps, H_STEPS) // GRAPH_LEN)
+    with torch.cuda.stream(stream):
+        for i in range(8):
+            launch_h(i)
+        stream.synchronize()
+        graph_h = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph_h, stream=stream):
+            for i in range(GRAPH_LEN):
+                launch_h(i)
+        graph_h.replay()
+        stream.synchronize()
+        if world > 1:
+            dist.barrier()
+        h0 = torch.cuda.Event(enable_timing=True)
+        h1 = torch.cuda.Event(enable_timing=True)
+        h0.record(stream)
+        for _ in range(h_reps):
+            graph_h.replay()
+        h1.record(stream)
+        h1.synchronize()
+    h_elapsed = max_over_ranks(h0.elapsed_time(h1) / 1e3, dev)
+    h_per_launch_s = h_elapsed / (h_reps * GRAPH_LEN)
+    h_bytes = step_bytes - C * G * G * 4 + G * G * 4
+    st, bits = W.wush_device_status(stream)
+    if st != 0:
+        raise RuntimeError(f"device error word {bits:#x} after the H+Quant timing")
+    del graph_h
     tokens_s = world * args.steps * n / elapsed_s
     achieved = step_bytes / per_launch_s / 1e9
     peak, peak_kind = hbm_peak()
@@ -369,6 +406,11 @@ def run_native(args):
         "cpu_baseline": cpu,
         "e2e": {"value": round(e2e_value, 3), "unit": "GB/s", "h2d_bytes_per_step": n * d * 2,
                 "d2h_bytes_per_step": n * d // 2 + n * C, "steps": args.e2e_steps},
+        "h_quant": {"value": round(job_throughput(world, h_reps * GRAPH_LEN, h_bytes, h_elapsed), 2),
+                    "unit": "GB/s", "us_per_launch": round(h_per_launch_s * 1e6, 3),
+                    "launches": h_reps * GRAPH_LEN,
+                    "wush_time_over_h_time": round(per_launch_s / h_per_launch_s, 4),
+                    "what": "same fused kernel, one shared Hadamard matrix for every block"},
         "gpu_launches": args.steps,
         "clocks": clk,
     }

@@ -16,15 +16,17 @@ import torch
 from ._build import LIB_PATH, build as build_library  # noqa: F401
 
 __all__ = ["FMT", "WushError", "wush_quant_act", "wush_quant_weight", "wush_quant_act_debug",
-           "wush_quant_weight_debug", "wush_build_transforms", "wush_device_status", "wush_set_wait_limit_ns",
+           "wush_quant_weight_debug", "wush_quant_act_shared", "wush_quant_act_shared_debug",
+           "wush_build_transforms", "wush_device_status", "wush_set_wait_limit_ns",
            "wush_selftest_wait_timeout", "wush_status_string", "wush_version", "load_library",
-           "EXPORTED_SYMBOLS", "output_shapes"]
+           "EXPORTED_SYMBOLS", "output_shapes", "hadamard_matrix"]
 
 FMT = {"mxfp4": 0, "nvfp4": 1, "int4": 2}
 STATUS = {0: "WUSH_OK", 1: "WUSH_ERR_INVALID_ARG", 2: "WUSH_ERR_UNSUPPORTED", 3: "WUSH_ERR_MISALIGNED",
           4: "WUSH_ERR_CUDA", 5: "WUSH_ERR_DEVICE_TIMEOUT"}
 EXPORTED_SYMBOLS = ("wush_quant_act", "wush_quant_weight", "wush_quant_act_debug",
-                    "wush_quant_weight_debug", "wush_build_transforms", "wush_device_status",
+                    "wush_quant_weight_debug", "wush_quant_act_shared", "wush_quant_act_shared_debug",
+                    "wush_build_transforms", "wush_device_status",
                     "wush_set_wait_limit_ns",
                     "wush_selftest_wait_timeout", "wush_status_string", "wush_version")
 
@@ -51,10 +53,13 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
     quant = [_P, _P, _I64, _I64, _I32, _I32, _P, _P, _P, _P]
     lib.wush_quant_act.argtypes = quant
     lib.wush_quant_weight.argtypes = quant
+    lib.wush_quant_act_shared.argtypes = quant
     dbg = [_P, _P, _I64, _I64, _I32, _I32, _P, _P, _P, _P, _P]
     lib.wush_quant_act_debug.argtypes = dbg
     lib.wush_quant_weight_debug.argtypes = dbg
-    for f in ("wush_quant_act", "wush_quant_weight", "wush_quant_act_debug", "wush_quant_weight_debug"):
+    lib.wush_quant_act_shared_debug.argtypes = dbg
+    for f in ("wush_quant_act", "wush_quant_weight", "wush_quant_act_debug", "wush_quant_weight_debug",
+              "wush_quant_act_shared", "wush_quant_act_shared_debug"):
         getattr(lib, f).restype = ctypes.c_int
     lib.wush_build_transforms.argtypes = [_P, _P, _I64, _I64, _I64, _I32, ctypes.c_double, _I32,
                                           _P, _P, _P, _P, _P, _P]
@@ -128,7 +133,7 @@ def _ptr(t):
     return None if t is None else t.data_ptr()
 
 
-def _call(fn_name, inp, in_dtype, T, G, fmt, codes, scales, tensor_scale, y, stream):
+def _call(fn_name, inp, in_dtype, T, G, fmt, codes, scales, tensor_scale, y, stream, shared=False):
     lib = load_library()
     _check_dev(inp, "input", in_dtype)
     _check_dev(T, "T", torch.float32)
@@ -137,8 +142,9 @@ def _call(fn_name, inp, in_dtype, T, G, fmt, codes, scales, tensor_scale, y, str
     rows, d_in = int(inp.shape[0]), int(inp.shape[1])
     if d_in % G:
         raise ValueError("d_in must be a multiple of G")
-    if tuple(T.shape) != (d_in // G, G, G):
-        raise ValueError(f"T must have shape {(d_in // G, G, G)}")
+    t_shape = (G, G) if shared else (d_in // G, G, G)
+    if tuple(T.shape) != t_shape:
+        raise ValueError(f"T must have shape {t_shape}")
     codes, scales, tensor_scale = _alloc_outputs(inp, rows, d_in, G, fmt, codes, scales, tensor_scale)
     args = [_ptr(inp), _ptr(T), rows, d_in, int(G), _fmt_code(fmt), _ptr(codes), _ptr(scales),
             _ptr(tensor_scale)]
@@ -182,6 +188,30 @@ def wush_quant_weight_debug(w, T, G, fmt, y_out=None, stream=None):
     y = _y_buffer(w, y_out)
     c, s, ts = _call("wush_quant_weight_debug", w, torch.float32, T, G, fmt, None, None, None, y, stream)
     return c, s, ts, y
+
+
+def wush_quant_act_shared(x, T, G, fmt, codes=None, scales=None, tensor_scale=None, stream=None):
+    """H+Quant comparator: every block uses the one fp32 [G][G] matrix T (e.g. Hadamard)."""
+    return _call("wush_quant_act_shared", x, torch.bfloat16, T, G, fmt, codes, scales, tensor_scale, None, stream,
+                 shared=True)
+
+
+def wush_quant_act_shared_debug(x, T, G, fmt, y_out=None, stream=None):
+    y = _y_buffer(x, y_out)
+    c, s, ts = _call("wush_quant_act_shared_debug", x, torch.bfloat16, T, G, fmt, None, None, None, y, stream,
+                     shared=True)
+    return c, s, ts, y
+
+
+def hadamard_matrix(G, device=None):
+    """The normalised Sylvester Hadamard matrix of order G (entries +-G^-1/2, H H^T = I)
+    as an fp32 [G][G] tensor: the shared matrix of the H+Quant comparator."""
+    if G < 1 or G & (G - 1):
+        raise ValueError("G must be a power of two")
+    H = torch.ones((1, 1), dtype=torch.float64)
+    while H.shape[0] < G:
+        H = torch.cat([torch.cat([H, H], 1), torch.cat([H, -H], 1)], 0)
+    return (H / G ** 0.5).to(torch.float32).to(device if device is not None else "cuda")
 
 
 def wush_build_transforms(w, xcal, G, lam=0.01, use_hadamard=True, want_f64=False, stream=None):

@@ -97,20 +97,20 @@ int launch_fused(const CUtensorMap& map, const CUtensorMap& cmap, wush::FusedPar
   return cudaGetLastError() == cudaSuccess ? WUSH_OK : WUSH_ERR_CUDA;
 }
 
-template <int G, int FMT, bool IN_F32, bool AMAX_ONLY>
+template <int G, int FMT, bool IN_F32, bool AMAX_ONLY, bool SHARED>
 int launch_pick_y(const CUtensorMap& map, const CUtensorMap& cmap, const wush::FusedParams& p, bool emit_y,
                   cudaStream_t s) {
-  if (emit_y) return launch_fused<wush::FusedCfg<G, FMT, IN_F32, AMAX_ONLY, true>>(map, cmap, p, s);
-  return launch_fused<wush::FusedCfg<G, FMT, IN_F32, AMAX_ONLY, false>>(map, cmap, p, s);
+  if (emit_y) return launch_fused<wush::FusedCfg<G, FMT, IN_F32, AMAX_ONLY, true, SHARED>>(map, cmap, p, s);
+  return launch_fused<wush::FusedCfg<G, FMT, IN_F32, AMAX_ONLY, false, SHARED>>(map, cmap, p, s);
 }
 
-template <bool IN_F32>
+template <bool IN_F32, bool SHARED>
 int dispatch(const CUtensorMap& map, const CUtensorMap& cmap, wush::FusedParams p, int G, int fmt, bool emit_y,
              float* tensor_scale, cudaStream_t s) {
-  if (fmt == WUSH_MXFP4) return launch_pick_y<32, wush::kMXFP4, IN_F32, false>(map, cmap, p, emit_y, s);
+  if (fmt == WUSH_MXFP4) return launch_pick_y<32, wush::kMXFP4, IN_F32, false, SHARED>(map, cmap, p, emit_y, s);
   if (fmt == WUSH_INT4) {
-    if (G == 32) return launch_pick_y<32, wush::kINT4, IN_F32, false>(map, cmap, p, emit_y, s);
-    return launch_pick_y<16, wush::kINT4, IN_F32, false>(map, cmap, p, emit_y, s);
+    if (G == 32) return launch_pick_y<32, wush::kINT4, IN_F32, false, SHARED>(map, cmap, p, emit_y, s);
+    return launch_pick_y<16, wush::kINT4, IN_F32, false, SHARED>(map, cmap, p, emit_y, s);
   }
   // NVFP4: pass 1 finds amax|y| (float bits, running max in *tensor_scale), a one-thread
   // kernel turns it into s_t in place, pass 2 quantises with s_t.
@@ -118,17 +118,17 @@ int dispatch(const CUtensorMap& map, const CUtensorMap& cmap, wush::FusedParams 
   wush::FusedParams p1 = p;
   p1.amax_word = reinterpret_cast<unsigned int*>(tensor_scale);
   p1.codes_via_tma = 0;
-  int st = launch_fused<wush::FusedCfg<16, wush::kNVFP4, IN_F32, true, false>>(map, cmap, p1, s);
+  int st = launch_fused<wush::FusedCfg<16, wush::kNVFP4, IN_F32, true, false, SHARED>>(map, cmap, p1, s);
   if (st != WUSH_OK) return st;
   wush::wush_nvfp4_tensor_scale_kernel<<<1, 32, 0, s>>>(tensor_scale);
   if (cudaGetLastError() != cudaSuccess) return WUSH_ERR_CUDA;
   p.tensor_scale = tensor_scale;
-  return launch_pick_y<16, wush::kNVFP4, IN_F32, false>(map, cmap, p, emit_y, s);
+  return launch_pick_y<16, wush::kNVFP4, IN_F32, false, SHARED>(map, cmap, p, emit_y, s);
 }
 
 int quant_common(const void* in, bool in_f32, const float* T, int64_t rows, int64_t d_in, int G, int fmt,
                  uint8_t* codes, void* scales, float* tensor_scale, float* y_out, bool debug,
-                 wush_stream_t stream) {
+                 wush_stream_t stream, bool shared_T = false) {
   if (fmt != WUSH_MXFP4 && fmt != WUSH_NVFP4 && fmt != WUSH_INT4) return WUSH_ERR_UNSUPPORTED;
   const bool g_ok = (fmt == WUSH_MXFP4 && G == 32) || (fmt == WUSH_NVFP4 && G == 16) ||
                     (fmt == WUSH_INT4 && (G == 16 || G == 32));
@@ -181,8 +181,9 @@ int quant_common(const void* in, bool in_f32, const float* T, int64_t rows, int6
   p.total_tiles = static_cast<int>(n_row_tiles * n_col_tiles);
   p.wait_limit_ns = g_wait_limit_ns.load(std::memory_order_relaxed);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  return in_f32 ? dispatch<true>(map, cmap, p, G, fmt, debug, tensor_scale, s)
-                : dispatch<false>(map, cmap, p, G, fmt, debug, tensor_scale, s);
+  if (shared_T) return dispatch<false, true>(map, cmap, p, G, fmt, debug, tensor_scale, s);
+  return in_f32 ? dispatch<true, false>(map, cmap, p, G, fmt, debug, tensor_scale, s)
+                : dispatch<false, false>(map, cmap, p, G, fmt, debug, tensor_scale, s);
 }
 
 }  // namespace
@@ -212,6 +213,19 @@ int wush_quant_weight_debug(const float* w_f32, const float* T_blocks, int64_t d
                             wush_stream_t stream) {
   return quant_common(w_f32, true, T_blocks, d_out, d_in, G, fmt, codes, scales, tensor_scale, y_out, true,
                       stream);
+}
+
+int wush_quant_act_shared(const void* x_bf16, const float* T_shared, int64_t n_tok, int64_t d_in, int G, int fmt,
+                          uint8_t* codes, void* scales, float* tensor_scale, wush_stream_t stream) {
+  return quant_common(x_bf16, false, T_shared, n_tok, d_in, G, fmt, codes, scales, tensor_scale, nullptr, false,
+                      stream, true);
+}
+
+int wush_quant_act_shared_debug(const void* x_bf16, const float* T_shared, int64_t n_tok, int64_t d_in, int G,
+                                int fmt, uint8_t* codes, void* scales, float* tensor_scale, float* y_out,
+                                wush_stream_t stream) {
+  return quant_common(x_bf16, false, T_shared, n_tok, d_in, G, fmt, codes, scales, tensor_scale, y_out, true,
+                      stream, true);
 }
 
 int wush_build_transforms(const float* w_f32, const void* xcal_bf16, int64_t d_out, int64_t n_cal, int64_t d_in,

@@ -10,9 +10,9 @@
 //  * persistent CTAs, one per SM, each owning a contiguous run of 128-row x CH-channel
 //    tiles, column-tile major so consecutive tiles share their transforms;
 //  * warp 0 streams the input tiles with TMA (128-byte swizzle) through a STAGES-deep
-//    mbarrier ring; warps 2-3 split each fp32 T_i into bf16 hi and lo and stack them
-//    along N in shared memory (for fp32 weights they also split each staged weight
-//    tile into bf16 hi + lo operands);
+//    mbarrier ring and bulk-copies each column tile's fp32 matrices into a transform
+//    slot; warps 2-3 split them in place into bf16 hi and lo, stacked along N (for fp32
+//    weights they also split each staged weight tile into bf16 hi + lo operands);
 //  * warp 1 issues tcgen05.mma (M=128, N=2G, K=16) into fp32 TMEM accumulators,
 //    double-buffered: one MMA per block and K-step yields X*T_hi^T and X*T_lo^T side
 //    by side (fp32 weights add W_lo*T_hi^T into the first half; the dropped W_lo*T_lo
@@ -57,10 +57,13 @@ struct FusedParams {
   unsigned long long wait_limit_ns;
 };
 
-template <int G_, int FMT_, bool IN_F32_, bool AMAX_ONLY_, bool EMIT_Y_>
+template <int G_, int FMT_, bool IN_F32_, bool AMAX_ONLY_, bool EMIT_Y_, bool SHARED_T_ = false>
 struct FusedCfg {
   static constexpr int G = G_;
   static constexpr int FMT = FMT_;
+  // SHARED_T: one G x G matrix for every block (the H+Quant comparator); it is converted
+  // once per CTA and the transform slot is never refilled
+  static constexpr bool SHARED_T = SHARED_T_;
   static constexpr bool IN_F32 = IN_F32_;
   static constexpr bool AMAX_ONLY = AMAX_ONLY_;
   static constexpr bool EMIT_Y = EMIT_Y_;
@@ -91,11 +94,13 @@ struct FusedCfg {
   static constexpr int OFF_T = OFF_OPER + (IN_F32 ? 2 * 2 * OPER_BYTES : 0);
   static constexpr int OFF_CODES = OFF_T + 2 * TSLOT_BYTES;   // [group][2] code staging buffers
   static constexpr int OFF_BAR = OFF_CODES + N_GROUPS * 2 * CODE_STAGE;
-  // barriers: full[S], empty[S], ofull[2], oempty[2], tfull[2], tempty[2], afull[NACC], aempty[NACC], drain
-  static constexpr int N_BARS = 2 * STAGES + 9 + 2 * NACC;
+  // barriers: full[S], empty[S], ofull[2], oempty[2], tfull[2], tempty[2], afull[NACC], aempty[NACC], drain,
+  // tload[2], tread[2]
+  static constexpr int N_BARS = 2 * STAGES + 13 + 2 * NACC;
   static constexpr int OFF_MISC = OFF_BAR + 8 * N_BARS;
   static constexpr int SMEM_BYTES = OFF_MISC + 64 + 1024;   // + alignment slack
   static_assert(G == 16 || G == 32, "G must be 16 or 32");
+  static_assert(!(SHARED_T && IN_F32), "the shared-matrix variant is an activation path");
   static_assert(!(FMT == kMXFP4 && G != 32) && !(FMT == kNVFP4 && G != 16), "format/group mismatch");
   static_assert(TMEM_COLS <= 512, "TMEM columns");
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
@@ -251,7 +256,8 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
   auto BAR = [&](int i) -> uint32_t { return bar0 + 8u * static_cast<uint32_t>(i); };
   const int B_FULL = 0, B_EMPTY = STAGES, B_OFULL = 2 * STAGES, B_OEMPTY = 2 * STAGES + 2,
             B_TFULL = 2 * STAGES + 4, B_TEMPTY = 2 * STAGES + 6, B_AFULL = 2 * STAGES + 8,
-            B_AEMPTY = 2 * STAGES + 8 + Cfg::NACC, B_DRAIN = 2 * STAGES + 8 + 2 * Cfg::NACC;
+            B_AEMPTY = 2 * STAGES + 8 + Cfg::NACC, B_DRAIN = 2 * STAGES + 8 + 2 * Cfg::NACC,
+            B_TLOAD = B_DRAIN + 1, B_TREAD = B_DRAIN + 3;
   constexpr int NACC = Cfg::NACC;
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + Cfg::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::OFF_MISC + 4);
@@ -278,6 +284,10 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
       mbar_init(BAR(B_AEMPTY + k), Cfg::GROUP_WARPS);
     }
     mbar_init(BAR(B_DRAIN), 1);
+    for (int k = 0; k < 2; ++k) {
+      mbar_init(BAR(B_TLOAD + k), 1);
+      mbar_init(BAR(B_TREAD + k), 64);
+    }
     *abort_flag = 0;
     fence_barrier_init();
     tma_prefetch_desc(&tmap_in);
@@ -287,32 +297,32 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
   // of the previous kernel in the stream; its results are visible only after this wait.
   grid_dependency_wait();
   grid_launch_dependents();
-  // The converter warps issue the loads of the first column tile's transforms before any
-  // input tile is requested (behind the input burst they would wait microseconds), then
-  // the producer starts streaming before the rest of the CTA is set up.
-  // One column tile's transforms: BPT blocks x G rows x (G/8) chunks of 8 values;
-  // converter id v (0..63) takes chunks v, v + 64, ...
-  constexpr int T_CHUNKS = BPT * G * (G / 8);
-  constexpr int T_PER_THREAD = (T_CHUNKS + 63) / 64;
-  float4 tpre[T_PER_THREAD][2];
-  auto load_T = [&](int ct, int v, float4 (&u)[T_PER_THREAD][2]) {
+  // A column tile's matrices (BPT blocks x G x G fp32, contiguous in global memory) reach
+  // their transform slot by one bulk copy; the converter warps then split them in place
+  // into the bf16 hi/lo panels.
+  constexpr int T_CHUNKS = BPT * G * (G / 8);            // 8-value chunks of one column tile
+  constexpr int T_PER_THREAD = (T_CHUNKS + 63) / 64;    // converter id v takes v, v + 64, ...
+  auto t_copy = [&](int ct, int slot) {                  // one thread
+    const int nblk = Cfg::SHARED_T ? 1 : min(BPT, p.C - ct * BPT);
+    const uint32_t bytes = static_cast<uint32_t>(nblk * G * G * 4);
+    const float* src = p.T + (Cfg::SHARED_T ? 0ll : static_cast<long long>(ct) * BPT * G * G);
+    mbar_arrive_expect_tx(BAR(B_TLOAD + slot), bytes);
+    bulk_load_1d(sbase + Cfg::OFF_T + slot * Cfg::TSLOT_BYTES, src, bytes, BAR(B_TLOAD + slot));
+  };
+  // raw fp32 chunks of a slot -> registers
+  auto read_T = [&](int v, const uint8_t* slot_raw, float4 (&u)[T_PER_THREAD][2]) {
 #pragma unroll
     for (int k = 0; k < T_PER_THREAD; ++k) {
       const int q = v + 64 * k;
-      const int b = q / (G * (G / 8));
-      const int rem = q - b * (G * (G / 8));
-      const int r = rem / (G / 8), j = rem - r * (G / 8);
-      const int blk = ct * BPT + b;
-      if (q < T_CHUNKS && blk < p.C) {
-        const float4* src = reinterpret_cast<const float4*>(p.T + (static_cast<long long>(blk) * G + r) * G + 8 * j);
-        u[k][0] = __ldg(src);
-        u[k][1] = __ldg(src + 1);
-      } else {
-        u[k][0] = u[k][1] = make_float4(0.f, 0.f, 0.f, 0.f);
+      const int qs = Cfg::SHARED_T ? q % (G * (G / 8)) : q;   // shared: every block reads the one matrix
+      if (q < T_CHUNKS) {
+        const float4* src = reinterpret_cast<const float4*>(slot_raw + qs * 32);
+        u[k][0] = src[0];
+        u[k][1] = src[1];
       }
     }
   };
-  // hi/lo split of loaded chunks into the K-major SW128 panels of a transform slot
+  // hi/lo split of the chunks into the K-major SW128 panels of the slot
   auto store_T = [&](int v, const float4 (&u)[T_PER_THREAD][2], uint8_t* tdst) {
 #pragma unroll
     for (int k = 0; k < T_PER_THREAD; ++k) {
@@ -331,20 +341,32 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
       *reinterpret_cast<uint4*>(panel + sw128_off(G + r, c)) = lo;
     }
   };
-  if ((warp == 2 || warp == 3) && t_begin < t_end) load_T(t_begin / nrt, threadIdx.x - 64, tpre);
-  if (warp == 0 || warp == 2 || warp == 3) named_bar_sync(3, 96);
+  // Thread 0, which initialised the barriers, issues the first input tile, then the
+  // transform copies of the CTA's first (and, if its tiles reach it, second) column tile,
+  // then the remaining input stages (this order measured fastest: the first tile and its
+  // matrices arrive together, ahead of the rest of the burst).  Every converter thread
+  // knows which copies exist.
+  const bool t_second = !Cfg::SHARED_T && t_begin < t_end && (t_end - 1) / nrt > t_begin / nrt;
+  int t_issued[2] = {t_begin < t_end ? 1 : 0, t_second ? 1 : 0};
   const uint64_t l2_pol = l2_policy_evict_first();
   int n_preloaded = 0;
   if (threadIdx.x == 0) {
-    for (; n_preloaded < STAGES && t_begin + n_preloaded < t_end; ++n_preloaded) {
-      const int t = t_begin + n_preloaded;
-      const int ct = t / nrt, rt = t - ct * nrt;
-      const uint32_t dst = sbase + Cfg::OFF_STAGE + n_preloaded * Cfg::STAGE_BYTES;
-      mbar_arrive_expect_tx(BAR(B_FULL + n_preloaded), Cfg::STAGE_BYTES);
+    auto issue_x = [&]() {
+      if (n_preloaded < STAGES && t_begin + n_preloaded < t_end) {
+        const int t = t_begin + n_preloaded;
+        const int ct = t / nrt, rt = t - ct * nrt;
+        const uint32_t dst = sbase + Cfg::OFF_STAGE + n_preloaded * Cfg::STAGE_BYTES;
+        mbar_arrive_expect_tx(BAR(B_FULL + n_preloaded), Cfg::STAGE_BYTES);
 #pragma unroll
-      for (int s = 0; s < Cfg::SUB; ++s)
-        tma_load_2d(dst + s * 16384, &tmap_in, BAR(B_FULL + n_preloaded), ct * CH + 64 * s, rt * 128, l2_pol);
-    }
+        for (int s = 0; s < Cfg::SUB; ++s)
+          tma_load_2d(dst + s * 16384, &tmap_in, BAR(B_FULL + n_preloaded), ct * CH + 64 * s, rt * 128, l2_pol);
+        ++n_preloaded;
+      }
+    };
+    issue_x();
+    if (t_begin < t_end) t_copy(t_begin / nrt, 0);
+    if (t_second) t_copy(t_begin / nrt + 1, 1);
+    while (n_preloaded < STAGES && t_begin + n_preloaded < t_end) issue_x();
   }
   __syncwarp();
   if (warp == 1) {
@@ -407,7 +429,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
       int ct = t_begin / nrt, rt = t_begin - (t_begin / nrt) * nrt;
       uint64_t db = db_slot0;
       for (int t = t_begin; t < t_end; ++t, ++it) {
-        if (ct != prev_ct) {
+        if (Cfg::SHARED_T ? it == 0 : ct != prev_ct) {
           ++epoch;
           prev_ct = ct;
           db = db_slot0 + ((epoch & 1) ? static_cast<uint64_t>(Cfg::TSLOT_BYTES >> 4) : 0ull);
@@ -436,7 +458,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
         }
         umma_commit(BAR(B_AFULL + acc));
         if (Cfg::IN_F32) umma_commit(BAR(B_OEMPTY + buf));
-        if (t + 1 == t_end || rt + 1 == nrt) umma_commit(BAR(B_TEMPTY + (epoch & 1)));
+        if (!Cfg::SHARED_T && (t + 1 == t_end || rt + 1 == nrt)) umma_commit(BAR(B_TEMPTY + (epoch & 1)));
         if (++rt == nrt) rt = 0, ++ct;
         if (++buf == NBUF) {
           buf = 0, phase ^= 1u, da_hi = da_first, full_bar = full_first;
@@ -452,25 +474,29 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
   } else if (warp < 4) {
     // ------------------------------------------------------------ converters (64 threads)
     const int v0 = threadIdx.x - 64;
+    int t_landed[2] = {0, 0};
     int epoch = -1, prev_ct = -1;
     int stage = 0, obuf = 0;
     uint32_t phase = 0, ophase = 0;
     for (int t = t_begin; t < t_end; ++t) {
       const int ct = t / nrt;
-      if (ct != prev_ct) {
+      if (Cfg::SHARED_T ? t == t_begin : ct != prev_ct) {
         ++epoch;
         prev_ct = ct;
         const int slot = epoch & 1;
-        if (!wait_bounded(BAR(B_TEMPTY + slot), static_cast<uint32_t>(((epoch >> 1) & 1) ^ 1), abort_flag, 4u, lim)) break;
         uint8_t* tdst = smem + Cfg::OFF_T + slot * Cfg::TSLOT_BYTES;
-        // the first column tile's values were loaded before the set-up, later ones here
-        float4 u[T_PER_THREAD][2];
-        if (epoch == 0) {
-#pragma unroll
-          for (int k = 0; k < T_PER_THREAD; ++k) u[k][0] = tpre[k][0], u[k][1] = tpre[k][1];
-        } else {
-          load_T(ct, v0, u);
+        const uint32_t par = static_cast<uint32_t>((epoch >> 1) & 1);
+        if (epoch >= 2) {     // the first two copies were issued at the start
+          if (!wait_bounded(BAR(B_TEMPTY + slot), par ^ 1u, abort_flag, 4u, lim)) break;
+          if (v0 == 0) t_copy(ct, slot), ++t_issued[slot];
         }
+        if (!wait_bounded(BAR(B_TLOAD + slot), par, abort_flag, 4u, lim)) break;
+        ++t_landed[slot];
+        float4 u[T_PER_THREAD][2];
+        read_T(v0, tdst, u);
+        // every raw chunk of the slot is in registers before any panel overwrites it
+        mbar_arrive(BAR(B_TREAD + slot));
+        if (!wait_bounded(BAR(B_TREAD + slot), par, abort_flag, 4u, lim)) break;
         store_T(v0, u, tdst);
         fence_proxy_async_smem();
         mbar_arrive(BAR(B_TFULL + slot));
@@ -499,6 +525,12 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
         if (++stage == STAGES) stage = 0, phase ^= 1u;
         if (++obuf == 2) obuf = 0, ophase ^= 1u;
       }
+    }
+    if (v0 == 0) {   // an aborted run still lets its transform copies land before the CTA exits
+      volatile int no_abort = 0;
+      for (int sl = 0; sl < 2; ++sl)
+        for (; t_landed[sl] < t_issued[sl]; ++t_landed[sl])
+          wait_bounded(BAR(B_TLOAD + sl), static_cast<uint32_t>(t_landed[sl] & 1), &no_abort, 4u, lim);
     }
   } else {
     // ------------------------------------------------------------ epilogue: 2 groups x 4 warps

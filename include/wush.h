@@ -106,6 +106,22 @@ int wush_quant_weight_debug(const float* w_f32, const float* T_blocks, int64_t d
                             int G, int fmt, uint8_t* codes, void* scales, float* tensor_scale,
                             float* y_out, wush_stream_t stream);
 
+/* H+Quant comparator: the same fused kernel with ONE G x G matrix shared by every block
+ * (the pages' uniform blockwise Hadamard baseline "H + Quant", against which the fused
+ * per-block WUSH kernel is compared: paper-graph-ui analysis, section 3.4.7 "GPU Kernel
+ * Design" and section 5 "GPU Kernel Benchmarks (Figure 2)").
+ *   y[t, iG + r] = sum_c T_shared[r, c] x[t, iG + c]   for every block i,
+ * then the same quantisers, layouts, tensor-scale handling and errors as wush_quant_act.
+ * T_shared: fp32 [G][G] row-major (device memory, 16-byte aligned), e.g. the normalised
+ * Sylvester Hadamard matrix rounded to fp32.  The matrix is converted once per CTA and
+ * stays resident in shared memory.  The _debug form also writes the fp32 y it quantised. */
+int wush_quant_act_shared(const void* x_bf16, const float* T_shared, int64_t n_tok, int64_t d_in,
+                          int G, int fmt, uint8_t* codes, void* scales, float* tensor_scale,
+                          wush_stream_t stream);
+int wush_quant_act_shared_debug(const void* x_bf16, const float* T_shared, int64_t n_tok,
+                                int64_t d_in, int G, int fmt, uint8_t* codes, void* scales,
+                                float* tensor_scale, float* y_out, wush_stream_t stream);
+
 /* Transform construction for one layer, on the device, in fp64 (one CTA per block).
  * Sources: paper-graph-ui analysis, section 3.2 "Second-Moment Computer" and "Transform
  * Constructor", sections 3.4.2 and 3.4.4 (Eq. 8); papernotes.org summary, "关键设计";
