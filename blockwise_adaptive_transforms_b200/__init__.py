@@ -19,14 +19,14 @@ __all__ = ["FMT", "WushError", "wush_quant_act", "wush_quant_weight", "wush_quan
            "wush_quant_weight_debug", "wush_quant_act_shared", "wush_quant_act_shared_debug",
            "wush_build_transforms", "wush_device_status", "wush_set_wait_limit_ns",
            "wush_selftest_wait_timeout", "wush_status_string", "wush_version", "load_library",
-           "EXPORTED_SYMBOLS", "output_shapes", "hadamard_matrix"]
+           "EXPORTED_SYMBOLS", "output_shapes", "hadamard_matrix", "wush_dequant"]
 
 FMT = {"mxfp4": 0, "nvfp4": 1, "int4": 2}
 STATUS = {0: "WUSH_OK", 1: "WUSH_ERR_INVALID_ARG", 2: "WUSH_ERR_UNSUPPORTED", 3: "WUSH_ERR_MISALIGNED",
           4: "WUSH_ERR_CUDA", 5: "WUSH_ERR_DEVICE_TIMEOUT"}
 EXPORTED_SYMBOLS = ("wush_quant_act", "wush_quant_weight", "wush_quant_act_debug",
                     "wush_quant_weight_debug", "wush_quant_act_shared", "wush_quant_act_shared_debug",
-                    "wush_build_transforms", "wush_device_status",
+                    "wush_dequant", "wush_build_transforms", "wush_device_status",
                     "wush_set_wait_limit_ns",
                     "wush_selftest_wait_timeout", "wush_status_string", "wush_version")
 
@@ -61,6 +61,8 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
     for f in ("wush_quant_act", "wush_quant_weight", "wush_quant_act_debug", "wush_quant_weight_debug",
               "wush_quant_act_shared", "wush_quant_act_shared_debug"):
         getattr(lib, f).restype = ctypes.c_int
+    lib.wush_dequant.argtypes = [_P, _P, _P, _I64, _I64, _I32, _I32, _P, _P]
+    lib.wush_dequant.restype = ctypes.c_int
     lib.wush_build_transforms.argtypes = [_P, _P, _I64, _I64, _I64, _I32, ctypes.c_double, _I32,
                                           _P, _P, _P, _P, _P, _P]
     lib.wush_build_transforms.restype = ctypes.c_int
@@ -201,6 +203,32 @@ def wush_quant_act_shared_debug(x, T, G, fmt, y_out=None, stream=None):
     c, s, ts = _call("wush_quant_act_shared_debug", x, torch.bfloat16, T, G, fmt, None, None, None, y, stream,
                      shared=True)
     return c, s, ts, y
+
+
+def wush_dequant(codes, scales, tensor_scale, G, fmt, out=None, stream=None):
+    """fp32 values [rows][d_in] represented by codes (u8 [rows][d_in/2]) and scales."""
+    lib = load_library()
+    _check_dev(codes, "codes", torch.uint8)
+    if codes.dim() != 2:
+        raise ValueError("codes must be 2-D [rows][d_in/2]")
+    rows, d_in = int(codes.shape[0]), 2 * int(codes.shape[1])
+    cs, ss, sdt = output_shapes(rows, d_in, G, fmt)
+    _check_dev(scales, "scales", sdt)
+    if tuple(scales.shape) != ss:
+        raise ValueError(f"scales must have shape {ss}")
+    if tensor_scale is not None:
+        _check_dev(tensor_scale, "tensor_scale", torch.float32)
+    if out is None:
+        out = torch.empty((rows, d_in), dtype=torch.float32, device=codes.device)
+    _check_dev(out, "out", torch.float32)
+    if tuple(out.shape) != (rows, d_in):
+        raise ValueError("out must be [rows][d_in]")
+    with torch.cuda.device(codes.device):
+        st = lib.wush_dequant(_ptr(codes), _ptr(scales), _ptr(tensor_scale), rows, d_in, int(G), _fmt_code(fmt),
+                              _ptr(out), _stream_handle(stream))
+    if st != 0:
+        raise WushError(st, "wush_dequant")
+    return out
 
 
 def hadamard_matrix(G, device=None):

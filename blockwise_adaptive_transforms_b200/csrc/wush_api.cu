@@ -13,6 +13,7 @@
 #include "wush.h"
 #include "wush_fused.cuh"
 #include "wush_build.cuh"
+#include "wush_dequant.cuh"
 
 namespace wush {
 // Waits on an mbarrier that no thread ever arrives on; the bounded wait must give up.
@@ -226,6 +227,35 @@ int wush_quant_act_shared_debug(const void* x_bf16, const float* T_shared, int64
                                 wush_stream_t stream) {
   return quant_common(x_bf16, false, T_shared, n_tok, d_in, G, fmt, codes, scales, tensor_scale, y_out, true,
                       stream, true);
+}
+
+int wush_dequant(const uint8_t* codes, const void* scales, const float* tensor_scale, int64_t rows, int64_t d_in,
+                 int G, int fmt, float* out, wush_stream_t stream) {
+  if (fmt != WUSH_MXFP4 && fmt != WUSH_NVFP4 && fmt != WUSH_INT4) return WUSH_ERR_UNSUPPORTED;
+  const bool g_ok = (fmt == WUSH_MXFP4 && G == 32) || (fmt == WUSH_NVFP4 && G == 16) ||
+                    (fmt == WUSH_INT4 && (G == 16 || G == 32));
+  if (!g_ok) return WUSH_ERR_UNSUPPORTED;
+  if (rows < 0 || d_in <= 0 || d_in % G != 0 || d_in > INT_MAX) return WUSH_ERR_INVALID_ARG;
+  if (rows == 0) return WUSH_OK;
+  if (!codes || !scales || !out || (fmt == WUSH_NVFP4 && !tensor_scale)) return WUSH_ERR_INVALID_ARG;
+  if (!aligned(codes, 4) || !aligned(out, 16) || (fmt == WUSH_INT4 && !aligned(scales, 4)) ||
+      (tensor_scale && !aligned(tensor_scale, 4)))
+    return WUSH_ERR_MISALIGNED;
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return WUSH_ERR_CUDA;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return WUSH_ERR_CUDA;
+  const long long n_words = rows * (d_in / 8);
+  const long long want = (n_words + 255) / 256;
+  const int grid = static_cast<int>(want < 8LL * sms ? want : 8LL * sms);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int di = static_cast<int>(d_in);
+  if (fmt == WUSH_MXFP4)
+    wush::wush_dequant_kernel<wush::kMXFP4><<<grid, 256, 0, s>>>(codes, scales, tensor_scale, rows, di, G, out);
+  else if (fmt == WUSH_NVFP4)
+    wush::wush_dequant_kernel<wush::kNVFP4><<<grid, 256, 0, s>>>(codes, scales, tensor_scale, rows, di, G, out);
+  else
+    wush::wush_dequant_kernel<wush::kINT4><<<grid, 256, 0, s>>>(codes, scales, tensor_scale, rows, di, G, out);
+  return cudaGetLastError() == cudaSuccess ? WUSH_OK : WUSH_ERR_CUDA;
 }
 
 int wush_build_transforms(const float* w_f32, const void* xcal_bf16, int64_t d_out, int64_t n_cal, int64_t d_in,

@@ -122,6 +122,17 @@ int wush_quant_act_shared_debug(const void* x_bf16, const float* T_shared, int64
                                 int64_t d_in, int G, int fmt, uint8_t* codes, void* scales,
                                 float* tensor_scale, float* y_out, wush_stream_t stream);
 
+/* Dequantisation: codes + scales (the layouts written by the calls above) -> fp32
+ * values out [rows][d_in] (device memory, 16-byte aligned; codes 4-byte aligned).
+ *   MXFP4: e2m1 * 2^(scale - 127);  NVFP4: e2m1 * e4m3(scale) * (*tensor_scale);
+ *   INT4:  q * scale.
+ * Each value is the exact product rounded once to fp32.  This is the "fake quantised"
+ * operand of the layerwise-loss measurements (paper-graph-ui analysis, section 5,
+ * "Metrics" and "Per-Layer Quantization Loss (Table 1)").  Same G / format rules and
+ * errors as wush_quant_act; rows == 0 returns WUSH_OK without touching the pointers. */
+int wush_dequant(const uint8_t* codes, const void* scales, const float* tensor_scale, int64_t rows,
+                 int64_t d_in, int G, int fmt, float* out, wush_stream_t stream);
+
 /* Transform construction for one layer, on the device, in fp64 (one CTA per block).
  * Sources: paper-graph-ui analysis, section 3.2 "Second-Moment Computer" and "Transform
  * Constructor", sections 3.4.2 and 3.4.4 (Eq. 8); papernotes.org summary, "关键设计";

@@ -419,6 +419,29 @@ def quant_weight(w: np.ndarray, T32: np.ndarray, G: int, fmt: str):
     return pack_nibbles(c), s, st, y
 
 
+def layer_loss(w: np.ndarray, x_bits: np.ndarray, T_w32: np.ndarray, T_x32: np.ndarray,
+               fmt: str, G: int) -> float:
+    """Layerwise RTN quantisation loss ([graph] §3.4.1, the normalised Frobenius loss of
+    Eq. (5); §5 "Metrics" and "Per-Layer Quantization Loss (Table 1)"):
+
+        L = || W^T X - q(T_W W)^T q(T_X X) ||_F^2 / (d_out d_batch)
+
+    with the pages' W [d_in][d_out] and X [d_in][d_batch].  Here, in row layouts,
+    ``w`` is float32 [d_out][d_in] (one row per output channel), ``x_bits`` bfloat16
+    [d_batch][d_in] (one row per token); T_W acts on the weight rows' blocks and T_X on
+    the tokens' blocks, each rounded once to float32; q is the format's RTN AbsMax
+    quantiser followed by dequantisation ("fake quantisation", [graph] §5 Metrics).
+    Everything in float64."""
+    w64 = np.asarray(w, dtype=np.float64)
+    x64 = bf16_to_f64(x_bits)
+    cw, sw, tw, _ = quant_weight(w, T_w32, G, fmt)
+    cx, sx, tx, _ = quant_act(x_bits, T_x32, G, fmt)
+    wq = dequant(unpack_nibbles(cw), sw, fmt, G, tw)
+    xq = dequant(unpack_nibbles(cx), sx, fmt, G, tx)
+    err = w64 @ x64.T - wq @ xq.T
+    return float(np.sum(err * err) / err.size)
+
+
 def grid_step_distance(ca: np.ndarray, cb: np.ndarray, fmt: str) -> np.ndarray:
     """Number of grid steps between two code arrays of the same scale, counting
     the step through zero (+0.5 <-> 0 <-> -0.5 for E2M1; +1 <-> 0 <-> -1 for INT4)."""

@@ -231,6 +231,43 @@ def test_transform_groups_basis_vectors_and_block_choice():
     assert np.array_equal(y, np.stack([T[2].sum(axis=1), T[0].sum(axis=1), T[1].sum(axis=1)]))
 
 
+def test_layer_loss_zero_when_quantisation_is_exact():
+    """Identity transforms and values already on the MXFP4 grid (scale 1): q is exact,
+    the loss is 0; an INT4 grid input likewise."""
+    G, d_in, d_out, n = 32, 64, 3, 4
+    I = np.stack([np.eye(G)] * (d_in // G)).astype(np.float32)
+    grid = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0, -0.5, -6.0])
+    rng = np.random.default_rng(3)
+    w = rng.choice(grid, (d_out, d_in)).astype(np.float32)
+    x = rng.choice(grid, (n, d_in))
+    w[:, 0] = 6.0                         # every group's amax is 6: scale 2^0
+    x[:, ::G] = 6.0
+    from workloads import bf16_bits_from_f64
+    xb = bf16_bits_from_f64(x)
+    assert O.layer_loss(w, xb, I, I, "mxfp4", G) == 0.0
+    wi = rng.integers(-7, 8, (d_out, d_in)).astype(np.float32)
+    xi = rng.integers(-7, 8, (n, d_in)).astype(np.float64)
+    wi[:, ::G] = 7.0
+    xi[:, ::G] = 7.0
+    assert O.layer_loss(wi, bf16_bits_from_f64(xi), I, I, "int4", G) == 0.0
+
+
+def test_layer_loss_matches_hand_computed_single_group():
+    """One output, one token, one INT4 group of 16: x = (7, 1.4, 0, ...), w = (1, 1, 0, ...).
+    s_x = 7/7 = 1, q(x) = (7, 1, 0...); s_w = fl32(1/7), w codes (7, 7, 0...), so the
+    quantised product is 7 s_w * 7 + 7 s_w * 1 = 56 s_w; W^T X = 7 + bf16(1.4)."""
+    G = 16
+    I = np.eye(G, dtype=np.float32)[None]
+    x = np.zeros((1, G)); x[0, 0] = 7.0; x[0, 1] = 1.4
+    w = np.zeros((1, G), np.float32); w[0, 0] = 1.0; w[0, 1] = 1.0
+    from workloads import bf16_bits_from_f64
+    xb = bf16_bits_from_f64(x)
+    x1 = O.bf16_to_f64(xb)[0, 1]               # 1.4 rounded to bfloat16
+    s_w = float(np.float32(1.0) / np.float32(7.0))
+    expect = (7.0 + x1 - 56.0 * s_w) ** 2
+    assert abs(O.layer_loss(w, xb, I, I, "int4", G) - expect) < 1e-12
+
+
 # ---------------------------------------------------------------- grids, brute force
 
 
