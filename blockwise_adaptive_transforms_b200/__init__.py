@@ -19,14 +19,16 @@ __all__ = ["FMT", "WushError", "wush_quant_act", "wush_quant_weight", "wush_quan
            "wush_quant_weight_debug", "wush_quant_act_shared", "wush_quant_act_shared_debug",
            "wush_build_transforms", "wush_device_status", "wush_set_wait_limit_ns",
            "wush_selftest_wait_timeout", "wush_status_string", "wush_version", "load_library",
-           "EXPORTED_SYMBOLS", "output_shapes", "hadamard_matrix", "wush_dequant"]
+           "EXPORTED_SYMBOLS", "output_shapes", "hadamard_matrix", "wush_dequant", "wush_gemm_mxfp4",
+           "wush_mx_scales_to_atoms", "atom_bytes"]
 
 FMT = {"mxfp4": 0, "nvfp4": 1, "int4": 2}
 STATUS = {0: "WUSH_OK", 1: "WUSH_ERR_INVALID_ARG", 2: "WUSH_ERR_UNSUPPORTED", 3: "WUSH_ERR_MISALIGNED",
           4: "WUSH_ERR_CUDA", 5: "WUSH_ERR_DEVICE_TIMEOUT"}
 EXPORTED_SYMBOLS = ("wush_quant_act", "wush_quant_weight", "wush_quant_act_debug",
                     "wush_quant_weight_debug", "wush_quant_act_shared", "wush_quant_act_shared_debug",
-                    "wush_dequant", "wush_build_transforms", "wush_device_status",
+                    "wush_dequant", "wush_gemm_mxfp4", "wush_mx_scales_to_atoms",
+                    "wush_build_transforms", "wush_device_status",
                     "wush_set_wait_limit_ns",
                     "wush_selftest_wait_timeout", "wush_status_string", "wush_version")
 
@@ -63,6 +65,10 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
         getattr(lib, f).restype = ctypes.c_int
     lib.wush_dequant.argtypes = [_P, _P, _P, _I64, _I64, _I32, _I32, _P, _P]
     lib.wush_dequant.restype = ctypes.c_int
+    lib.wush_gemm_mxfp4.argtypes = [_P, _P, _P, _P, _I64, _I64, _I64, _P, _P]
+    lib.wush_gemm_mxfp4.restype = ctypes.c_int
+    lib.wush_mx_scales_to_atoms.argtypes = [_P, _I64, _I64, _P, _P]
+    lib.wush_mx_scales_to_atoms.restype = ctypes.c_int
     lib.wush_build_transforms.argtypes = [_P, _P, _I64, _I64, _I64, _I32, ctypes.c_double, _I32,
                                           _P, _P, _P, _P, _P, _P]
     lib.wush_build_transforms.restype = ctypes.c_int
@@ -228,6 +234,53 @@ def wush_dequant(codes, scales, tensor_scale, G, fmt, out=None, stream=None):
                               _ptr(out), _stream_handle(stream))
     if st != 0:
         raise WushError(st, "wush_dequant")
+    return out
+
+
+def atom_bytes(rows: int, C: int) -> int:
+    """Size of the scale-atom buffer for [rows][C] scales (rows padded to 128, C to 4)."""
+    return ((rows + 127) // 128 * 128) * ((C + 3) // 4 * 4)
+
+
+def wush_mx_scales_to_atoms(scales, out=None, stream=None):
+    """Row-major E8M0 scales u8 [rows][C] -> the tcgen05 scale-atom layout (u8, flat)."""
+    lib = load_library()
+    _check_dev(scales, "scales", torch.uint8)
+    rows, C = int(scales.shape[0]), int(scales.shape[1])
+    if out is None:
+        out = torch.empty(atom_bytes(rows, C), dtype=torch.uint8, device=scales.device)
+    _check_dev(out, "atoms", torch.uint8)
+    if out.numel() < atom_bytes(rows, C):
+        raise ValueError("atoms buffer too small")
+    with torch.cuda.device(scales.device):
+        st = lib.wush_mx_scales_to_atoms(_ptr(scales), rows, C, _ptr(out), _stream_handle(stream))
+    if st != 0:
+        raise WushError(st, "wush_mx_scales_to_atoms")
+    return out
+
+
+def wush_gemm_mxfp4(a_codes, a_atoms, b_codes, b_atoms, out=None, stream=None):
+    """bf16 [M][N] = A B^T from MXFP4 codes ([M][K/2], [N][K/2]) and scale atoms."""
+    lib = load_library()
+    for t, n in ((a_codes, "a_codes"), (b_codes, "b_codes"), (a_atoms, "a_atoms"), (b_atoms, "b_atoms")):
+        _check_dev(t, n, torch.uint8)
+    M, K2 = int(a_codes.shape[0]), int(a_codes.shape[1])
+    N = int(b_codes.shape[0])
+    if int(b_codes.shape[1]) != K2:
+        raise ValueError("A and B must share K")
+    K = 2 * K2
+    if a_atoms.numel() < atom_bytes(M, K // 32) or b_atoms.numel() < atom_bytes(N, K // 32):
+        raise ValueError("scale atom buffers too small")
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=a_codes.device)
+    _check_dev(out, "out", torch.bfloat16)
+    if tuple(out.shape) != (M, N):
+        raise ValueError("out must be [M][N]")
+    with torch.cuda.device(a_codes.device):
+        st = lib.wush_gemm_mxfp4(_ptr(a_codes), _ptr(a_atoms), _ptr(b_codes), _ptr(b_atoms), M, N, K, _ptr(out),
+                                 _stream_handle(stream))
+    if st != 0:
+        raise WushError(st, "wush_gemm_mxfp4")
     return out
 
 

@@ -14,6 +14,7 @@
 #include "wush_fused.cuh"
 #include "wush_build.cuh"
 #include "wush_dequant.cuh"
+#include "wush_gemm.cuh"
 
 namespace wush {
 // Waits on an mbarrier that no thread ever arrives on; the bounded wait must give up.
@@ -64,6 +65,20 @@ int encode_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dt, int el
   cuuint32_t estr[2] = {1u, 1u};
   CUresult r = enc(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                    swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? WUSH_OK : WUSH_ERR_CUDA;
+}
+
+// 2-D row-major uint8 [rows][cols] tensor, box {box_cols, box_rows}, 128-byte swizzle.
+int encode_u8_sw128(CUtensorMap* map, const void* base, int64_t rows, int64_t cols, int box_cols, int box_rows) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return WUSH_ERR_CUDA;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols)};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t estr[2] = {1u, 1u};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? WUSH_OK : WUSH_ERR_CUDA;
 }
 
@@ -255,6 +270,77 @@ int wush_dequant(const uint8_t* codes, const void* scales, const float* tensor_s
     wush::wush_dequant_kernel<wush::kNVFP4><<<grid, 256, 0, s>>>(codes, scales, tensor_scale, rows, di, G, out);
   else
     wush::wush_dequant_kernel<wush::kINT4><<<grid, 256, 0, s>>>(codes, scales, tensor_scale, rows, di, G, out);
+  return cudaGetLastError() == cudaSuccess ? WUSH_OK : WUSH_ERR_CUDA;
+}
+
+int wush_mx_scales_to_atoms(const uint8_t* scales, int64_t rows, int64_t C, uint8_t* atoms, wush_stream_t stream) {
+  if (rows < 0 || C <= 0 || C > INT_MAX / 4) return WUSH_ERR_INVALID_ARG;
+  if (rows == 0) return WUSH_OK;
+  if (!scales || !atoms) return WUSH_ERR_INVALID_ARG;
+  const long long rows_pad = (rows + 127) / 128 * 128;
+  const int C_pad = static_cast<int>((C + 3) / 4 * 4);
+  const long long n = rows_pad * C_pad;
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return WUSH_ERR_CUDA;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return WUSH_ERR_CUDA;
+  const long long want = (n + 255) / 256;
+  const int grid = static_cast<int>(want < 8LL * sms ? want : 8LL * sms);
+  wush::wush_scales_to_atoms_kernel<<<grid, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      scales, rows, static_cast<int>(C), atoms, rows_pad, C_pad);
+  return cudaGetLastError() == cudaSuccess ? WUSH_OK : WUSH_ERR_CUDA;
+}
+
+int wush_gemm_mxfp4(const uint8_t* a_codes, const uint8_t* a_atoms, const uint8_t* b_codes, const uint8_t* b_atoms,
+                    int64_t M, int64_t N, int64_t K, void* d_bf16, wush_stream_t stream) {
+  using Cfg = wush::GemmCfg;
+  if (M < 0 || N <= 0 || K <= 0) return WUSH_ERR_INVALID_ARG;
+  if (M % Cfg::BM || N % Cfg::BN || K % Cfg::BK) return WUSH_ERR_UNSUPPORTED;
+  if (M > INT_MAX || N > INT_MAX || K > INT_MAX) return WUSH_ERR_INVALID_ARG;
+  if (M == 0) return WUSH_OK;
+  if (!a_codes || !a_atoms || !b_codes || !b_atoms || !d_bf16) return WUSH_ERR_INVALID_ARG;
+  if (!aligned(a_codes, 16) || !aligned(b_codes, 16) || !aligned(a_atoms, 16) || !aligned(b_atoms, 16) ||
+      !aligned(d_bf16, 16))
+    return WUSH_ERR_MISALIGNED;
+  CUtensorMap ma, mb;
+  int st = encode_u8_sw128(&ma, a_codes, M, K / 2, 128, Cfg::BM);
+  if (st != WUSH_OK) return st;
+  st = encode_u8_sw128(&mb, b_codes, N, K / 2, 128, Cfg::BN);
+  if (st != WUSH_OK) return st;
+  wush::GemmParams p{};
+  p.sfa = a_atoms;
+  p.sfb = b_atoms;
+  p.d = static_cast<__nv_bfloat16*>(d_bf16);
+  p.M = static_cast<int>(M);
+  p.N = static_cast<int>(N);
+  p.K = static_cast<int>(K);
+  p.tiles_m = static_cast<int>(M / Cfg::BM);
+  p.tiles_n = static_cast<int>(N / Cfg::BN);
+  p.wait_limit_ns = g_wait_limit_ns.load(std::memory_order_relaxed);
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return WUSH_ERR_CUDA;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return WUSH_ERR_CUDA;
+  static std::atomic<unsigned long long> configured{0ull};
+  const unsigned long long bit = 1ull << (dev & 63);
+  if (!(configured.load(std::memory_order_acquire) & bit)) {
+    if (cudaFuncSetAttribute(wush::wush_gemm_mxf4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             Cfg::SMEM_BYTES) != cudaSuccess)
+      return WUSH_ERR_CUDA;
+    configured.fetch_or(bit, std::memory_order_acq_rel);
+  }
+  const long long tiles = static_cast<long long>(p.tiles_m) * p.tiles_n;
+  if (tiles > INT_MAX) return WUSH_ERR_INVALID_ARG;
+  const int grid = static_cast<int>(tiles < sms ? tiles : sms);
+  cudaLaunchConfig_t lc = {};
+  lc.gridDim = dim3(static_cast<unsigned>(grid));
+  lc.blockDim = dim3(Cfg::THREADS);
+  lc.dynamicSmemBytes = Cfg::SMEM_BYTES;
+  lc.stream = reinterpret_cast<cudaStream_t>(stream);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  lc.attrs = attr;
+  lc.numAttrs = WUSH_USE_PDL ? 1 : 0;
+  if (cudaLaunchKernelEx(&lc, wush::wush_gemm_mxf4_kernel, ma, mb, p) != cudaSuccess) return WUSH_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? WUSH_OK : WUSH_ERR_CUDA;
 }
 

@@ -1,0 +1,273 @@
+// MXFP4 x MXFP4 -> bf16 GEMM for sm_100a on block-scaled tcgen05 MMAs: the consumer of the
+// quantised operands (the pages' "WUSH + Quant + FP4 MatMul" layer: paper-graph-ui
+// analysis, section 3.4.7 "GPU Kernel Design" and section 5 "GPU Kernel Benchmarks
+// (Figure 2)").
+//
+//   D[m][n] = sum_k A[m][k] * B[n][k]
+//
+// A (activations, M rows) and B (weights, N rows = output channels) are E2M1 codes packed
+// two per byte along K (low nibble = even k), each 32-element group with an E8M0 scale.
+// The scales are read in the layout the block-scaled MMA consumes ("tcgen05 scale
+// atoms"): for rows [128 r, 128 r + 128) and scale columns [4 c, 4 c + 4) one 512-byte
+// atom at byte (r * (K / 128) + c) * 512, in which row 128 r + i + 32 j, scale 4 c + k
+// sits at byte 16 i + 4 j + k (i < 32, j < 4, k < 4).
+//
+// Tiles of 128 x 256 outputs, 256 K-elements (128 bytes of codes per row) per pipeline
+// stage; per stage the producer brings A (16 KB) and B (32 KB) by TMA with 128-byte
+// swizzle and the three scale atoms' 1 KB pieces by bulk copies; the MMA thread moves the
+// scale atoms into TMEM (tcgen05.cp 32x128b, broadcast to the four lane quadrants) and
+// issues four M=128, N=256, K=64 MMAs (kind::mxf4, block32); four epilogue warps read the
+// fp32 accumulator (tcgen05.ld), round to bf16 and store.  Persistent CTAs, one per SM.
+#pragma once
+#include <cstdint>
+#include <cuda_bf16.h>
+#include "wush_ptx.cuh"
+
+namespace wush {
+
+struct GemmParams {
+  const uint8_t* sfa;        // A scale atoms
+  const uint8_t* sfb;        // B scale atoms
+  __nv_bfloat16* d;          // [M][N]
+  int M, N, K;
+  int tiles_m, tiles_n;
+  unsigned long long wait_limit_ns;
+};
+
+struct GemmCfg {
+  static constexpr int BM = 128, BN = 256, BK = 256;   // BK in elements (128 bytes of codes)
+  static constexpr int STAGES = 4;
+  static constexpr int A_BYTES = BM * BK / 2;          // 16 KB
+  static constexpr int B_BYTES = BN * BK / 2;          // 32 KB
+  static constexpr int SFA_BYTES = BM * BK / 32;       // 1 KB: two atoms
+  static constexpr int SFB_BYTES = BN * BK / 32;       // 2 KB: two atoms per 128-row half
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
+  static constexpr int OFF_A = 0, OFF_B = A_BYTES, OFF_SFA = A_BYTES + B_BYTES, OFF_SFB = OFF_SFA + SFA_BYTES;
+  static constexpr int OFF_BAR = STAGES * STAGE_BYTES;
+  static constexpr int N_BARS = 2 * STAGES + 3;        // full[S], empty[S], afull, aempty, drain
+  static constexpr int OFF_MISC = OFF_BAR + 8 * N_BARS;
+  static constexpr int SMEM_BYTES = OFF_MISC + 64 + 1024;
+  static constexpr int THREADS = 8 * 32;               // producer, MMA, 2 idle, 4 epilogue warps
+  // TMEM: accumulator columns [0, 256); per stage slot 24 scale columns from 256
+  static constexpr int TMEM_COLS = 512;
+  static constexpr int SF_COL0 = 256, SF_SLOT_COLS = 24;
+  static_assert(STAGE_BYTES % 1024 == 0, "stage alignment");
+  static_assert(SF_COL0 + STAGES * SF_SLOT_COLS <= TMEM_COLS, "TMEM columns");
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+};
+
+// Instruction descriptor of kind::mxf4 block-scaled MMAs: E2M1 A and B (format 1),
+// K-major, E8M0 scales (bit 23), M = 128, N = 256, dense K = 64; the scale-factor ids
+// (bits 29-30 for A, 4-5 for B) select the byte of the TMEM word the first scale sits in.
+__device__ __forceinline__ uint32_t idesc_mxf4(int M, int N, uint32_t sf_id) {
+  return (sf_id << 4)                               // B scale-factor id
+         | (1u << 7)                                // A format: E2M1
+         | (1u << 10)                               // B format: E2M1
+         | (static_cast<uint32_t>(N >> 3) << 17)    // N / 8
+         | (1u << 23)                               // scale format: E8M0
+         | (static_cast<uint32_t>(M >> 4) << 24)    // M / 16
+         | (sf_id << 29);                           // A scale-factor id
+}
+
+__device__ __forceinline__ void umma_mxf4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+
+// Shared-memory descriptor of one scale atom (32 rows x 16 bytes, rows contiguous, no
+// swizzle): 8-row core matrices 128 bytes apart.
+__device__ __forceinline__ uint64_t desc_sf_atom(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);   // start address
+  d |= static_cast<uint64_t>(1) << 16;                     // leading byte offset (one core matrix wide)
+  d |= static_cast<uint64_t>(128 >> 4) << 32;              // stride byte offset: 8 rows x 16 B
+  d |= static_cast<uint64_t>(1) << 46;                     // descriptor version for sm_100
+  return d;                                                // layout type 0: no swizzle
+}
+
+// 32 lanes x 128 bits from shared memory into TMEM, repeated in all four lane quadrants.
+__device__ __forceinline__ void tmem_cp_32x128b_x4(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
+__global__ void __launch_bounds__(GemmCfg::THREADS, 1)
+    wush_gemm_mxf4_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
+                          const GemmParams p) {
+  using Cfg = GemmCfg;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_addr(smem);
+  const uint32_t bar0 = sbase + Cfg::OFF_BAR;
+  auto BAR = [&](int i) -> uint32_t { return bar0 + 8u * static_cast<uint32_t>(i); };
+  constexpr int STAGES = Cfg::STAGES;
+  const int B_FULL = 0, B_EMPTY = STAGES, B_AFULL = 2 * STAGES, B_AEMPTY = 2 * STAGES + 1, B_DRAIN = 2 * STAGES + 2;
+  volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + Cfg::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::OFF_MISC + 4);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint64_t lim = p.wait_limit_ns;
+  const int n_tiles = p.tiles_m * p.tiles_n;
+  const int k_stages = p.K / Cfg::BK;
+  const int k_chunks = p.K / 128;                       // scale atoms along K per 128-row block
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(BAR(B_FULL + s), 1);
+      mbar_init(BAR(B_EMPTY + s), 1);
+    }
+    mbar_init(BAR(B_AFULL), 1);
+    mbar_init(BAR(B_AEMPTY), 4);
+    mbar_init(BAR(B_DRAIN), 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+    tma_prefetch_desc(&tmap_a);
+    tma_prefetch_desc(&tmap_b);
+  }
+  grid_dependency_wait();
+  grid_launch_dependents();
+  if (warp == 1) {
+    tmem_alloc(smem_addr(const_cast<uint32_t*>(tmem_slot)), Cfg::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      const uint64_t pol = l2_policy_evict_first();
+      int stage = 0, n_issued = 0;
+      uint32_t phase = 0;
+      for (int tile = blockIdx.x; tile < n_tiles && !*abort_flag; tile += gridDim.x) {
+        const int tm = tile % p.tiles_m, tn = tile / p.tiles_m;
+        for (int ks = 0; ks < k_stages; ++ks) {
+          if (!wait_bounded(BAR(B_EMPTY + stage), phase ^ 1u, abort_flag, 1u, lim)) break;
+          const uint32_t dst = sbase + stage * Cfg::STAGE_BYTES;
+          const uint32_t fb = BAR(B_FULL + stage);
+          mbar_arrive_expect_tx(fb, Cfg::STAGE_BYTES);
+          tma_load_2d(dst + Cfg::OFF_A, &tmap_a, fb, ks * 128, tm * Cfg::BM, 0ull);
+          tma_load_2d(dst + Cfg::OFF_B, &tmap_b, fb, ks * 128, tn * Cfg::BN, pol);
+          // scale atoms: K chunks 2 ks and 2 ks + 1 of the tile's row blocks (1 KB each)
+          bulk_load_1d(dst + Cfg::OFF_SFA, p.sfa + (static_cast<long long>(tm) * k_chunks + 2 * ks) * 512, 1024u, fb);
+          for (int h = 0; h < 2; ++h)
+            bulk_load_1d(dst + Cfg::OFF_SFB + h * 1024,
+                         p.sfb + (static_cast<long long>(2 * tn + h) * k_chunks + 2 * ks) * 512, 1024u, fb);
+          ++n_issued;
+          if (++stage == STAGES) stage = 0, phase ^= 1u;
+        }
+      }
+      if (*abort_flag) {   // copies in flight land before the CTA exits
+        volatile int no_abort = 0;
+        for (int k = (n_issued > STAGES ? n_issued - STAGES : 0); k < n_issued; ++k)
+          wait_bounded(BAR(B_FULL + k % STAGES), static_cast<uint32_t>((k / STAGES) & 1), &no_abort, 16u, lim);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int stage = 0, it = 0;
+      uint32_t phase = 0;
+      for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++it) {
+        if (!wait_bounded(BAR(B_AEMPTY), static_cast<uint32_t>((it & 1) ^ 1), abort_flag, 2u, lim)) break;
+        tc_fence_after();
+        bool ok = true;
+        for (int ks = 0; ks < k_stages; ++ks) {
+          if (!wait_bounded(BAR(B_FULL + stage), phase, abort_flag, 2u, lim)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t st = sbase + stage * Cfg::STAGE_BYTES;
+          const uint32_t sf_cols = tmem_base + static_cast<uint32_t>(Cfg::SF_COL0 + stage * Cfg::SF_SLOT_COLS);
+          // scale atoms -> TMEM: A chunk c at columns +4c, B chunk c, half h at +8 + 8c + 4h
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {
+            tmem_cp_32x128b_x4(sf_cols + 4 * c, desc_sf_atom(st + Cfg::OFF_SFA + c * 512));
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+              tmem_cp_32x128b_x4(sf_cols + 8 + 8 * c + 4 * h, desc_sf_atom(st + Cfg::OFF_SFB + h * 1024 + c * 512));
+          }
+          const uint64_t da = desc_k_sw128(st + Cfg::OFF_A);
+          const uint64_t db = desc_k_sw128(st + Cfg::OFF_B);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {        // K = 64 each: 32 bytes along the 128-byte rows
+            const int c = j >> 1;
+            const uint32_t sub = static_cast<uint32_t>(2 * (j & 1));   // scale byte 0 or 2 of the word
+            const uint32_t sfa = (sf_cols + 4 * c) | (sub << 30);
+            const uint32_t sfb = (sf_cols + 8 + 8 * c) | (sub << 30);
+            umma_mxf4(tmem_base, da + ((j * 32) >> 4), db + ((j * 32) >> 4), idesc_mxf4(128, 256, sub), sfa, sfb,
+                      (ks > 0 || j > 0) ? 1u : 0u);
+          }
+          umma_commit(BAR(B_EMPTY + stage));
+          if (++stage == STAGES) stage = 0, phase ^= 1u;
+        }
+        if (!ok) break;
+        umma_commit(BAR(B_AFULL));
+      }
+      umma_commit(BAR(B_DRAIN));
+      volatile int no_abort = 0;
+      wait_bounded(BAR(B_DRAIN), 0u, &no_abort, 16u, lim);
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ epilogue (4 warps)
+    const int quad = warp & 3;
+    const int row_in_tile = quad * 32 + lane;
+    int it = 0;
+    bool live = true;
+    for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++it) {
+      const int tm = tile % p.tiles_m, tn = tile / p.tiles_m;
+      if (live && !wait_bounded(BAR(B_AFULL), static_cast<uint32_t>(it & 1), abort_flag, 8u, lim)) live = false;
+      const bool warp_live = __all_sync(0xffffffffu, live) && !*abort_flag;
+      if (warp_live) tc_fence_after();
+      const long long row = static_cast<long long>(tm) * Cfg::BM + row_in_tile;
+      __nv_bfloat16* drow = p.d + row * p.N + static_cast<long long>(tn) * Cfg::BN;
+#pragma unroll 1
+      for (int ch = 0; ch < Cfg::BN / 32; ++ch) {
+        float v[32];
+        if (warp_live) tmem_ld32_sync(tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(32 * ch), v);
+        if (!warp_live) continue;
+        uint32_t packed[16];
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+          const __nv_bfloat162 b2 = __floats2bfloat162_rn(v[2 * k], v[2 * k + 1]);
+          packed[k] = *reinterpret_cast<const uint32_t*>(&b2);
+        }
+        uint4* dst = reinterpret_cast<uint4*>(drow + 32 * ch);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) dst[k] = make_uint4(packed[4 * k], packed[4 * k + 1], packed[4 * k + 2], packed[4 * k + 3]);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(BAR(B_AEMPTY));
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, Cfg::TMEM_COLS);
+  }
+}
+
+// Row-major E8M0 scales [rows][C] (C = K / 32) -> tcgen05 scale atoms (rows padded to a
+// multiple of 128 with zero bytes, C to a multiple of 4).
+__global__ void wush_scales_to_atoms_kernel(const uint8_t* __restrict__ src, long long rows, int C,
+                                            uint8_t* __restrict__ dst, long long rows_pad, int C_pad) {
+  const long long n = rows_pad * C_pad;
+  const int k_chunks = C_pad / 4;
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const long long r = i / C_pad;
+    const int c = static_cast<int>(i - r * C_pad);
+    const uint8_t v = (r < rows && c < C) ? src[r * C + c] : static_cast<uint8_t>(0);
+    const long long rb = r >> 7;
+    const int rr = static_cast<int>(r & 127);
+    dst[(rb * k_chunks + (c >> 2)) * 512 + (rr & 31) * 16 + (rr >> 5) * 4 + (c & 3)] = v;
+  }
+}
+
+}  // namespace wush

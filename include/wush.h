@@ -133,6 +133,29 @@ int wush_quant_act_shared_debug(const void* x_bf16, const float* T_shared, int64
 int wush_dequant(const uint8_t* codes, const void* scales, const float* tensor_scale, int64_t rows,
                  int64_t d_in, int G, int fmt, float* out, wush_stream_t stream);
 
+/* FP4 GEMM consumer: D = A * B^T in bf16 from MXFP4 operands, on block-scaled tcgen05
+ * MMAs (the "FP4 MatMul" after WUSH + Quant: paper-graph-ui analysis, section 3.4.7
+ * "GPU Kernel Design"; section 5 "GPU Kernel Benchmarks (Figure 2)").
+ *   D[m][n] = sum_k A[m][k] B[n][k]      (fp32 accumulation, one bf16 rounding)
+ * a_codes u8 [M][K/2] (e.g. wush_quant_act's MXFP4 codes), b_codes u8 [N][K/2] (e.g.
+ * wush_quant_weight's, one row per output channel), both E2M1 pairs, low nibble = even k.
+ * a_atoms / b_atoms: the E8M0 scales in the tcgen05 scale-atom layout (see
+ * wush_mx_scales_to_atoms).  d_bf16: [M][N] row-major.  All device memory, 16-byte aligned.
+ * Supported: M % 128 == 0, N % 256 == 0, K % 256 == 0 (else WUSH_ERR_UNSUPPORTED).
+ * Asynchronous on `stream`; allocates nothing. */
+int wush_gemm_mxfp4(const uint8_t* a_codes, const uint8_t* a_atoms, const uint8_t* b_codes,
+                    const uint8_t* b_atoms, int64_t M, int64_t N, int64_t K, void* d_bf16,
+                    wush_stream_t stream);
+
+/* Row-major E8M0 scales [rows][C] -> the scale-atom layout the block-scaled MMA reads:
+ * rows padded to a multiple of 128 and C to a multiple of 4 (zero bytes); the atom of
+ * row block r and scale columns [4c, 4c + 4) is the 512 bytes at (r * (C_pad/4) + c) * 512,
+ * holding row 128 r + i + 32 j, column 4 c + k at byte 16 i + 4 j + k (i < 32, j < 4,
+ * k < 4).  `atoms` (device) must hold rows_pad * C_pad bytes.  This layout is NVIDIA's
+ * tcgen05 block-scale format, not something the pages define. */
+int wush_mx_scales_to_atoms(const uint8_t* scales, int64_t rows, int64_t C, uint8_t* atoms,
+                            wush_stream_t stream);
+
 /* Transform construction for one layer, on the device, in fp64 (one CTA per block).
  * Sources: paper-graph-ui analysis, section 3.2 "Second-Moment Computer" and "Transform
  * Constructor", sections 3.4.2 and 3.4.4 (Eq. 8); papernotes.org summary, "关键设计";

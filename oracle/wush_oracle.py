@@ -442,6 +442,31 @@ def layer_loss(w: np.ndarray, x_bits: np.ndarray, T_w32: np.ndarray, T_x32: np.n
     return float(np.sum(err * err) / err.size)
 
 
+def scale_atoms(scales: np.ndarray) -> np.ndarray:
+    """E8M0 scales [rows][C] in the block-scaled MMA's scale-atom layout (a hardware
+    format, not from the pages): rows padded to a multiple of 128 and C to a multiple
+    of 4 with zero bytes; row 128 r + i + 32 j, column 4 c + k goes to byte
+    (r * C_pad / 4 + c) * 512 + 16 i + 4 j + k."""
+    s = np.asarray(scales, dtype=np.uint8)
+    rows, C = s.shape
+    rows_pad, C_pad = -(-rows // 128) * 128, -(-C // 4) * 4
+    full = np.zeros((rows_pad, C_pad), np.uint8)
+    full[:rows, :C] = s
+    # [r][j][i][c][k] -> [r][c][i][j][k]
+    t = full.reshape(rows_pad // 128, 4, 32, C_pad // 4, 4)
+    return np.ascontiguousarray(t.transpose(0, 3, 2, 1, 4)).reshape(-1)
+
+
+def gemm_mx(a_codes: np.ndarray, a_scales: np.ndarray, b_codes: np.ndarray, b_scales: np.ndarray) -> np.ndarray:
+    """The FP4 MatMul after WUSH + Quant ([graph] §3.4.7 "GPU Kernel Design": the
+    transformed, quantised activations multiply the pre-quantised weights):
+    D = deq(A) deq(B)^T in float64, A packed MXFP4 codes [M][K/2] with scales [M][K/32],
+    B packed codes [N][K/2] with scales [N][K/32] (one row per output channel)."""
+    A = dequant(unpack_nibbles(a_codes), a_scales, "mxfp4", 32)
+    B = dequant(unpack_nibbles(b_codes), b_scales, "mxfp4", 32)
+    return A @ B.T
+
+
 def grid_step_distance(ca: np.ndarray, cb: np.ndarray, fmt: str) -> np.ndarray:
     """Number of grid steps between two code arrays of the same scale, counting
     the step through zero (+0.5 <-> 0 <-> -0.5 for E2M1; +1 <-> 0 <-> -1 for INT4)."""

@@ -1,0 +1,83 @@
+"""MXFP4 GEMM consumer and the scale-atom relayout vs the fp64 oracle (needs a B200).
+
+D = deq(A) deq(B)^T (paper-graph-ui analysis, section 3.4.7 "GPU Kernel Design": the
+FP4 MatMul that follows WUSH + Quant).  The kernel accumulates in fp32 and rounds D once
+to bf16, so each element must lie within 2^-8 |D| (bf16 rounding) plus the fp32
+accumulation bound K 2^-23 (|A| |B|^T) of the oracle's value.
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import wush_oracle as O
+from workloads import make_inputs, workload
+import blockwise_adaptive_transforms_b200 as W
+
+pytestmark = pytest.mark.gpu
+
+
+def dev(a):
+    return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+
+def random_operand(rows, K, seed, lo=120, hi=134):
+    rng = np.random.default_rng(seed)
+    codes = rng.integers(0, 256, (rows, K // 2), dtype=np.uint8)
+    scales = rng.integers(lo, hi, (rows, K // 32), dtype=np.uint8)
+    return codes, scales
+
+
+def assert_gemm_close(d_gpu, a_c, a_s, b_c, b_s, K):
+    ref = O.gemm_mx(a_c, a_s, b_c, b_s)
+    A = np.abs(O.dequant(O.unpack_nibbles(a_c), a_s, "mxfp4", 32))
+    B = np.abs(O.dequant(O.unpack_nibbles(b_c), b_s, "mxfp4", 32))
+    bound = 2.0 ** -8 * np.abs(ref) + K * 2.0 ** -23 * (A @ B.T) + 1e-30
+    err = np.abs(d_gpu.astype(np.float64) - ref)
+    worst = np.unravel_index(np.argmax(err / bound), err.shape)
+    assert np.all(err <= bound), f"at {worst}: gpu {d_gpu[worst]} oracle {ref[worst]} bound {bound[worst]}"
+
+
+@pytest.mark.parametrize("rows,C", [(128, 8), (300, 10), (1024, 128)])
+def test_scale_atoms_match_the_layout(rows, C):
+    s = np.random.default_rng(rows).integers(0, 255, (rows, C), dtype=np.uint8)
+    at = W.wush_mx_scales_to_atoms(dev(s))
+    torch.cuda.synchronize()
+    assert np.array_equal(at.cpu().numpy(), O.scale_atoms(s))
+
+
+@pytest.mark.parametrize("M,N,K", [(128, 256, 256), (256, 512, 1024), (384, 768, 768), (128, 256, 4096)])
+def test_gemm_random_operands(M, N, K):
+    a_c, a_s = random_operand(M, K, 1)
+    b_c, b_s = random_operand(N, K, 2)
+    d = W.wush_gemm_mxfp4(dev(a_c), W.wush_mx_scales_to_atoms(dev(a_s)), dev(b_c), W.wush_mx_scales_to_atoms(dev(b_s)))
+    torch.cuda.synchronize()
+    st, bits = W.wush_device_status()
+    assert st == 0 and bits == 0, f"device error word {bits:#x}"
+    assert_gemm_close(d.float().cpu().numpy(), a_c, a_s, b_c, b_s, K)
+
+
+def test_gemm_after_wush_quantisation():
+    """The layer: activations and weights quantised with the WUSH transforms by the
+    library's kernels, then the FP4 GEMM; the oracle multiplies the kernels' own codes."""
+    wl = workload("attn_mxfp4_4096", n_tok=256, d_in=1024, d_out=512, n_cal=1024)
+    inp = make_inputs(wl)
+    b = O.build_transforms(inp.w, inp.xcal_bits, 32)
+    x = dev(inp.x_bits.view(np.int16)).view(torch.bfloat16)
+    cx, sx, _ = W.wush_quant_act(x, dev(b["T_wush32"]), 32, "mxfp4")
+    cw, sw, _ = W.wush_quant_weight(dev(inp.w), dev(b["T_xvsh32"]), 32, "mxfp4")
+    d = W.wush_gemm_mxfp4(cx, W.wush_mx_scales_to_atoms(sx), cw, W.wush_mx_scales_to_atoms(sw))
+    torch.cuda.synchronize()
+    assert_gemm_close(d.float().cpu().numpy(), cx.cpu().numpy(), sx.cpu().numpy(), cw.cpu().numpy(),
+                      sw.cpu().numpy(), wl.d_in)
+    # and the quantised layer approximates the full-precision one
+    ref = O.bf16_to_f64(inp.x_bits) @ inp.w.astype(np.float64).T
+    rel = np.linalg.norm(d.float().cpu().numpy() - ref) / np.linalg.norm(ref)
+    assert rel < 0.25, rel
+
+
+def test_gemm_rejects_unsupported_shapes():
+    a = torch.zeros((100, 128), dtype=torch.uint8, device="cuda")
+    b = torch.zeros((256, 128), dtype=torch.uint8, device="cuda")
+    with pytest.raises(W.WushError):
+        W.wush_gemm_mxfp4(a, torch.zeros(W.atom_bytes(100, 8), dtype=torch.uint8, device="cuda"), b,
+                          torch.zeros(W.atom_bytes(256, 8), dtype=torch.uint8, device="cuda"))

@@ -268,6 +268,34 @@ def test_layer_loss_matches_hand_computed_single_group():
     assert abs(O.layer_loss(w, xb, I, I, "int4", G) - expect) < 1e-12
 
 
+def test_scale_atoms_places_bytes_by_the_atom_formula():
+    rows, C = 300, 10
+    s = (np.arange(rows * C) % 251).astype(np.uint8).reshape(rows, C)
+    at = O.scale_atoms(s)
+    rows_pad, C_pad = 384, 12
+    assert at.shape == (rows_pad * C_pad,)
+    for r, c in [(0, 0), (33, 5), (127, 9), (128, 0), (299, 9), (200, 3)]:
+        rb, i, j = r // 128, r % 32, (r % 128) // 32
+        off = (rb * (C_pad // 4) + c // 4) * 512 + 16 * i + 4 * j + c % 4
+        assert at[off] == s[r, c]
+    assert at[(2 * 3 + 2) * 512 + 16 * 31 + 4 * 3 + 3] == 0       # padding row 383, column 11
+    assert sorted(at[at > 0].tolist()) == sorted(s[s > 0].tolist())
+
+
+def test_gemm_mx_exact_small_cases():
+    """All codes 1.0 at scale 2^0: every output is K.  A at 2^1 and B at 2^-1 with codes
+    1.5 and -2: every output is K * 1.5 * -2."""
+    M, N, K = 4, 3, 64
+    one = O.pack_nibbles(np.full((M, K), 2, np.uint8))               # E2M1 code 2 = 1.0
+    oneb = O.pack_nibbles(np.full((N, K), 2, np.uint8))
+    d = O.gemm_mx(one, np.full((M, K // 32), 127, np.uint8), oneb, np.full((N, K // 32), 127, np.uint8))
+    assert np.array_equal(d, np.full((M, N), float(K)))
+    a = O.pack_nibbles(np.full((M, K), 3, np.uint8))                 # 1.5
+    b = O.pack_nibbles(np.full((N, K), 0xC, np.uint8))               # -2
+    d = O.gemm_mx(a, np.full((M, K // 32), 128, np.uint8), b, np.full((N, K // 32), 126, np.uint8))
+    assert np.array_equal(d, np.full((M, N), K * 1.5 * -2.0))
+
+
 # ---------------------------------------------------------------- grids, brute force
 
 
