@@ -20,14 +20,16 @@ __all__ = ["FMT", "WushError", "wush_quant_act", "wush_quant_weight", "wush_quan
            "wush_build_transforms", "wush_device_status", "wush_set_wait_limit_ns",
            "wush_selftest_wait_timeout", "wush_status_string", "wush_version", "load_library",
            "EXPORTED_SYMBOLS", "output_shapes", "hadamard_matrix", "wush_dequant", "wush_gemm_mxfp4",
-           "wush_mx_scales_to_atoms", "atom_bytes"]
+           "wush_mx_scales_to_atoms", "atom_bytes", "wush_quant_act_mx_atoms", "wush_quant_weight_mx_atoms",
+           "wush_quant_act_shared_mx_atoms"]
 
 FMT = {"mxfp4": 0, "nvfp4": 1, "int4": 2}
 STATUS = {0: "WUSH_OK", 1: "WUSH_ERR_INVALID_ARG", 2: "WUSH_ERR_UNSUPPORTED", 3: "WUSH_ERR_MISALIGNED",
           4: "WUSH_ERR_CUDA", 5: "WUSH_ERR_DEVICE_TIMEOUT"}
 EXPORTED_SYMBOLS = ("wush_quant_act", "wush_quant_weight", "wush_quant_act_debug",
                     "wush_quant_weight_debug", "wush_quant_act_shared", "wush_quant_act_shared_debug",
-                    "wush_dequant", "wush_gemm_mxfp4", "wush_mx_scales_to_atoms",
+                    "wush_dequant", "wush_gemm_mxfp4", "wush_mx_scales_to_atoms", "wush_quant_act_mx_atoms",
+                    "wush_quant_weight_mx_atoms", "wush_quant_act_shared_mx_atoms",
                     "wush_build_transforms", "wush_device_status",
                     "wush_set_wait_limit_ns",
                     "wush_selftest_wait_timeout", "wush_status_string", "wush_version")
@@ -65,6 +67,9 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
         getattr(lib, f).restype = ctypes.c_int
     lib.wush_dequant.argtypes = [_P, _P, _P, _I64, _I64, _I32, _I32, _P, _P]
     lib.wush_dequant.restype = ctypes.c_int
+    for f in ("wush_quant_act_mx_atoms", "wush_quant_weight_mx_atoms", "wush_quant_act_shared_mx_atoms"):
+        getattr(lib, f).argtypes = [_P, _P, _I64, _I64, _P, _P, _P]
+        getattr(lib, f).restype = ctypes.c_int
     lib.wush_gemm_mxfp4.argtypes = [_P, _P, _P, _P, _I64, _I64, _I64, _P, _P]
     lib.wush_gemm_mxfp4.restype = ctypes.c_int
     lib.wush_mx_scales_to_atoms.argtypes = [_P, _I64, _I64, _P, _P]
@@ -257,6 +262,44 @@ def wush_mx_scales_to_atoms(scales, out=None, stream=None):
     if st != 0:
         raise WushError(st, "wush_mx_scales_to_atoms")
     return out
+
+
+def _quant_atoms(fn_name, inp, in_dtype, T, codes, atoms, stream, shared=False):
+    lib = load_library()
+    _check_dev(inp, "input", in_dtype)
+    _check_dev(T, "T", torch.float32)
+    rows, d_in = int(inp.shape[0]), int(inp.shape[1])
+    if d_in % 32:
+        raise ValueError("d_in must be a multiple of 32")
+    t_shape = (32, 32) if shared else (d_in // 32, 32, 32)
+    if tuple(T.shape) != t_shape:
+        raise ValueError(f"T must have shape {t_shape}")
+    if codes is None:
+        codes = torch.empty((rows, d_in // 2), dtype=torch.uint8, device=inp.device)
+    if atoms is None:
+        atoms = torch.zeros(atom_bytes(rows, d_in // 32), dtype=torch.uint8, device=inp.device)
+    _check_dev(codes, "codes", torch.uint8)
+    _check_dev(atoms, "scale atoms", torch.uint8)
+    if tuple(codes.shape) != (rows, d_in // 2) or atoms.numel() < atom_bytes(rows, d_in // 32):
+        raise ValueError("output buffers have the wrong size")
+    with torch.cuda.device(inp.device):
+        st = getattr(lib, fn_name)(_ptr(inp), _ptr(T), rows, d_in, _ptr(codes), _ptr(atoms), _stream_handle(stream))
+    if st != 0:
+        raise WushError(st, fn_name)
+    return codes, atoms
+
+
+def wush_quant_act_mx_atoms(x, T, codes=None, atoms=None, stream=None):
+    """MXFP4 activations with the scales written in the scale-atom layout: (codes, atoms)."""
+    return _quant_atoms("wush_quant_act_mx_atoms", x, torch.bfloat16, T, codes, atoms, stream)
+
+
+def wush_quant_weight_mx_atoms(w, T, codes=None, atoms=None, stream=None):
+    return _quant_atoms("wush_quant_weight_mx_atoms", w, torch.float32, T, codes, atoms, stream)
+
+
+def wush_quant_act_shared_mx_atoms(x, T, codes=None, atoms=None, stream=None):
+    return _quant_atoms("wush_quant_act_shared_mx_atoms", x, torch.bfloat16, T, codes, atoms, stream, shared=True)
 
 
 def wush_gemm_mxfp4(a_codes, a_atoms, b_codes, b_atoms, out=None, stream=None):

@@ -144,7 +144,7 @@ int dispatch(const CUtensorMap& map, const CUtensorMap& cmap, wush::FusedParams 
 
 int quant_common(const void* in, bool in_f32, const float* T, int64_t rows, int64_t d_in, int G, int fmt,
                  uint8_t* codes, void* scales, float* tensor_scale, float* y_out, bool debug,
-                 wush_stream_t stream, bool shared_T = false) {
+                 wush_stream_t stream, bool shared_T = false, bool scale_atoms = false) {
   if (fmt != WUSH_MXFP4 && fmt != WUSH_NVFP4 && fmt != WUSH_INT4) return WUSH_ERR_UNSUPPORTED;
   const bool g_ok = (fmt == WUSH_MXFP4 && G == 32) || (fmt == WUSH_NVFP4 && G == 16) ||
                     (fmt == WUSH_INT4 && (G == 16 || G == 32));
@@ -157,6 +157,7 @@ int quant_common(const void* in, bool in_f32, const float* T, int64_t rows, int6
   if (debug && !y_out) return WUSH_ERR_INVALID_ARG;
   if (!aligned(in, 16) || !aligned(T, 16) || !aligned(codes, 16)) return WUSH_ERR_MISALIGNED;
   if (fmt == WUSH_INT4 && !aligned(scales, 4)) return WUSH_ERR_MISALIGNED;
+  if (scale_atoms && !aligned(scales, 16)) return WUSH_ERR_MISALIGNED;
   if (tensor_scale && !aligned(tensor_scale, 4)) return WUSH_ERR_MISALIGNED;
   if (debug && !aligned(y_out, 16)) return WUSH_ERR_MISALIGNED;
 
@@ -184,6 +185,8 @@ int quant_common(const void* in, bool in_f32, const float* T, int64_t rows, int6
 
   wush::FusedParams p{};
   p.codes_via_tma = codes_tma ? 1 : 0;
+  p.scale_atoms = scale_atoms ? 1 : 0;
+  p.atom_cols = static_cast<int>((d_in / G + 3) / 4);
   p.T = T;
   p.codes = codes;
   p.scales = scales;
@@ -342,6 +345,24 @@ int wush_gemm_mxfp4(const uint8_t* a_codes, const uint8_t* a_atoms, const uint8_
   lc.numAttrs = WUSH_USE_PDL ? 1 : 0;
   if (cudaLaunchKernelEx(&lc, wush::wush_gemm_mxf4_kernel, ma, mb, p) != cudaSuccess) return WUSH_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? WUSH_OK : WUSH_ERR_CUDA;
+}
+
+int wush_quant_act_mx_atoms(const void* x_bf16, const float* T_blocks, int64_t n_tok, int64_t d_in, uint8_t* codes,
+                            uint8_t* scale_atoms, wush_stream_t stream) {
+  return quant_common(x_bf16, false, T_blocks, n_tok, d_in, 32, WUSH_MXFP4, codes, scale_atoms, nullptr, nullptr,
+                      false, stream, false, true);
+}
+
+int wush_quant_weight_mx_atoms(const float* w_f32, const float* T_blocks, int64_t d_out, int64_t d_in, uint8_t* codes,
+                               uint8_t* scale_atoms, wush_stream_t stream) {
+  return quant_common(w_f32, true, T_blocks, d_out, d_in, 32, WUSH_MXFP4, codes, scale_atoms, nullptr, nullptr,
+                      false, stream, false, true);
+}
+
+int wush_quant_act_shared_mx_atoms(const void* x_bf16, const float* T_shared, int64_t n_tok, int64_t d_in,
+                                   uint8_t* codes, uint8_t* scale_atoms, wush_stream_t stream) {
+  return quant_common(x_bf16, false, T_shared, n_tok, d_in, 32, WUSH_MXFP4, codes, scale_atoms, nullptr, nullptr,
+                      false, stream, true, true);
 }
 
 int wush_build_transforms(const float* w_f32, const void* xcal_bf16, int64_t d_out, int64_t n_cal, int64_t d_in,

@@ -54,6 +54,8 @@ struct FusedParams {
   int n_row_tiles;
   int total_tiles;
   int codes_via_tma;        // 1: codes leave through the TMA store map (needs d_in % 32 == 0)
+  int scale_atoms;          // MXFP4 only: 1 = scales in the block-scaled MMA's scale-atom layout
+  int atom_cols;            // scale atoms per 128-row block (C padded to 4, / 4)
   unsigned long long wait_limit_ns;
 };
 
@@ -609,7 +611,28 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
       }
       if (Cfg::AMAX_ONLY) continue;
       // scales: this thread's row of the tile, straight from registers
-      if (warp_live && row_ok) {
+      if (Cfg::FMT == kMXFP4 && p.scale_atoms) {
+        // scale-atom layout: row 128 r + i + 32 j, scale column 4 c + k at byte
+        // (r * atom_cols + c) * 512 + 16 i + 4 j + k; this tile's BPT columns are
+        // consecutive k of one atom word
+        if (warp_live && row_ok) {
+          const int col0 = ct * BPT;
+          const int rr = static_cast<int>(grow & 127);
+          uint8_t* word = static_cast<uint8_t*>(p.scales) +
+                          ((grow >> 7) * p.atom_cols + (col0 >> 2)) * 512 + (rr & 31) * 16 + (rr >> 5) * 4;
+          const int nb = min(BPT, C - col0);
+          if constexpr (BPT == 4) {
+            if (nb == 4) {
+              *reinterpret_cast<uint32_t*>(word) = static_cast<uint32_t>(sc[0]) | (static_cast<uint32_t>(sc[1]) << 8) |
+                                                   (static_cast<uint32_t>(sc[2]) << 16) | (static_cast<uint32_t>(sc[3]) << 24);
+            } else {
+              for (int k = 0; k < nb; ++k) word[k] = static_cast<uint8_t>(sc[k]);
+            }
+          } else {
+            for (int k = 0; k < nb; ++k) word[(col0 & 3) + k] = static_cast<uint8_t>(sc[k]);
+          }
+        }
+      } else if (warp_live && row_ok) {
         const int nb = min(BPT, C - ct * BPT);
         ScaleT* dst = reinterpret_cast<ScaleT*>(p.scales) + grow * C + static_cast<long long>(ct) * BPT;
         constexpr int RB = BPT * static_cast<int>(sizeof(ScaleT));   // 2..32 bytes

@@ -147,6 +147,21 @@ int wush_gemm_mxfp4(const uint8_t* a_codes, const uint8_t* a_atoms, const uint8_
                     const uint8_t* b_atoms, int64_t M, int64_t N, int64_t K, void* d_bf16,
                     wush_stream_t stream);
 
+/* MXFP4 (G = 32) quantisation that writes its E8M0 scales straight into the scale-atom
+ * layout wush_gemm_mxfp4 reads (instead of row-major [rows][C]): the same kernels,
+ * codes and errors as wush_quant_act / wush_quant_weight / wush_quant_act_shared with
+ * fmt = MXFP4.  scale_atoms (device) must hold atom_bytes = rows_pad * C_pad bytes
+ * (rows padded to 128, C = d_in / 32 padded to 4); bytes of padding rows and columns
+ * are not written. */
+int wush_quant_act_mx_atoms(const void* x_bf16, const float* T_blocks, int64_t n_tok, int64_t d_in,
+                            uint8_t* codes, uint8_t* scale_atoms, wush_stream_t stream);
+int wush_quant_weight_mx_atoms(const float* w_f32, const float* T_blocks, int64_t d_out,
+                               int64_t d_in, uint8_t* codes, uint8_t* scale_atoms,
+                               wush_stream_t stream);
+int wush_quant_act_shared_mx_atoms(const void* x_bf16, const float* T_shared, int64_t n_tok,
+                                   int64_t d_in, uint8_t* codes, uint8_t* scale_atoms,
+                                   wush_stream_t stream);
+
 /* Row-major E8M0 scales [rows][C] -> the scale-atom layout the block-scaled MMA reads:
  * rows padded to a multiple of 128 and C to a multiple of 4 (zero bytes); the atom of
  * row block r and scale columns [4c, 4c + 4) is the 512 bytes at (r * (C_pad/4) + c) * 512,

@@ -81,3 +81,25 @@ def test_gemm_rejects_unsupported_shapes():
     with pytest.raises(W.WushError):
         W.wush_gemm_mxfp4(a, torch.zeros(W.atom_bytes(100, 8), dtype=torch.uint8, device="cuda"), b,
                           torch.zeros(W.atom_bytes(256, 8), dtype=torch.uint8, device="cuda"))
+
+
+@pytest.mark.parametrize("n_tok,d_in", [(256, 1024), (300, 416), (129, 4096 + 128)])
+def test_quantiser_writes_scale_atoms_directly(n_tok, d_in):
+    wl = workload("attn_mxfp4_4096", n_tok=n_tok, d_in=d_in, d_out=256, n_cal=512)
+    inp = make_inputs(wl)
+    b = O.build_transforms(inp.w, inp.xcal_bits, 32)
+    x = dev(inp.x_bits.view(np.int16)).view(torch.bfloat16)
+    T = dev(b["T_wush32"])
+    c, s, _ = W.wush_quant_act(x, T, 32, "mxfp4")
+    ca, at = W.wush_quant_act_mx_atoms(x, T)
+    cw, sw, _ = W.wush_quant_weight(dev(inp.w), dev(b["T_xvsh32"]), 32, "mxfp4")
+    cwa, atw = W.wush_quant_weight_mx_atoms(dev(inp.w), dev(b["T_xvsh32"]))
+    H = W.hadamard_matrix(32)
+    ch, sh, _ = W.wush_quant_act_shared(x, H, 32, "mxfp4")
+    cha, ath = W.wush_quant_act_shared_mx_atoms(x, H)
+    torch.cuda.synchronize()
+    assert torch.equal(c, ca) and torch.equal(cw, cwa) and torch.equal(ch, cha)
+    # atom buffers start zeroed, so their padding matches the oracle's zero padding
+    assert np.array_equal(at.cpu().numpy(), O.scale_atoms(s.cpu().numpy()))
+    assert np.array_equal(atw.cpu().numpy(), O.scale_atoms(sw.cpu().numpy()))
+    assert np.array_equal(ath.cpu().numpy(), O.scale_atoms(sh.cpu().numpy()))
