@@ -39,6 +39,12 @@ design notes of the repository):
   R8  Packing: byte j holds element 2j in its low nibble and 2j+1 in its high nibble.
   R9  A group whose scale reciprocal fl32(1/S) is not a finite float32 (S = 0, or S so
       small that 1/S overflows) encodes as all zero codes (the pages are silent).
+  R12 GPTQ-WUSH: the target is Y = W^T X' with X' the Cholesky factor of the damped global
+      second moment; per block (reverse order) the SVD of Y's block gives U, S_Y, V,
+      S = S_Y / sqrt(d_out), T_X = H S^1/2 V^T X'_ii^-1, transformed weights
+      sqrt(d_out) H S^1/2 U^T, GPTQ with the block Hessian H S H^T (damped 1 %), and
+      Y -= (quantised weights)^T T_X X'[blk, :] ([graph] §3.4.6, whose formulas are
+      garbled; re-derived from its text and Eq. (8)).  GPTQ-WUSH covers MXFP4 and INT4.
 fl32(.) marks a float32 rounding point: the oracle computes in float64 and rounds
 to float32 there, which equals the IEEE float32 result of a single +, -, *, /.
 """
@@ -439,6 +445,133 @@ def layer_loss(w: np.ndarray, x_bits: np.ndarray, T_w32: np.ndarray, T_x32: np.n
     wq = dequant(unpack_nibbles(cw), sw, fmt, G, tw)
     xq = dequant(unpack_nibbles(cx), sx, fmt, G, tx)
     err = w64 @ x64.T - wq @ xq.T
+    return float(np.sum(err * err) / err.size)
+
+
+# ---------------------------------------------------------------------------
+# GPTQ-WUSH (offline weight quantisation with error feedback)
+# ---------------------------------------------------------------------------
+
+
+def _group_scale(Wb: np.ndarray, fmt: str):
+    """Per-row scale of one G-wide group, fixed from the row's starting values: MXFP4
+    2^e (R5), INT4 s = fl32(amax / 7) (R7).  Returns (scale bytes or values, multiplier
+    used to reach the grid, dequantisation factor)."""
+    amax = np.max(np.abs(Wb), axis=1)
+    if fmt == "mxfp4":
+        e = mxfp4_exponent(amax)
+        return (e + 127).astype(np.uint8), np.exp2(-e.astype(np.float64)), np.exp2(e.astype(np.float64))
+    if fmt == "int4":
+        sc = fl32(amax / 7.0)
+        return sc.astype(np.float32), _recip32(sc), sc
+    raise ValueError("GPTQ-WUSH supports mxfp4 and int4")
+
+
+def _quant_column(w: np.ndarray, mul: np.ndarray, deq: np.ndarray, fmt: str):
+    """One column of a block (one element of every row's group) at the fixed scales:
+    (codes, dequantised values)."""
+    if fmt == "mxfp4":
+        c = e2m1_encode(w * mul)                     # exact: power-of-two multiplier
+        return c, e2m1_decode(c) * deq
+    v = fl32(w * mul)
+    q = np.clip(np.rint(v), -7, 7)
+    return (q.astype(np.int64) & 0xF).astype(np.uint8), q * deq
+
+
+def gptq_block(Wb: np.ndarray, Hb: np.ndarray, fmt: str, damp_frac: float = 0.01):
+    """GPTQ on one block (Frantar et al., 2023, restated): the block's columns are
+    quantised one after the other at the group scales fixed from the starting values;
+    the rounding error of column j, divided by the j-th diagonal of the upper Cholesky
+    factor R of Hb^-1 (Hb^-1 = R^T R), is taken off the later columns in proportion to
+    row j of R.  ``Wb`` is [d_out][G] (rows = output channels), ``Hb`` [G][G] is damped by
+    damp_frac * mean(diag) (the usual GPTQ damping).
+    Returns (dequantised [d_out][G], unpacked codes [d_out][G], scales [d_out])."""
+    W = np.array(Wb, dtype=np.float64, copy=True)
+    G = W.shape[1]
+    Hd = np.asarray(Hb, dtype=np.float64) + damp_frac * np.trace(Hb) / G * np.eye(G)
+    R = np.linalg.cholesky(np.linalg.inv(Hd)).T
+    sc, mul, deq = _group_scale(W, fmt)
+    Q = np.empty_like(W)
+    codes = np.empty(W.shape, np.uint8)
+    for j in range(G):
+        codes[:, j], Q[:, j] = _quant_column(W[:, j], mul, deq, fmt)
+        err = (W[:, j] - Q[:, j]) / R[j, j]
+        W[:, j + 1:] -= np.outer(err, R[j, j + 1:])
+    return Q, codes, sc
+
+
+def gptq_wush(w: np.ndarray, xcal_bits: np.ndarray, G: int, fmt: str, gptq: bool = True, lam: float = 0.01,
+              use_hadamard: bool = True):
+    """GPTQ-WUSH, the pages' interleaved schedule ([graph] §3.4.6 "GPTQ Integration
+    (Algorithm 1)"; the printed formulas are garbled, the steps below are re-derived from
+    the surrounding text and Eq. (8), reading R12):
+
+      Sigma = d_batch^-1 X X^T + lam mean(diag) I,  X' = chol(Sigma) (global, lower),
+      Y = W^T X'                                   (d_out x d_in, the target)
+      for blocks i = C-1 .. 0 (reverse):
+        Y[:, blk] = U S_Y V^T,  S = S_Y / sqrt(d_out)   (sign rule R3 on U's columns)
+        T_X = H S^1/2 V^T X'_ii^-1                  (activation transform, online)
+        T_W = H S^-1/2 V^T X'_ii^T                  (T_W^T T_X = I)
+        W_bar = sqrt(d_out) H S^1/2 U^T              (= T_W applied to the block's
+                                                      effective weights, G x d_out)
+        GPTQ: W~ = GPTQ(W_bar^T, H S H^T);  RTN: W~ = q(W_bar^T)
+        Y -= (GPTQ ? W~ : W_bar^T) T_X X'[blk, :]    (error feedback to earlier blocks)
+
+    Inputs as in ``layer_loss``: w float32 [d_out][d_in], xcal_bits bfloat16 [n][d_in].
+    Returns a dict: T_act, T_w [C][G][G]; W_bar [C][G][d_out]; Wq [d_out][d_in]
+    (dequantised transformed weights); codes [d_out][d_in/2] packed; scales [d_out][C];
+    Y (the final residual target)."""
+    Wt = np.asarray(w, dtype=np.float64)                    # [d_out][d_in] = W^T
+    X = bf16_to_f64(xcal_bits)                              # [n][d_in] = X^T
+    d_out, d_in = Wt.shape
+    n = X.shape[0]
+    C = d_in // G
+    Sig = X.T @ X / n
+    Sig += lam * np.trace(Sig) / d_in * np.eye(d_in)
+    Xp = np.linalg.cholesky(Sig)
+    Y = Wt @ Xp
+    H = sylvester_hadamard(G) if use_hadamard else np.eye(G)
+    out = {"T_act": np.empty((C, G, G)), "T_w": np.empty((C, G, G)), "W_bar": np.empty((C, G, d_out)),
+           "Wq": np.empty((d_out, d_in)), "codes_u": np.empty((d_out, d_in), np.uint8),
+           "scales": np.empty((d_out, C), np.uint8 if fmt == "mxfp4" else np.float32)}
+    for i in reversed(range(C)):
+        blk = slice(i * G, (i + 1) * G)
+        U, sY, Vt = np.linalg.svd(Y[:, blk], full_matrices=False)
+        V = Vt.T
+        for k in range(G):                       # reading R3 on the columns of U
+            j = int(np.argmax(np.abs(U[:, k])))
+            if U[j, k] < 0:
+                U[:, k] = -U[:, k]
+                V[:, k] = -V[:, k]
+        s = sY / np.sqrt(d_out)
+        Xii = Xp[blk, blk]
+        T_x = H @ np.diag(np.sqrt(s)) @ V.T @ np.linalg.inv(Xii)
+        T_w = H @ np.diag(1.0 / np.sqrt(s)) @ V.T @ Xii.T
+        W_bar = np.sqrt(d_out) * H @ np.diag(np.sqrt(s)) @ U.T
+        if gptq:
+            Q, cu, sc = gptq_block(W_bar.T, H @ np.diag(s) @ H.T, fmt)
+            contrib = Q
+        else:
+            cu, sc = quantize(W_bar.T, fmt, G)[:2]
+            Q = dequant(cu, sc.reshape(-1, 1), fmt, G)
+            sc = sc.reshape(-1)
+            contrib = W_bar.T
+        Y -= contrib @ T_x @ Xp[blk, :]
+        out["T_act"][i], out["T_w"][i], out["W_bar"][i] = T_x, T_w, W_bar
+        out["Wq"][:, blk], out["codes_u"][:, blk], out["scales"][:, i] = Q, cu, sc
+    out["codes"] = pack_nibbles(out.pop("codes_u"))
+    out["Y"] = Y
+    return out
+
+
+def layer_loss_prequantised(wq: np.ndarray, w: np.ndarray, x_bits: np.ndarray, T_x32: np.ndarray,
+                            fmt: str, G: int) -> float:
+    """Eq. (5) when the transformed weights are already quantised (GPTQ-WUSH):
+    || W^T X - Wq^T q(T_X X) ||_F^2 / (d_out d_batch), wq [d_out][d_in] dequantised."""
+    x64 = bf16_to_f64(x_bits)
+    cx, sx, tx, _ = quant_act(x_bits, T_x32, G, fmt)
+    xq = dequant(unpack_nibbles(cx), sx, fmt, G, tx)
+    err = np.asarray(w, dtype=np.float64) @ x64.T - np.asarray(wq, dtype=np.float64) @ xq.T
     return float(np.sum(err * err) / err.size)
 
 

@@ -296,6 +296,69 @@ def test_gemm_mx_exact_small_cases():
     assert np.array_equal(d, np.full((M, N), K * 1.5 * -2.0))
 
 
+def test_gptq_block_second_column_takes_the_obs_correction():
+    """Two columns, Hb = [[a, b], [b, c]] undamped: after column 0 is rounded, column 1
+    moves by (w0 - q0) b / c (the optimal brain surgeon update), then is rounded."""
+    a_, b_, c_ = 2.0, 0.7, 1.5
+    Hb = np.array([[a_, b_], [b_, c_]])
+    Wb = np.array([[1.3, 0.4], [-0.9, 2.2], [0.26, -1.1]])
+    Q, codes, sc = O.gptq_block(Wb, Hb, "int4", damp_frac=0.0)
+    s = O.fl32(np.max(np.abs(Wb), axis=1) / 7.0)
+    inv = O._recip32(s)
+    q0 = np.clip(np.rint(O.fl32(Wb[:, 0] * inv)), -7, 7) * s
+    w1 = Wb[:, 1] + (Wb[:, 0] - q0) * b_ / c_
+    q1 = np.clip(np.rint(O.fl32(w1 * inv)), -7, 7) * s
+    assert np.allclose(Q[:, 0], q0, rtol=0, atol=0) and np.allclose(Q[:, 1], q1, rtol=1e-15, atol=0)
+
+
+def test_gptq_block_with_diagonal_hessian_is_plain_rounding():
+    rng = np.random.default_rng(4)
+    Wb = rng.standard_normal((6, 32))
+    for fmt in ("mxfp4", "int4"):
+        Q, codes, sc = O.gptq_block(Wb, np.diag(rng.uniform(0.5, 2.0, 32)), fmt)
+        c_ref, s_ref, _ = O.quantize(Wb, fmt, 32)
+        assert np.array_equal(codes, c_ref) and np.array_equal(sc, s_ref.reshape(-1))
+
+
+def test_gptq_wush_rtn_mode_reconstructs_the_target_exactly():
+    """RTN mode feeds back the unquantised transformed weights, so the residual target
+    vanishes; every block's transforms satisfy T_W^T T_X = I and
+    T_X X'_ii X'_ii^T T_X^T = H S H^T."""
+    wl = workload("tiny_mxfp4")
+    inp = make_inputs(wl)
+    r = O.gptq_wush(inp.w, inp.xcal_bits, 32, "mxfp4", gptq=False)
+    assert np.linalg.norm(r["Y"]) <= 1e-10 * np.linalg.norm(inp.w.astype(np.float64))
+    for i in range(r["T_act"].shape[0]):
+        assert np.max(np.abs(r["T_w"][i].T @ r["T_act"][i] - np.eye(32))) < 1e-9
+
+
+def test_gptq_wush_single_block_agrees_with_the_per_block_construction():
+    """With one block the global factor is the block's own Cholesky factor, so up to the
+    signs of the singular-vector pairs the transforms and transformed weights are those
+    of the per-block WUSH builder: |H^T T| and |H^T W_bar| agree entry by entry."""
+    wl = workload("tiny_mxfp4", d_in=32, d_out=64, n_cal=256)
+    inp = make_inputs(wl)
+    # undamped on both sides (the per-block builder also damps the weight moment)
+    r = O.gptq_wush(inp.w, inp.xcal_bits, 32, "mxfp4", gptq=False, lam=0.0)
+    b = O.build_transforms(inp.w, inp.xcal_bits, 32, lam=0.0)
+    H = O.sylvester_hadamard(32)
+    assert np.allclose(np.abs(H.T @ r["T_act"][0]), np.abs(H.T @ b["T_wush"][0]), rtol=1e-7, atol=1e-9)
+    wbar_ref = b["T_xvsh"][0] @ inp.w.astype(np.float64).T
+    assert np.allclose(np.abs(H.T @ r["W_bar"][0]), np.abs(H.T @ wbar_ref), rtol=1e-7, atol=1e-9)
+
+
+def test_gptq_error_feedback_lowers_the_layer_loss():
+    wl = workload("tiny_mxfp4")
+    inp = make_inputs(wl)
+    for fmt in ("mxfp4", "int4"):
+        losses = {}
+        for gq in (False, True):
+            r = O.gptq_wush(inp.w, inp.xcal_bits, 32, fmt, gptq=gq)
+            losses[gq] = O.layer_loss_prequantised(r["Wq"], inp.w, inp.xcal_bits, r["T_act"].astype(np.float32),
+                                                   fmt, 32)
+        assert losses[True] < 0.95 * losses[False], (fmt, losses)
+
+
 # ---------------------------------------------------------------- grids, brute force
 
 
