@@ -345,9 +345,10 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
   };
   // Thread 0, which initialised the barriers, issues the first input tile, then the
   // transform copies of the CTA's first (and, if its tiles reach it, second) column tile,
-  // then the remaining input stages (this order measured fastest: the first tile and its
-  // matrices arrive together, ahead of the rest of the burst).  Every converter thread
-  // knows which copies exist.
+  // then the second input tile; the producer loop issues the other stages after the
+  // set-up (this order and depth measured fastest: the first tile and its matrices
+  // arrive ahead of the rest of the burst).  Every converter thread knows which copies
+  // exist.
   const bool t_second = !Cfg::SHARED_T && t_begin < t_end && (t_end - 1) / nrt > t_begin / nrt;
   int t_issued[2] = {t_begin < t_end ? 1 : 0, t_second ? 1 : 0};
   const uint64_t l2_pol = l2_policy_evict_first();
@@ -368,7 +369,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
     issue_x();
     if (t_begin < t_end) t_copy(t_begin / nrt, 0);
     if (t_second) t_copy(t_begin / nrt + 1, 1);
-    while (n_preloaded < STAGES && t_begin + n_preloaded < t_end) issue_x();
+    while (n_preloaded < 2 && t_begin + n_preloaded < t_end) issue_x();   // the rest after the set-up
   }
   __syncwarp();
   if (warp == 1) {
