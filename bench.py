@@ -48,6 +48,8 @@ def parse_args():
     ap.add_argument("--e2e-steps", type=int, default=30)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-rows", action="store_true",
+                    help="skip the per-configuration rows (NVFP4, large batch, weights, INT4 sweep, FP4 GEMM)")
     return ap.parse_args()
 
 
@@ -224,6 +226,132 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def _time_calls(fn, stream, n_calls: int, reps: int = 3) -> float:
+    """Seconds per call of fn, from CUDA graphs of n_calls launches replayed on stream
+    (CUDA events on that stream, best of reps)."""
+    import torch
+    with torch.cuda.stream(stream):
+        for i in range(3):
+            fn(i)
+        stream.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for i in range(n_calls):
+                fn(i)
+        g.replay()
+        stream.synchronize()
+        best = float("inf")
+        for _ in range(reps):
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            g.replay()
+            e1.record(stream)
+            e1.synchronize()
+            best = min(best, e0.elapsed_time(e1) / 1e3 / n_calls)
+    del g
+    return best
+
+
+def config_rows(dev, peak_gbs: float) -> dict:
+    """The other configurations of the hot path, each timed the same way (graphs, inputs
+    rotated over two sets whose total exceeds L2 where the size allows), with its
+    algorithmic bytes and fraction of the HBM peak; plus the MXFP4 GEMM consumer at one of
+    the pages' M = 1024 shapes against the FP4 tensor roofline."""
+    import numpy as np
+    import torch
+    import blockwise_adaptive_transforms_b200 as W
+    from workloads import make_inputs, workload
+    from workloads.synthetic import INT4_SWEEP_TOKENS
+
+    rows = {}
+    stream = torch.cuda.Stream(device=dev)
+
+    def bf16_dev(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
+
+    def row(name, seconds, nbytes, note=None, **extra):
+        r = {"us": round(seconds * 1e6, 3), "GB/s": round(nbytes / seconds / 1e9, 1),
+             "hbm_frac": round(nbytes / seconds / 1e9 / peak_gbs, 4), "algorithmic_bytes": nbytes}
+        if note:
+            r["note"] = note
+        r.update(extra)
+        rows[name] = r
+
+    # NVFP4 MLP down-projection input, 4096 x 14336, G = 16 (two passes + tensor-scale finalise)
+    wl = workload("mlp_down_nvfp4_14336")
+    inp = make_inputs(wl)
+    T, _ = W.wush_build_transforms(torch.from_numpy(inp.w).to(dev), bf16_dev(inp.xcal_bits), wl.G)
+    xs = [bf16_dev(inp.x_bits) for _ in range(2)]
+    outs = [W.wush_quant_act(xs[0], T, wl.G, "nvfp4") for _ in range(2)]
+    sec = _time_calls(lambda i: W.wush_quant_act(xs[i % 2], T, wl.G, "nvfp4", codes=outs[i % 2][0],
+                                                 scales=outs[i % 2][1], tensor_scale=outs[i % 2][2], stream=stream),
+                      stream, 20)
+    n, d, C = wl.n_tok, wl.d_in, wl.d_in // wl.G
+    one_read = n * d * 2 + n * d // 2 + n * C + C * wl.G * wl.G * 4 + 4
+    row("nvfp4_4096x14336", sec, one_read, "bytes count X once; the two passes move "
+        f"{one_read + n * d * 2 + C * wl.G * wl.G * 4} B", moved_GB_s=round((one_read + n * d * 2 + C * wl.G * wl.G * 4) / sec / 1e9, 1))
+    del xs, outs, inp
+
+    # 70B-like large batch: activations 16384 x 8192 and weights 8192 x 8192, MXFP4
+    wl = workload("large_mxfp4_8192")
+    inp = make_inputs(wl)
+    w_dev = torch.from_numpy(inp.w).to(dev)
+    T_act, T_wt = W.wush_build_transforms(w_dev, bf16_dev(inp.xcal_bits), wl.G)   # T_wush, T_xvsh
+    n, d, C = wl.n_tok, wl.d_in, wl.d_in // wl.G
+    xs = [bf16_dev(inp.x_bits) for _ in range(2)]
+    outs = [W.wush_quant_act(xs[0], T_act, wl.G, "mxfp4") for _ in range(2)]
+    sec = _time_calls(lambda i: W.wush_quant_act(xs[i % 2], T_act, wl.G, "mxfp4", codes=outs[i % 2][0],
+                                                 scales=outs[i % 2][1], stream=stream), stream, 20)
+    row("mxfp4_act_16384x8192", sec, algorithmic_bytes(n, d, wl.G))
+    del xs, outs
+    ws = [w_dev, w_dev.clone()]
+    d_out = ws[0].shape[0]
+    wouts = [W.wush_quant_weight(ws[0], T_wt, wl.G, "mxfp4") for _ in range(2)]
+    sec = _time_calls(lambda i: W.wush_quant_weight(ws[i % 2], T_wt, wl.G, "mxfp4", codes=wouts[i % 2][0],
+                                                    scales=wouts[i % 2][1], stream=stream), stream, 20)
+    row("mxfp4_weight_8192x8192", sec, d_out * d * 4 + d_out * d // 2 + d_out * C + C * wl.G * wl.G * 4)
+    del ws, wouts, inp, w_dev
+
+    # INT4, G = 32, d_in = 4096, token sweep (the small batches are launch-bound)
+    wl = workload("int4_sweep_4096")
+    inp = make_inputs(wl)
+    T, _ = W.wush_build_transforms(torch.from_numpy(inp.w).to(dev), bf16_dev(inp.xcal_bits), wl.G)
+    sweep = {}
+    for n in INT4_SWEEP_TOKENS:
+        xs = [bf16_dev(inp.x_bits[:n]) for _ in range(2)]
+        outs = [W.wush_quant_act(xs[0], T, wl.G, "int4") for _ in range(2)]
+        sec = _time_calls(lambda i: W.wush_quant_act(xs[i % 2], T, wl.G, "int4", codes=outs[i % 2][0],
+                                                     scales=outs[i % 2][1], stream=stream), stream, 50)
+        nbytes = n * wl.d_in * 2 + n * wl.d_in // 2 + n * (wl.d_in // wl.G) * 4 + (wl.d_in // wl.G) * wl.G * wl.G * 4
+        sweep[str(n)] = {"us": round(sec * 1e6, 3), "GB/s": round(nbytes / sec / 1e9, 1)}
+    rows["int4_4096_token_sweep"] = dict(sweep, note="inputs of 1 to 1024 tokens stay in L2; n <= 128 is launch-bound")
+    del inp
+
+    # MXFP4 GEMM consumer, M = 1024, N = K = 4096 (Qwen3-8B square projection)
+    M, N, K = 1024, 4096, 4096
+    g = torch.Generator().manual_seed(7)
+    x = torch.randn(M, K, generator=g).to(torch.bfloat16).to(dev)
+    w = (torch.randn(N, K, generator=g) / K ** 0.5).to(dev)
+    Tg = (torch.eye(32) + 0.1 * torch.randn(K // 32, 32, 32, generator=g)).to(dev)
+    cw, aw = W.wush_quant_weight_mx_atoms(w, Tg)
+    cx, ax = W.wush_quant_act_mx_atoms(x, Tg)
+    out = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    sec = _time_calls(lambda i: W.wush_gemm_mxfp4(cx, ax, cw, aw, out=out, stream=stream), stream, 50)
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            bf16_peak, kind = float(json.load(f)["bf16_tflops"]), "measured"
+    except (OSError, KeyError, ValueError):
+        bf16_peak, kind = 1590.0, "fallback"
+    tflops = 2.0 * M * N * K / sec / 1e12
+    rows["fp4_gemm_1024x4096x4096"] = {"us": round(sec * 1e6, 3), "TFLOP/s": round(tflops, 1),
+                                       "tensor_frac": round(tflops / (4 * bf16_peak), 4),
+                                       "peak_TFLOP_s": round(4 * bf16_peak, 1),
+                                       "peak_source": f"4 x {kind} bf16 (nominal fp4/bf16 ratio)"}
+    torch.cuda.synchronize()
+    return rows
+
+
 def run_native(args):
     import numpy as np
     import torch
@@ -382,6 +510,11 @@ def run_native(args):
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(inp, wl, args.cpu_seconds)
+    rows = None
+    if world == 1 and not args.no_rows:
+        del xs, codes, scales
+        torch.cuda.empty_cache()
+        rows = config_rows(dev, peak)
 
     if world > 1:
         dist.barrier()
@@ -411,6 +544,7 @@ def run_native(args):
                     "launches": h_reps * GRAPH_LEN,
                     "wush_time_over_h_time": round(per_launch_s / h_per_launch_s, 4),
                     "what": "same fused kernel, one shared Hadamard matrix for every block"},
+        "rows": rows,
         "gpu_launches": args.steps,
         "clocks": clk,
     }
