@@ -85,7 +85,10 @@ struct FusedCfg {
   static constexpr int ACC_COLS = 2 * CH;              // hi|lo of every block of a tile
   static constexpr int NACC = 512 / ACC_COLS;          // accumulator buffers in TMEM
   static constexpr int TMEM_COLS = NACC * ACC_COLS;
-  static constexpr int N_GROUPS = 2;                   // epilogue groups, alternate tiles
+  // fp32 (weight) tiles need their hi/lo split, a job for more threads than the two
+  // converter warps: there warps 8-11 convert too and one epilogue group remains
+  static constexpr int N_GROUPS = IN_F32 ? 1 : 2;      // epilogue groups, alternate tiles
+  static constexpr int CONV_THREADS = IN_F32 ? 192 : 64;
   static constexpr int GROUP_WARPS = 4;                // one warp per TMEM lane quadrant
   static constexpr int THREADS = 12 * 32;
   static constexpr int CODE_STAGE = 128 * CH / 2;      // one tile of packed codes
@@ -273,10 +276,10 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(BAR(B_FULL + s), 1);
-      mbar_init(BAR(B_EMPTY + s), Cfg::IN_F32 ? 64 : 1);
+      mbar_init(BAR(B_EMPTY + s), Cfg::IN_F32 ? Cfg::CONV_THREADS : 1);
     }
     for (int k = 0; k < 2; ++k) {
-      mbar_init(BAR(B_OFULL + k), 64);
+      mbar_init(BAR(B_OFULL + k), Cfg::CONV_THREADS);
       mbar_init(BAR(B_OEMPTY + k), 1);
       mbar_init(BAR(B_TFULL + k), 64);
       mbar_init(BAR(B_TEMPTY + k), 1);
@@ -474,16 +477,19 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
       volatile int no_abort = 0;
       wait_bounded(BAR(B_DRAIN), 0u, &no_abort, 16u, lim);
     }
-  } else if (warp < 4) {
-    // ------------------------------------------------------------ converters (64 threads)
-    const int v0 = threadIdx.x - 64;
+  } else if (warp < 4 || (Cfg::IN_F32 && warp >= 8)) {
+    // ------------------------------------------------------------ converters
+    // warps 2-3 (ids 0..63) split the transforms; on the fp32 path warps 2-3 and 8-11
+    // (ids 0..191) split the input tiles
+    const int v0 = warp < 4 ? threadIdx.x - 64 : 64 + (threadIdx.x - 256);
+    const bool t_conv = v0 < 64;
     int t_landed[2] = {0, 0};
     int epoch = -1, prev_ct = -1;
     int stage = 0, obuf = 0;
     uint32_t phase = 0, ophase = 0;
     for (int t = t_begin; t < t_end; ++t) {
       const int ct = t / nrt;
-      if (Cfg::SHARED_T ? t == t_begin : ct != prev_ct) {
+      if (t_conv && (Cfg::SHARED_T ? t == t_begin : ct != prev_ct)) {
         ++epoch;
         prev_ct = ct;
         const int slot = epoch & 1;
@@ -511,7 +517,11 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
         uint8_t* dhi = smem + Cfg::OFF_OPER + obuf * 2 * Cfg::OPER_BYTES;
         uint8_t* dlo = dhi + Cfg::OPER_BYTES;
         constexpr int CPR = CH / 8;    // 16-byte output chunks per row
-        for (int q = v0; q < 128 * CPR; q += 64) {
+        constexpr int PER = (128 * CPR + Cfg::CONV_THREADS - 1) / Cfg::CONV_THREADS;
+#pragma unroll
+        for (int k = 0; k < PER; ++k) {
+          const int q = v0 + k * Cfg::CONV_THREADS;
+          if (q >= 128 * CPR) break;
           const int r = q / CPR, j = q - r * CPR;
           const float4* s4 = reinterpret_cast<const float4*>(src + r * CH * 4 + j * 32);
           const float4 u0 = s4[0], u1 = s4[1];
@@ -541,7 +551,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
     // those tiles; the groups run independently, so one group's TMEM loads, barrier and
     // store overlap the other group's arithmetic.  Thread = token row of the tile; it
     // handles the tile's blocks one after the other.
-    const int grp = (warp - 4) >> 2;           // epilogue group
+    const int grp = (warp - 4) >> 2;           // epilogue group (warps 4-7: 0, 8-11: 1)
     const int quad = warp & 3;                 // TMEM lanes this warp may read
     const int row = quad * 32 + lane;          // row within the tile
     const bool store_leader = (quad == 0) && lane == 0;
