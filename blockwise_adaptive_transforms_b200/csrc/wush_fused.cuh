@@ -117,21 +117,30 @@ __device__ __forceinline__ uint32_t sw128_off(int row, int chunk) {
   return static_cast<uint32_t>(row * 128 + ((chunk ^ (row & 7)) << 4));
 }
 
-__device__ __forceinline__ uint32_t bf16x2_bits(__nv_bfloat16 lo, __nv_bfloat16 hi) {
-  return static_cast<uint32_t>(__bfloat16_as_ushort(lo)) |
-         (static_cast<uint32_t>(__bfloat16_as_ushort(hi)) << 16);
-}
 
-// Split 8 fp32 values into bf16 hi = rn(v) and lo = rn(v - hi), packed 2 per word.
+// Split 8 fp32 values into bf16 hi = rn(v) and lo = rn(v - hi), packed 2 per word (the
+// first value in the low half).  v - hi is exact in fp32, so lo is the one rounding of
+// the remainder; pairs go through cvt.rn.bf16x2.f32 and one packed fp32 subtraction.
+__device__ __forceinline__ uint32_t cvt_bf16x2(float lo_half, float hi_half) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi_half), "f"(lo_half));
+  return r;
+}
 __device__ __forceinline__ void split8(const float* v, uint4& hi, uint4& lo) {
   uint32_t h[4], l[4];
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
-    __nv_bfloat16 a = __float2bfloat16_rn(v[2 * k]), b = __float2bfloat16_rn(v[2 * k + 1]);
-    __nv_bfloat16 ar = __float2bfloat16_rn(v[2 * k] - __bfloat162float(a));
-    __nv_bfloat16 br = __float2bfloat16_rn(v[2 * k + 1] - __bfloat162float(b));
-    h[k] = bf16x2_bits(a, b);
-    l[k] = bf16x2_bits(ar, br);
+    h[k] = cvt_bf16x2(v[2 * k], v[2 * k + 1]);
+    float r0 = v[2 * k], r1 = v[2 * k + 1];
+    const float b0 = __uint_as_float(h[k] << 16), b1 = __uint_as_float(h[k] & 0xFFFF0000u);
+    asm("{\n\t.reg .b64 ra, rb;\n\t"
+        "mov.b64 ra, {%0, %1};\n\t"
+        "mov.b64 rb, {%2, %3};\n\t"
+        "sub.rn.f32x2 ra, ra, rb;\n\t"
+        "mov.b64 {%0, %1}, ra;\n\t}"
+        : "+f"(r0), "+f"(r1)
+        : "f"(b0), "f"(b1));
+    l[k] = cvt_bf16x2(r0, r1);
   }
   hi = make_uint4(h[0], h[1], h[2], h[3]);
   lo = make_uint4(l[0], l[1], l[2], l[3]);
