@@ -256,8 +256,8 @@ def _time_calls(fn, stream, n_calls: int, reps: int = 3) -> float:
 def config_rows(dev, peak_gbs: float) -> dict:
     """The other configurations of the hot path, each timed the same way (graphs, inputs
     rotated over two sets whose total exceeds L2 where the size allows), with its
-    algorithmic bytes and fraction of the HBM peak; plus the MXFP4 GEMM consumer at one of
-    the pages' M = 1024 shapes against the FP4 tensor roofline."""
+    algorithmic bytes and fraction of the HBM peak; plus the MXFP4 and NVFP4 GEMM consumers
+    at one of the pages' M = 1024 shapes against the FP4 tensor roofline."""
     import numpy as np
     import torch
     import blockwise_adaptive_transforms_b200 as W
@@ -348,6 +348,16 @@ def config_rows(dev, peak_gbs: float) -> dict:
                                        "tensor_frac": round(tflops / (4 * bf16_peak), 4),
                                        "peak_TFLOP_s": round(4 * bf16_peak, 1),
                                        "peak_source": f"4 x {kind} bf16 (nominal fp4/bf16 ratio)"}
+    # the same shape with NVFP4 operands (G = 16 transforms, E4M3 scales, tensor scales)
+    Tn = (torch.eye(16) + 0.1 * torch.randn(K // 16, 16, 16, generator=g)).to(dev)
+    cwn, awn, twn = W.wush_quant_weight_nv_atoms(w, Tn)
+    cxn, axn, txn = W.wush_quant_act_nv_atoms(x, Tn)
+    sec = _time_calls(lambda i: W.wush_gemm_nvfp4(cxn, axn, txn, cwn, awn, twn, out=out, stream=stream), stream, 50)
+    tflops = 2.0 * M * N * K / sec / 1e12
+    rows["nvfp4_gemm_1024x4096x4096"] = {"us": round(sec * 1e6, 3), "TFLOP/s": round(tflops, 1),
+                                         "tensor_frac": round(tflops / (4 * bf16_peak), 4),
+                                         "peak_TFLOP_s": round(4 * bf16_peak, 1),
+                                         "peak_source": f"4 x {kind} bf16 (nominal fp4/bf16 ratio)"}
     torch.cuda.synchronize()
     return rows
 
@@ -413,6 +423,9 @@ def run_native(args):
         while done < args.warmup:
             graph.replay()
             done += GRAPH_LEN
+        graph.replay()                      # each graph once before the timed region: its
+        if tail is not None:                # first replay uploads it to the device
+            tail.replay()
         stream.synchronize()
     st, bits = W.wush_device_status(stream)
     if st != 0:

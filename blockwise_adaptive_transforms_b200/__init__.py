@@ -21,7 +21,8 @@ __all__ = ["FMT", "WushError", "wush_quant_act", "wush_quant_weight", "wush_quan
            "wush_selftest_wait_timeout", "wush_status_string", "wush_version", "load_library",
            "EXPORTED_SYMBOLS", "output_shapes", "hadamard_matrix", "wush_dequant", "wush_gemm_mxfp4",
            "wush_mx_scales_to_atoms", "atom_bytes", "wush_quant_act_mx_atoms", "wush_quant_weight_mx_atoms",
-           "wush_quant_act_shared_mx_atoms"]
+           "wush_quant_act_shared_mx_atoms", "wush_gemm_nvfp4", "wush_quant_act_nv_atoms",
+           "wush_quant_weight_nv_atoms"]
 
 FMT = {"mxfp4": 0, "nvfp4": 1, "int4": 2}
 STATUS = {0: "WUSH_OK", 1: "WUSH_ERR_INVALID_ARG", 2: "WUSH_ERR_UNSUPPORTED", 3: "WUSH_ERR_MISALIGNED",
@@ -30,6 +31,7 @@ EXPORTED_SYMBOLS = ("wush_quant_act", "wush_quant_weight", "wush_quant_act_debug
                     "wush_quant_weight_debug", "wush_quant_act_shared", "wush_quant_act_shared_debug",
                     "wush_dequant", "wush_gemm_mxfp4", "wush_mx_scales_to_atoms", "wush_quant_act_mx_atoms",
                     "wush_quant_weight_mx_atoms", "wush_quant_act_shared_mx_atoms",
+                    "wush_gemm_nvfp4", "wush_quant_act_nv_atoms", "wush_quant_weight_nv_atoms",
                     "wush_build_transforms", "wush_device_status",
                     "wush_set_wait_limit_ns",
                     "wush_selftest_wait_timeout", "wush_status_string", "wush_version")
@@ -70,8 +72,13 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
     for f in ("wush_quant_act_mx_atoms", "wush_quant_weight_mx_atoms", "wush_quant_act_shared_mx_atoms"):
         getattr(lib, f).argtypes = [_P, _P, _I64, _I64, _P, _P, _P]
         getattr(lib, f).restype = ctypes.c_int
+    for f in ("wush_quant_act_nv_atoms", "wush_quant_weight_nv_atoms"):
+        getattr(lib, f).argtypes = [_P, _P, _I64, _I64, _P, _P, _P, _P]
+        getattr(lib, f).restype = ctypes.c_int
     lib.wush_gemm_mxfp4.argtypes = [_P, _P, _P, _P, _I64, _I64, _I64, _P, _P]
     lib.wush_gemm_mxfp4.restype = ctypes.c_int
+    lib.wush_gemm_nvfp4.argtypes = [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _P]
+    lib.wush_gemm_nvfp4.restype = ctypes.c_int
     lib.wush_mx_scales_to_atoms.argtypes = [_P, _I64, _I64, _P, _P]
     lib.wush_mx_scales_to_atoms.restype = ctypes.c_int
     lib.wush_build_transforms.argtypes = [_P, _P, _I64, _I64, _I64, _I32, ctypes.c_double, _I32,
@@ -264,29 +271,35 @@ def wush_mx_scales_to_atoms(scales, out=None, stream=None):
     return out
 
 
-def _quant_atoms(fn_name, inp, in_dtype, T, codes, atoms, stream, shared=False):
+def _quant_atoms(fn_name, inp, in_dtype, T, codes, atoms, stream, shared=False, G=32, tensor_scale=None):
     lib = load_library()
     _check_dev(inp, "input", in_dtype)
     _check_dev(T, "T", torch.float32)
     rows, d_in = int(inp.shape[0]), int(inp.shape[1])
-    if d_in % 32:
-        raise ValueError("d_in must be a multiple of 32")
-    t_shape = (32, 32) if shared else (d_in // 32, 32, 32)
+    if d_in % G:
+        raise ValueError(f"d_in must be a multiple of {G}")
+    t_shape = (G, G) if shared else (d_in // G, G, G)
     if tuple(T.shape) != t_shape:
         raise ValueError(f"T must have shape {t_shape}")
     if codes is None:
         codes = torch.empty((rows, d_in // 2), dtype=torch.uint8, device=inp.device)
     if atoms is None:
-        atoms = torch.zeros(atom_bytes(rows, d_in // 32), dtype=torch.uint8, device=inp.device)
+        atoms = torch.zeros(atom_bytes(rows, d_in // G), dtype=torch.uint8, device=inp.device)
     _check_dev(codes, "codes", torch.uint8)
     _check_dev(atoms, "scale atoms", torch.uint8)
-    if tuple(codes.shape) != (rows, d_in // 2) or atoms.numel() < atom_bytes(rows, d_in // 32):
+    if tuple(codes.shape) != (rows, d_in // 2) or atoms.numel() < atom_bytes(rows, d_in // G):
         raise ValueError("output buffers have the wrong size")
+    args = [_ptr(inp), _ptr(T), rows, d_in, _ptr(codes), _ptr(atoms)]
+    if G == 16:
+        if tensor_scale is None:
+            tensor_scale = torch.empty(1, dtype=torch.float32, device=inp.device)
+        _check_dev(tensor_scale, "tensor_scale", torch.float32)
+        args.append(_ptr(tensor_scale))
     with torch.cuda.device(inp.device):
-        st = getattr(lib, fn_name)(_ptr(inp), _ptr(T), rows, d_in, _ptr(codes), _ptr(atoms), _stream_handle(stream))
+        st = getattr(lib, fn_name)(*args, _stream_handle(stream))
     if st != 0:
         raise WushError(st, fn_name)
-    return codes, atoms
+    return (codes, atoms) if G == 32 else (codes, atoms, tensor_scale)
 
 
 def wush_quant_act_mx_atoms(x, T, codes=None, atoms=None, stream=None):
@@ -302,9 +315,19 @@ def wush_quant_act_shared_mx_atoms(x, T, codes=None, atoms=None, stream=None):
     return _quant_atoms("wush_quant_act_shared_mx_atoms", x, torch.bfloat16, T, codes, atoms, stream, shared=True)
 
 
-def wush_gemm_mxfp4(a_codes, a_atoms, b_codes, b_atoms, out=None, stream=None):
-    """bf16 [M][N] = A B^T from MXFP4 codes ([M][K/2], [N][K/2]) and scale atoms."""
-    lib = load_library()
+def wush_quant_act_nv_atoms(x, T, codes=None, atoms=None, tensor_scale=None, stream=None):
+    """NVFP4 activations with the E4M3 scales in the scale-atom layout:
+    (codes, atoms, tensor_scale)."""
+    return _quant_atoms("wush_quant_act_nv_atoms", x, torch.bfloat16, T, codes, atoms, stream, G=16,
+                        tensor_scale=tensor_scale)
+
+
+def wush_quant_weight_nv_atoms(w, T, codes=None, atoms=None, tensor_scale=None, stream=None):
+    return _quant_atoms("wush_quant_weight_nv_atoms", w, torch.float32, T, codes, atoms, stream, G=16,
+                        tensor_scale=tensor_scale)
+
+
+def _gemm_args(a_codes, a_atoms, b_codes, b_atoms, out, vs):
     for t, n in ((a_codes, "a_codes"), (b_codes, "b_codes"), (a_atoms, "a_atoms"), (b_atoms, "b_atoms")):
         _check_dev(t, n, torch.uint8)
     M, K2 = int(a_codes.shape[0]), int(a_codes.shape[1])
@@ -312,18 +335,40 @@ def wush_gemm_mxfp4(a_codes, a_atoms, b_codes, b_atoms, out=None, stream=None):
     if int(b_codes.shape[1]) != K2:
         raise ValueError("A and B must share K")
     K = 2 * K2
-    if a_atoms.numel() < atom_bytes(M, K // 32) or b_atoms.numel() < atom_bytes(N, K // 32):
+    if a_atoms.numel() < atom_bytes(M, K // vs) or b_atoms.numel() < atom_bytes(N, K // vs):
         raise ValueError("scale atom buffers too small")
     if out is None:
         out = torch.empty((M, N), dtype=torch.bfloat16, device=a_codes.device)
     _check_dev(out, "out", torch.bfloat16)
     if tuple(out.shape) != (M, N):
         raise ValueError("out must be [M][N]")
+    return M, N, K, out
+
+
+def wush_gemm_mxfp4(a_codes, a_atoms, b_codes, b_atoms, out=None, stream=None):
+    """bf16 [M][N] = A B^T from MXFP4 codes ([M][K/2], [N][K/2]) and scale atoms."""
+    lib = load_library()
+    M, N, K, out = _gemm_args(a_codes, a_atoms, b_codes, b_atoms, out, 32)
     with torch.cuda.device(a_codes.device):
         st = lib.wush_gemm_mxfp4(_ptr(a_codes), _ptr(a_atoms), _ptr(b_codes), _ptr(b_atoms), M, N, K, _ptr(out),
                                  _stream_handle(stream))
     if st != 0:
         raise WushError(st, "wush_gemm_mxfp4")
+    return out
+
+
+def wush_gemm_nvfp4(a_codes, a_atoms, a_tensor_scale, b_codes, b_atoms, b_tensor_scale, out=None, stream=None):
+    """bf16 [M][N] = s_A s_B A B^T from NVFP4 codes, E4M3 scale atoms and the two fp32
+    tensor scales (device tensors of one element)."""
+    lib = load_library()
+    M, N, K, out = _gemm_args(a_codes, a_atoms, b_codes, b_atoms, out, 16)
+    _check_dev(a_tensor_scale, "a_tensor_scale", torch.float32)
+    _check_dev(b_tensor_scale, "b_tensor_scale", torch.float32)
+    with torch.cuda.device(a_codes.device):
+        st = lib.wush_gemm_nvfp4(_ptr(a_codes), _ptr(a_atoms), _ptr(a_tensor_scale), _ptr(b_codes), _ptr(b_atoms),
+                                 _ptr(b_tensor_scale), M, N, K, _ptr(out), _stream_handle(stream))
+    if st != 0:
+        raise WushError(st, "wush_gemm_nvfp4")
     return out
 
 

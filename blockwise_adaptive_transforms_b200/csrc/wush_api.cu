@@ -293,17 +293,26 @@ int wush_mx_scales_to_atoms(const uint8_t* scales, int64_t rows, int64_t C, uint
   return cudaGetLastError() == cudaSuccess ? WUSH_OK : WUSH_ERR_CUDA;
 }
 
-int wush_gemm_mxfp4(const uint8_t* a_codes, const uint8_t* a_atoms, const uint8_t* b_codes, const uint8_t* b_atoms,
-                    int64_t M, int64_t N, int64_t K, void* d_bf16, wush_stream_t stream) {
-  using Cfg = wush::GemmCfg;
+}  // extern "C"
+
+namespace {
+
+// One launch of the block-scaled FP4 GEMM (MXFP4 or NVFP4 operands).
+template <bool NV>
+int gemm_fp4(const uint8_t* a_codes, const uint8_t* a_atoms, const float* a_ts, const uint8_t* b_codes,
+             const uint8_t* b_atoms, const float* b_ts, int64_t M, int64_t N, int64_t K, void* d_bf16,
+             wush_stream_t stream) {
+  using Cfg = wush::GemmCfg<NV>;
   if (M < 0 || N <= 0 || K <= 0) return WUSH_ERR_INVALID_ARG;
   if (M % Cfg::BM || N % Cfg::BN || K % Cfg::BK) return WUSH_ERR_UNSUPPORTED;
   if (M > INT_MAX || N > INT_MAX || K > INT_MAX) return WUSH_ERR_INVALID_ARG;
   if (M == 0) return WUSH_OK;
   if (!a_codes || !a_atoms || !b_codes || !b_atoms || !d_bf16) return WUSH_ERR_INVALID_ARG;
+  if (NV && (!a_ts || !b_ts)) return WUSH_ERR_INVALID_ARG;
   if (!aligned(a_codes, 16) || !aligned(b_codes, 16) || !aligned(a_atoms, 16) || !aligned(b_atoms, 16) ||
       !aligned(d_bf16, 16))
     return WUSH_ERR_MISALIGNED;
+  if (NV && (!aligned(a_ts, 4) || !aligned(b_ts, 4))) return WUSH_ERR_MISALIGNED;
   CUtensorMap ma, mb;
   int st = encode_u8_sw128(&ma, a_codes, M, K / 2, 128, Cfg::BM);
   if (st != WUSH_OK) return st;
@@ -312,6 +321,8 @@ int wush_gemm_mxfp4(const uint8_t* a_codes, const uint8_t* a_atoms, const uint8_
   wush::GemmParams p{};
   p.sfa = a_atoms;
   p.sfb = b_atoms;
+  p.ts_a = a_ts;
+  p.ts_b = b_ts;
   p.d = static_cast<__nv_bfloat16*>(d_bf16);
   p.M = static_cast<int>(M);
   p.N = static_cast<int>(N);
@@ -325,7 +336,7 @@ int wush_gemm_mxfp4(const uint8_t* a_codes, const uint8_t* a_atoms, const uint8_
   static std::atomic<unsigned long long> configured{0ull};
   const unsigned long long bit = 1ull << (dev & 63);
   if (!(configured.load(std::memory_order_acquire) & bit)) {
-    if (cudaFuncSetAttribute(wush::wush_gemm_mxf4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(wush::wush_gemm_fp4_kernel<Cfg>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              Cfg::SMEM_BYTES) != cudaSuccess)
       return WUSH_ERR_CUDA;
     configured.fetch_or(bit, std::memory_order_acq_rel);
@@ -343,8 +354,23 @@ int wush_gemm_mxfp4(const uint8_t* a_codes, const uint8_t* a_atoms, const uint8_
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   lc.attrs = attr;
   lc.numAttrs = WUSH_USE_PDL ? 1 : 0;
-  if (cudaLaunchKernelEx(&lc, wush::wush_gemm_mxf4_kernel, ma, mb, p) != cudaSuccess) return WUSH_ERR_CUDA;
+  if (cudaLaunchKernelEx(&lc, wush::wush_gemm_fp4_kernel<Cfg>, ma, mb, p) != cudaSuccess) return WUSH_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? WUSH_OK : WUSH_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+int wush_gemm_mxfp4(const uint8_t* a_codes, const uint8_t* a_atoms, const uint8_t* b_codes, const uint8_t* b_atoms,
+                    int64_t M, int64_t N, int64_t K, void* d_bf16, wush_stream_t stream) {
+  return gemm_fp4<false>(a_codes, a_atoms, nullptr, b_codes, b_atoms, nullptr, M, N, K, d_bf16, stream);
+}
+
+int wush_gemm_nvfp4(const uint8_t* a_codes, const uint8_t* a_atoms, const float* a_tensor_scale,
+                    const uint8_t* b_codes, const uint8_t* b_atoms, const float* b_tensor_scale, int64_t M, int64_t N,
+                    int64_t K, void* d_bf16, wush_stream_t stream) {
+  return gemm_fp4<true>(a_codes, a_atoms, a_tensor_scale, b_codes, b_atoms, b_tensor_scale, M, N, K, d_bf16, stream);
 }
 
 int wush_quant_act_mx_atoms(const void* x_bf16, const float* T_blocks, int64_t n_tok, int64_t d_in, uint8_t* codes,
@@ -363,6 +389,18 @@ int wush_quant_act_shared_mx_atoms(const void* x_bf16, const float* T_shared, in
                                    uint8_t* codes, uint8_t* scale_atoms, wush_stream_t stream) {
   return quant_common(x_bf16, false, T_shared, n_tok, d_in, 32, WUSH_MXFP4, codes, scale_atoms, nullptr, nullptr,
                       false, stream, true, true);
+}
+
+int wush_quant_act_nv_atoms(const void* x_bf16, const float* T_blocks, int64_t n_tok, int64_t d_in, uint8_t* codes,
+                            uint8_t* scale_atoms, float* tensor_scale, wush_stream_t stream) {
+  return quant_common(x_bf16, false, T_blocks, n_tok, d_in, 16, WUSH_NVFP4, codes, scale_atoms, tensor_scale, nullptr,
+                      false, stream, false, true);
+}
+
+int wush_quant_weight_nv_atoms(const float* w_f32, const float* T_blocks, int64_t d_out, int64_t d_in, uint8_t* codes,
+                               uint8_t* scale_atoms, float* tensor_scale, wush_stream_t stream) {
+  return quant_common(w_f32, true, T_blocks, d_out, d_in, 16, WUSH_NVFP4, codes, scale_atoms, tensor_scale, nullptr,
+                      false, stream, false, true);
 }
 
 int wush_build_transforms(const float* w_f32, const void* xcal_bf16, int64_t d_out, int64_t n_cal, int64_t d_in,

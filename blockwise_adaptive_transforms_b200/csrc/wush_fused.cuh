@@ -631,25 +631,30 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
       }
       if (Cfg::AMAX_ONLY) continue;
       // scales: this thread's row of the tile, straight from registers
-      if (Cfg::FMT == kMXFP4 && p.scale_atoms) {
+      if (Cfg::FMT != kINT4 && p.scale_atoms) {
         // scale-atom layout: row 128 r + i + 32 j, scale column 4 c + k at byte
-        // (r * atom_cols + c) * 512 + 16 i + 4 j + k; this tile's BPT columns are
-        // consecutive k of one atom word
+        // (r * atom_cols + c) * 512 + 16 i + 4 j + k; each aligned group of four of this
+        // tile's columns is one 32-bit word of an atom
         if (warp_live && row_ok) {
           const int col0 = ct * BPT;
           const int rr = static_cast<int>(grow & 127);
-          uint8_t* word = static_cast<uint8_t*>(p.scales) +
-                          ((grow >> 7) * p.atom_cols + (col0 >> 2)) * 512 + (rr & 31) * 16 + (rr >> 5) * 4;
+          uint8_t* row_base = static_cast<uint8_t*>(p.scales) + (grow >> 7) * p.atom_cols * 512 + (rr & 31) * 16 +
+                              (rr >> 5) * 4;
           const int nb = min(BPT, C - col0);
-          if constexpr (BPT == 4) {
-            if (nb == 4) {
-              *reinterpret_cast<uint32_t*>(word) = static_cast<uint32_t>(sc[0]) | (static_cast<uint32_t>(sc[1]) << 8) |
-                                                   (static_cast<uint32_t>(sc[2]) << 16) | (static_cast<uint32_t>(sc[3]) << 24);
-            } else {
-              for (int k = 0; k < nb; ++k) word[k] = static_cast<uint8_t>(sc[k]);
+          if constexpr (BPT % 4 == 0) {
+#pragma unroll
+            for (int w4 = 0; w4 < BPT / 4; ++w4) {
+              uint8_t* word = row_base + ((col0 >> 2) + w4) * 512;
+              if (4 * w4 + 4 <= nb) {
+                *reinterpret_cast<uint32_t*>(word) =
+                    static_cast<uint32_t>(sc[4 * w4]) | (static_cast<uint32_t>(sc[4 * w4 + 1]) << 8) |
+                    (static_cast<uint32_t>(sc[4 * w4 + 2]) << 16) | (static_cast<uint32_t>(sc[4 * w4 + 3]) << 24);
+              } else {
+                for (int k = 4 * w4; k < nb; ++k) word[k - 4 * w4] = static_cast<uint8_t>(sc[k]);
+              }
             }
           } else {
-            for (int k = 0; k < nb; ++k) word[(col0 & 3) + k] = static_cast<uint8_t>(sc[k]);
+            for (int k = 0; k < nb; ++k) row_base[((col0 + k) >> 2) * 512 + ((col0 + k) & 3)] = static_cast<uint8_t>(sc[k]);
           }
         }
       } else if (warp_live && row_ok) {

@@ -1,23 +1,26 @@
-// MXFP4 x MXFP4 -> bf16 GEMM for sm_100a on block-scaled tcgen05 MMAs: the consumer of the
+// Block-scaled FP4 x FP4 -> bf16 GEMM for sm_100a on tcgen05 MMAs: the consumer of the
 // quantised operands (the pages' "WUSH + Quant + FP4 MatMul" layer: paper-graph-ui
 // analysis, section 3.4.7 "GPU Kernel Design" and section 5 "GPU Kernel Benchmarks
 // (Figure 2)").
 //
-//   D[m][n] = sum_k A[m][k] * B[n][k]
+//   D[m][n] = alpha * sum_k A[m][k] * B[n][k]
 //
 // A (activations, M rows) and B (weights, N rows = output channels) are E2M1 codes packed
-// two per byte along K (low nibble = even k), each 32-element group with an E8M0 scale.
-// The scales are read in the layout the block-scaled MMA consumes ("tcgen05 scale
-// atoms"): for rows [128 r, 128 r + 128) and scale columns [4 c, 4 c + 4) one 512-byte
-// atom at byte (r * (K / 128) + c) * 512, in which row 128 r + i + 32 j, scale 4 c + k
-// sits at byte 16 i + 4 j + k (i < 32, j < 4, k < 4).
+// two per byte along K (low nibble = even k).  MXFP4: each 32-element group has an E8M0
+// scale and alpha = 1.  NVFP4: each 16-element group has an E4M3 scale and alpha is the
+// product of the two fp32 tensor scales.  The scales are read in the layout the
+// block-scaled MMA consumes ("tcgen05 scale atoms"): for rows [128 r, 128 r + 128) and
+// scale columns [4 c, 4 c + 4) one 512-byte atom at byte (r * (C / 4) + c) * 512, in which
+// row 128 r + i + 32 j, scale 4 c + k sits at byte 16 i + 4 j + k (i < 32, j < 4, k < 4).
 //
 // Tiles of 128 x 256 outputs, 256 K-elements (128 bytes of codes per row) per pipeline
 // stage; per stage the producer brings A (16 KB) and B (32 KB) by TMA with 128-byte
-// swizzle and the three scale atoms' 1 KB pieces by bulk copies; the MMA thread moves the
-// scale atoms into TMEM (tcgen05.cp 32x128b, broadcast to the four lane quadrants) and
-// issues four M=128, N=256, K=64 MMAs (kind::mxf4, block32); four epilogue warps read the
-// fp32 accumulator (tcgen05.ld), round to bf16 and store.  Persistent CTAs, one per SM.
+// swizzle and the stage's scale atoms (A: 2 (MX) or 4 (NV); B: twice that, for its two
+// 128-row halves) by bulk copies; the MMA thread moves the atoms into TMEM (tcgen05.cp
+// 32x128b, broadcast to the four lane quadrants) and issues four M=128, N=256, K=64 MMAs
+// (kind::mxf4 block32, or kind::mxf4nvf4 block16); four epilogue warps read the fp32
+// accumulator (tcgen05.ld), scale by alpha, round to bf16 and store.  Persistent CTAs,
+// one per SM.
 #pragma once
 #include <cstdint>
 #include <cuda_bf16.h>
@@ -28,19 +31,29 @@ namespace wush {
 struct GemmParams {
   const uint8_t* sfa;        // A scale atoms
   const uint8_t* sfb;        // B scale atoms
+  const float* ts_a;         // NVFP4: A's fp32 tensor scale (device)
+  const float* ts_b;         // NVFP4: B's fp32 tensor scale (device)
   __nv_bfloat16* d;          // [M][N]
   int M, N, K;
   int tiles_m, tiles_n;
   unsigned long long wait_limit_ns;
 };
 
+// NV = false: MXFP4 (E8M0 scales per 32 elements, kind::mxf4 block32);
+// NV = true:  NVFP4 (E4M3 scales per 16 elements, kind::mxf4nvf4 block16, times the two
+//             fp32 tensor scales in the epilogue).
+template <bool NV_>
 struct GemmCfg {
+  static constexpr bool NV = NV_;
+  static constexpr int VS = NV ? 16 : 32;              // elements per scale
   static constexpr int BM = 128, BN = 256, BK = 256;   // BK in elements (128 bytes of codes)
   static constexpr int STAGES = 4;
+  static constexpr int ATOM_K = 4 * VS;                // K elements one scale atom covers
+  static constexpr int ATOMS_PER_STAGE = BK / ATOM_K;  // MX 2, NV 4
   static constexpr int A_BYTES = BM * BK / 2;          // 16 KB
   static constexpr int B_BYTES = BN * BK / 2;          // 32 KB
-  static constexpr int SFA_BYTES = BM * BK / 32;       // 1 KB: two atoms
-  static constexpr int SFB_BYTES = BN * BK / 32;       // 2 KB: two atoms per 128-row half
+  static constexpr int SFA_BYTES = ATOMS_PER_STAGE * 512;          // one atom per K chunk
+  static constexpr int SFB_BYTES = 2 * ATOMS_PER_STAGE * 512;      // and per 128-row half
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
   static constexpr int OFF_A = 0, OFF_B = A_BYTES, OFF_SFA = A_BYTES + B_BYTES, OFF_SFB = OFF_SFA + SFA_BYTES;
   static constexpr int OFF_BAR = STAGES * STAGE_BYTES;
@@ -48,23 +61,26 @@ struct GemmCfg {
   static constexpr int OFF_MISC = OFF_BAR + 8 * N_BARS;
   static constexpr int SMEM_BYTES = OFF_MISC + 64 + 1024;
   static constexpr int THREADS = 8 * 32;               // producer, MMA, 2 idle, 4 epilogue warps
-  // TMEM: accumulator columns [0, 256); per stage slot 24 scale columns from 256
+  // TMEM: accumulator columns [0, 256); per stage slot the scale columns from 256: A atom
+  // a at +4a, B atom a of half h at +4 * ATOMS_PER_STAGE + 8a + 4h
   static constexpr int TMEM_COLS = 512;
-  static constexpr int SF_COL0 = 256, SF_SLOT_COLS = 24;
+  static constexpr int SF_COL0 = 256, SFB_COL = 4 * ATOMS_PER_STAGE, SF_SLOT_COLS = 12 * ATOMS_PER_STAGE;
   static_assert(STAGE_BYTES % 1024 == 0, "stage alignment");
   static_assert(SF_COL0 + STAGES * SF_SLOT_COLS <= TMEM_COLS, "TMEM columns");
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
-// Instruction descriptor of kind::mxf4 block-scaled MMAs: E2M1 A and B (format 1),
-// K-major, E8M0 scales (bit 23), M = 128, N = 256, dense K = 64; the scale-factor ids
-// (bits 29-30 for A, 4-5 for B) select the byte of the TMEM word the first scale sits in.
-__device__ __forceinline__ uint32_t idesc_mxf4(int M, int N, uint32_t sf_id) {
+// Instruction descriptor of the block-scaled FP4 MMAs (kind::mxf4 / kind::mxf4nvf4):
+// E2M1 A and B (format 1), K-major, scale type in bit 23 (1 = E8M0, 0 = UE4M3),
+// M = 128, N = 256, dense K = 64; the scale-factor ids (bits 29-30 for A, 4-5 for B)
+// select the byte of the TMEM word the first scale sits in (always 0 for block16, whose
+// four scales fill the word).
+__device__ __forceinline__ uint32_t idesc_mxf4(int M, int N, uint32_t sf_id, bool e8m0) {
   return (sf_id << 4)                               // B scale-factor id
          | (1u << 7)                                // A format: E2M1
          | (1u << 10)                               // B format: E2M1
          | (static_cast<uint32_t>(N >> 3) << 17)    // N / 8
-         | (1u << 23)                               // scale format: E8M0
+         | ((e8m0 ? 1u : 0u) << 23)                 // scale format: E8M0 or UE4M3
          | (static_cast<uint32_t>(M >> 4) << 24)    // M / 16
          | (sf_id << 29);                           // A scale-factor id
 }
@@ -75,6 +91,15 @@ __device__ __forceinline__ void umma_mxf4(uint32_t d_tmem, uint64_t a_desc, uint
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+__device__ __forceinline__ void umma_nvf4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
       : "memory");
 }
@@ -95,10 +120,10 @@ __device__ __forceinline__ void tmem_cp_32x128b_x4(uint32_t taddr, uint64_t sdes
   asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
 }
 
-__global__ void __launch_bounds__(GemmCfg::THREADS, 1)
-    wush_gemm_mxf4_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
-                          const GemmParams p) {
-  using Cfg = GemmCfg;
+template <class Cfg>
+__global__ void __launch_bounds__(Cfg::THREADS, 1)
+    wush_gemm_fp4_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
+                         const GemmParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_addr(smem);
@@ -112,7 +137,7 @@ __global__ void __launch_bounds__(GemmCfg::THREADS, 1)
   const uint64_t lim = p.wait_limit_ns;
   const int n_tiles = p.tiles_m * p.tiles_n;
   const int k_stages = p.K / Cfg::BK;
-  const int k_chunks = p.K / 128;                       // scale atoms along K per 128-row block
+  const int k_chunks = p.K / Cfg::ATOM_K;               // scale atoms along K per 128-row block
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -153,11 +178,13 @@ __global__ void __launch_bounds__(GemmCfg::THREADS, 1)
           mbar_arrive_expect_tx(fb, Cfg::STAGE_BYTES);
           tma_load_2d(dst + Cfg::OFF_A, &tmap_a, fb, ks * 128, tm * Cfg::BM, 0ull);
           tma_load_2d(dst + Cfg::OFF_B, &tmap_b, fb, ks * 128, tn * Cfg::BN, pol);
-          // scale atoms: K chunks 2 ks and 2 ks + 1 of the tile's row blocks (1 KB each)
-          bulk_load_1d(dst + Cfg::OFF_SFA, p.sfa + (static_cast<long long>(tm) * k_chunks + 2 * ks) * 512, 1024u, fb);
+          // scale atoms of this stage's K chunks, for the tile's A row block and B's two halves
+          constexpr uint32_t APS = Cfg::ATOMS_PER_STAGE;
+          bulk_load_1d(dst + Cfg::OFF_SFA, p.sfa + (static_cast<long long>(tm) * k_chunks + APS * ks) * 512,
+                       APS * 512u, fb);
           for (int h = 0; h < 2; ++h)
-            bulk_load_1d(dst + Cfg::OFF_SFB + h * 1024,
-                         p.sfb + (static_cast<long long>(2 * tn + h) * k_chunks + 2 * ks) * 512, 1024u, fb);
+            bulk_load_1d(dst + Cfg::OFF_SFB + h * APS * 512,
+                         p.sfb + (static_cast<long long>(2 * tn + h) * k_chunks + APS * ks) * 512, APS * 512u, fb);
           ++n_issued;
           if (++stage == STAGES) stage = 0, phase ^= 1u;
         }
@@ -182,24 +209,29 @@ __global__ void __launch_bounds__(GemmCfg::THREADS, 1)
           tc_fence_after();
           const uint32_t st = sbase + stage * Cfg::STAGE_BYTES;
           const uint32_t sf_cols = tmem_base + static_cast<uint32_t>(Cfg::SF_COL0 + stage * Cfg::SF_SLOT_COLS);
-          // scale atoms -> TMEM: A chunk c at columns +4c, B chunk c, half h at +8 + 8c + 4h
+          // scale atoms -> TMEM: A atom a at columns +4a, B atom a of half h at +SFB_COL + 8a + 4h
 #pragma unroll
-          for (int c = 0; c < 2; ++c) {
-            tmem_cp_32x128b_x4(sf_cols + 4 * c, desc_sf_atom(st + Cfg::OFF_SFA + c * 512));
+          for (int a = 0; a < Cfg::ATOMS_PER_STAGE; ++a) {
+            tmem_cp_32x128b_x4(sf_cols + 4 * a, desc_sf_atom(st + Cfg::OFF_SFA + a * 512));
 #pragma unroll
             for (int h = 0; h < 2; ++h)
-              tmem_cp_32x128b_x4(sf_cols + 8 + 8 * c + 4 * h, desc_sf_atom(st + Cfg::OFF_SFB + h * 1024 + c * 512));
+              tmem_cp_32x128b_x4(sf_cols + Cfg::SFB_COL + 8 * a + 4 * h,
+                                 desc_sf_atom(st + Cfg::OFF_SFB + h * Cfg::ATOMS_PER_STAGE * 512 + a * 512));
           }
           const uint64_t da = desc_k_sw128(st + Cfg::OFF_A);
           const uint64_t db = desc_k_sw128(st + Cfg::OFF_B);
 #pragma unroll
           for (int j = 0; j < 4; ++j) {        // K = 64 each: 32 bytes along the 128-byte rows
-            const int c = j >> 1;
-            const uint32_t sub = static_cast<uint32_t>(2 * (j & 1));   // scale byte 0 or 2 of the word
-            const uint32_t sfa = (sf_cols + 4 * c) | (sub << 30);
-            const uint32_t sfb = (sf_cols + 8 + 8 * c) | (sub << 30);
-            umma_mxf4(tmem_base, da + ((j * 32) >> 4), db + ((j * 32) >> 4), idesc_mxf4(128, 256, sub), sfa, sfb,
-                      (ks > 0 || j > 0) ? 1u : 0u);
+            // MXFP4: two MMAs per atom word, scales at byte 0 or 2; NVFP4: one word per MMA
+            const int a = Cfg::NV ? j : (j >> 1);
+            const uint32_t sub = Cfg::NV ? 0u : static_cast<uint32_t>(2 * (j & 1));
+            const uint32_t sfa = (sf_cols + 4 * a) | (sub << 30);
+            const uint32_t sfb = (sf_cols + Cfg::SFB_COL + 8 * a) | (sub << 30);
+            const uint32_t idesc = idesc_mxf4(128, 256, sub, !Cfg::NV);
+            if constexpr (Cfg::NV)
+              umma_nvf4(tmem_base, da + ((j * 32) >> 4), db + ((j * 32) >> 4), idesc, sfa, sfb, (ks > 0 || j > 0) ? 1u : 0u);
+            else
+              umma_mxf4(tmem_base, da + ((j * 32) >> 4), db + ((j * 32) >> 4), idesc, sfa, sfb, (ks > 0 || j > 0) ? 1u : 0u);
           }
           umma_commit(BAR(B_EMPTY + stage));
           if (++stage == STAGES) stage = 0, phase ^= 1u;
@@ -215,6 +247,7 @@ __global__ void __launch_bounds__(GemmCfg::THREADS, 1)
     // ------------------------------------------------------------ epilogue (4 warps)
     const int quad = warp & 3;
     const int row_in_tile = quad * 32 + lane;
+    const float alpha = Cfg::NV ? __fmul_rn(*p.ts_a, *p.ts_b) : 1.0f;
     int it = 0;
     bool live = true;
     for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++it) {
@@ -232,7 +265,8 @@ __global__ void __launch_bounds__(GemmCfg::THREADS, 1)
         uint32_t packed[16];
 #pragma unroll
         for (int k = 0; k < 16; ++k) {
-          const __nv_bfloat162 b2 = __floats2bfloat162_rn(v[2 * k], v[2 * k + 1]);
+          const __nv_bfloat162 b2 = Cfg::NV ? __floats2bfloat162_rn(v[2 * k] * alpha, v[2 * k + 1] * alpha)
+                                            : __floats2bfloat162_rn(v[2 * k], v[2 * k + 1]);
           packed[k] = *reinterpret_cast<const uint32_t*>(&b2);
         }
         uint4* dst = reinterpret_cast<uint4*>(drow + 32 * ch);
@@ -253,8 +287,8 @@ __global__ void __launch_bounds__(GemmCfg::THREADS, 1)
   }
 }
 
-// Row-major E8M0 scales [rows][C] (C = K / 32) -> tcgen05 scale atoms (rows padded to a
-// multiple of 128 with zero bytes, C to a multiple of 4).
+// Row-major one-byte scales [rows][C] -> tcgen05 scale atoms (rows padded to a multiple
+// of 128 with zero bytes, C to a multiple of 4).
 __global__ void wush_scales_to_atoms_kernel(const uint8_t* __restrict__ src, long long rows, int C,
                                             uint8_t* __restrict__ dst, long long rows_pad, int C_pad) {
   const long long n = rows_pad * C_pad;

@@ -7,7 +7,9 @@ for a square, a wide and a deep projection of each model) on one B200:
   bf16   X W^T in bf16 (cuBLAS through torch.matmul),
   none   the MXFP4 GEMM alone, operands already quantised (the upper bound),
   H      shared-Hadamard transform + quantisation of X, then the MXFP4 GEMM,
-  WUSH   per-block WUSH transform + quantisation of X, then the MXFP4 GEMM.
+  WUSH   per-block WUSH transform + quantisation of X, then the MXFP4 GEMM;
+  nv_none / nv_WUSH   the same two for NVFP4 (G = 16 transforms, two-pass tensor scale,
+         the NVFP4 GEMM).
 
 Weights are quantised once beforehand (offline, as on the pages).  Every variant is
 timed as a CUDA graph of repeated calls with events on its stream.
@@ -23,8 +25,8 @@ import sys
 
 import torch
 
-from . import (hadamard_matrix, wush_gemm_mxfp4, wush_quant_act_mx_atoms, wush_quant_act_shared_mx_atoms,
-               wush_quant_weight_mx_atoms)
+from . import (hadamard_matrix, wush_gemm_mxfp4, wush_gemm_nvfp4, wush_quant_act_mx_atoms, wush_quant_act_nv_atoms,
+               wush_quant_act_shared_mx_atoms, wush_quant_weight_mx_atoms, wush_quant_weight_nv_atoms)
 
 # (N, K) per projection kind.  The Qwen3-8B shapes are the pages' own; the other two rows
 # are the same three kinds for a 14B-class (hidden 5120, MLP 17408) and a 70B-class
@@ -71,6 +73,9 @@ def bench_shape(M: int, N: int, K: int, device="cuda", seed=0) -> dict:
     w_bf16 = w.to(torch.bfloat16)
     cw, aw = wush_quant_weight_mx_atoms(w, T)             # offline
     cx, ax = wush_quant_act_mx_atoms(x, T)
+    Tn = (torch.eye(16) + 0.1 * torch.randn(K // 16, 16, 16, generator=gen)).to(device)
+    cwn, awn, twn = wush_quant_weight_nv_atoms(w, Tn)     # offline
+    cxn, axn, txn = wush_quant_act_nv_atoms(x, Tn)
     out = torch.empty((M, N), dtype=torch.bfloat16, device=device)
     out_ref = torch.empty((M, N), dtype=torch.bfloat16, device=device)
     s = torch.cuda.Stream(device=device)
@@ -89,10 +94,18 @@ def bench_shape(M: int, N: int, K: int, device="cuda", seed=0) -> dict:
         wush_quant_act_mx_atoms(x, T, codes=cx, atoms=ax, stream=s)
         wush_gemm_mxfp4(cx, ax, cw, aw, out=out, stream=s)
 
-    t = {name: _time_graph(fn, s) for name, fn in (("bf16", bf16), ("none", none), ("H", h_quant), ("WUSH", wush))}
+    def nv_none():
+        wush_gemm_nvfp4(cxn, axn, txn, cwn, awn, twn, out=out, stream=s)
+
+    def nv_wush():
+        wush_quant_act_nv_atoms(x, Tn, codes=cxn, atoms=axn, tensor_scale=txn, stream=s)
+        wush_gemm_nvfp4(cxn, axn, txn, cwn, awn, twn, out=out, stream=s)
+
+    t = {name: _time_graph(fn, s) for name, fn in (("bf16", bf16), ("none", none), ("H", h_quant), ("WUSH", wush),
+                                                   ("nv_none", nv_none), ("nv_WUSH", nv_wush))}
     flops = 2.0 * M * N * K
     return {"M": M, "N": N, "K": K, "us": {k: round(v, 2) for k, v in t.items()},
-            "speedup_vs_bf16": {k: round(t["bf16"] / t[k], 3) for k in ("none", "H", "WUSH")},
+            "speedup_vs_bf16": {k: round(t["bf16"] / t[k], 3) for k in ("none", "H", "WUSH", "nv_none", "nv_WUSH")},
             "fp4_gemm_tflops": round(flops / t["none"] / 1e6, 1), "bf16_tflops": round(flops / t["bf16"] / 1e6, 1)}
 
 
@@ -111,7 +124,8 @@ def main(argv=None) -> int:
             print(f"{key:10s} M={a.M} N={N:6d} K={K:6d}  bf16 {r['us']['bf16']:8.1f} us  fp4 gemm {r['us']['none']:8.1f} us"
                   f" ({r['fp4_gemm_tflops']:7.1f} TFLOP/s)  H {r['us']['H']:8.1f}  WUSH {r['us']['WUSH']:8.1f}   "
                   f"speedup none/H/WUSH {r['speedup_vs_bf16']['none']:.2f}/{r['speedup_vs_bf16']['H']:.2f}/"
-                  f"{r['speedup_vs_bf16']['WUSH']:.2f}", flush=True)
+                  f"{r['speedup_vs_bf16']['WUSH']:.2f}   nvfp4 none/WUSH {r['us']['nv_none']:8.1f}/{r['us']['nv_WUSH']:8.1f} us",
+                  flush=True)
     if a.json:
         with open(a.json, "w") as f:
             json.dump(rows, f, indent=1)

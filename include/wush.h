@@ -147,6 +147,19 @@ int wush_gemm_mxfp4(const uint8_t* a_codes, const uint8_t* a_atoms, const uint8_
                     const uint8_t* b_atoms, int64_t M, int64_t N, int64_t K, void* d_bf16,
                     wush_stream_t stream);
 
+/* The same GEMM for NVFP4 operands: E2M1 codes with one E4M3 scale per 16 elements
+ * (kind::mxf4nvf4 block16 MMAs) and one fp32 tensor scale per operand:
+ *   D[m][n] = s_A s_B sum_k (e2m1 e4m3)_A[m][k] (e2m1 e4m3)_B[n][k]
+ * (fp32 accumulation, the sum times fl32(s_A s_B) in fp32, one bf16 rounding).
+ * a_atoms / b_atoms: the E4M3 scale bytes [rows][K/16] in the scale-atom layout (see
+ * wush_mx_scales_to_atoms, which relays out any one-byte scales, or the *_nv_atoms
+ * quantisers); a_tensor_scale / b_tensor_scale: device fp32 (the quantisers' s_t).
+ * Same shapes, alignment and errors as wush_gemm_mxfp4 (NULL tensor scales:
+ * WUSH_ERR_INVALID_ARG; not 4-byte aligned: WUSH_ERR_MISALIGNED). */
+int wush_gemm_nvfp4(const uint8_t* a_codes, const uint8_t* a_atoms, const float* a_tensor_scale,
+                    const uint8_t* b_codes, const uint8_t* b_atoms, const float* b_tensor_scale,
+                    int64_t M, int64_t N, int64_t K, void* d_bf16, wush_stream_t stream);
+
 /* MXFP4 (G = 32) quantisation that writes its E8M0 scales straight into the scale-atom
  * layout wush_gemm_mxfp4 reads (instead of row-major [rows][C]): the same kernels,
  * codes and errors as wush_quant_act / wush_quant_weight / wush_quant_act_shared with
@@ -162,7 +175,20 @@ int wush_quant_act_shared_mx_atoms(const void* x_bf16, const float* T_shared, in
                                    int64_t d_in, uint8_t* codes, uint8_t* scale_atoms,
                                    wush_stream_t stream);
 
-/* Row-major E8M0 scales [rows][C] -> the scale-atom layout the block-scaled MMA reads:
+/* NVFP4 (G = 16) quantisation that writes its E4M3 scales in the scale-atom layout
+ * wush_gemm_nvfp4 reads: the same kernels, codes, tensor scale and errors as
+ * wush_quant_act / wush_quant_weight with fmt = NVFP4.  scale_atoms (device, 16-byte
+ * aligned) must hold atom_bytes = rows_pad * C_pad bytes (C = d_in / 16); bytes of
+ * padding rows and columns are not written.  tensor_scale: device fp32, written. */
+int wush_quant_act_nv_atoms(const void* x_bf16, const float* T_blocks, int64_t n_tok, int64_t d_in,
+                            uint8_t* codes, uint8_t* scale_atoms, float* tensor_scale,
+                            wush_stream_t stream);
+int wush_quant_weight_nv_atoms(const float* w_f32, const float* T_blocks, int64_t d_out,
+                               int64_t d_in, uint8_t* codes, uint8_t* scale_atoms,
+                               float* tensor_scale, wush_stream_t stream);
+
+/* Row-major one-byte scales [rows][C] (E8M0 or E4M3) -> the scale-atom layout the
+ * block-scaled MMA reads:
  * rows padded to a multiple of 128 and C to a multiple of 4 (zero bytes); the atom of
  * row block r and scale columns [4c, 4c + 4) is the 512 bytes at (r * (C_pad/4) + c) * 512,
  * holding row 128 r + i + 32 j, column 4 c + k at byte 16 i + 4 j + k (i < 32, j < 4,

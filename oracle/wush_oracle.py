@@ -576,8 +576,8 @@ def layer_loss_prequantised(wq: np.ndarray, w: np.ndarray, x_bits: np.ndarray, T
 
 
 def scale_atoms(scales: np.ndarray) -> np.ndarray:
-    """E8M0 scales [rows][C] in the block-scaled MMA's scale-atom layout (a hardware
-    format, not from the pages): rows padded to a multiple of 128 and C to a multiple
+    """One-byte scales [rows][C] (E8M0 or E4M3) in the block-scaled MMA's scale-atom
+    layout (a hardware format, not from the pages): rows padded to a multiple of 128 and C to a multiple
     of 4 with zero bytes; row 128 r + i + 32 j, column 4 c + k goes to byte
     (r * C_pad / 4 + c) * 512 + 16 i + 4 j + k."""
     s = np.asarray(scales, dtype=np.uint8)
@@ -597,6 +597,15 @@ def gemm_mx(a_codes: np.ndarray, a_scales: np.ndarray, b_codes: np.ndarray, b_sc
     B packed codes [N][K/2] with scales [N][K/32] (one row per output channel)."""
     A = dequant(unpack_nibbles(a_codes), a_scales, "mxfp4", 32)
     B = dequant(unpack_nibbles(b_codes), b_scales, "mxfp4", 32)
+    return A @ B.T
+
+
+def gemm_nv(a_codes: np.ndarray, a_scales: np.ndarray, a_ts: float, b_codes: np.ndarray, b_scales: np.ndarray,
+            b_ts: float) -> np.ndarray:
+    """The same product for NVFP4 operands (E4M3 scales per 16 elements [rows][K/16] and
+    an fp32 tensor scale each): D = deq(A) deq(B)^T in float64."""
+    A = dequant(unpack_nibbles(a_codes), a_scales, "nvfp4", 16, a_ts)
+    B = dequant(unpack_nibbles(b_codes), b_scales, "nvfp4", 16, b_ts)
     return A @ B.T
 
 

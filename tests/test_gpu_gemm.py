@@ -1,9 +1,10 @@
-"""MXFP4 GEMM consumer and the scale-atom relayout vs the fp64 oracle (needs a B200).
+"""MXFP4 / NVFP4 GEMM consumers and the scale-atom relayout vs the fp64 oracle (needs a B200).
 
 D = deq(A) deq(B)^T (paper-graph-ui analysis, section 3.4.7 "GPU Kernel Design": the
 FP4 MatMul that follows WUSH + Quant).  The kernel accumulates in fp32 and rounds D once
 to bf16, so each element must lie within 2^-8 |D| (bf16 rounding) plus the fp32
-accumulation bound K 2^-23 (|A| |B|^T) of the oracle's value.
+accumulation bound K 2^-23 (|A| |B|^T) of the oracle's value (NVFP4: K + 2, for the
+product of the tensor scales and the product with it).
 """
 import numpy as np
 import pytest
@@ -103,3 +104,91 @@ def test_quantiser_writes_scale_atoms_directly(n_tok, d_in):
     assert np.array_equal(at.cpu().numpy(), O.scale_atoms(s.cpu().numpy()))
     assert np.array_equal(atw.cpu().numpy(), O.scale_atoms(sw.cpu().numpy()))
     assert np.array_equal(ath.cpu().numpy(), O.scale_atoms(sh.cpu().numpy()))
+
+
+def random_nv_operand(rows, K, seed):
+    """Random E2M1 codes and E4M3 scales over the normal and subnormal range (0x01..0x7E,
+    never the NaN code)."""
+    rng = np.random.default_rng(seed)
+    codes = rng.integers(0, 256, (rows, K // 2), dtype=np.uint8)
+    scales = rng.integers(0x01, 0x7F, (rows, K // 16), dtype=np.uint8)
+    return codes, scales
+
+
+def assert_gemm_nv_close(d_gpu, a_c, a_s, a_t, b_c, b_s, b_t, K):
+    ref = O.gemm_nv(a_c, a_s, a_t, b_c, b_s, b_t)
+    A = np.abs(O.dequant(O.unpack_nibbles(a_c), a_s, "nvfp4", 16, a_t))
+    B = np.abs(O.dequant(O.unpack_nibbles(b_c), b_s, "nvfp4", 16, b_t))
+    bound = 2.0 ** -8 * np.abs(ref) + (K + 2) * 2.0 ** -23 * (A @ B.T) + 1e-30
+    err = np.abs(d_gpu.astype(np.float64) - ref)
+    worst = np.unravel_index(np.argmax(err / bound), err.shape)
+    assert np.all(err <= bound), f"at {worst}: gpu {d_gpu[worst]} oracle {ref[worst]} bound {bound[worst]}"
+
+
+@pytest.mark.parametrize("M,N,K", [(128, 256, 256), (256, 512, 1024), (384, 768, 768), (128, 256, 4096)])
+def test_gemm_nvfp4_random_operands(M, N, K):
+    a_c, a_s = random_nv_operand(M, K, 3)
+    b_c, b_s = random_nv_operand(N, K, 4)
+    a_t, b_t = float(np.float32(0.37)), float(np.float32(1.9))
+    ta = torch.tensor([a_t], dtype=torch.float32, device="cuda")
+    tb = torch.tensor([b_t], dtype=torch.float32, device="cuda")
+    d = W.wush_gemm_nvfp4(dev(a_c), W.wush_mx_scales_to_atoms(dev(a_s)), ta, dev(b_c),
+                          W.wush_mx_scales_to_atoms(dev(b_s)), tb)
+    torch.cuda.synchronize()
+    st, bits = W.wush_device_status()
+    assert st == 0 and bits == 0, f"device error word {bits:#x}"
+    assert_gemm_nv_close(d.float().cpu().numpy(), a_c, a_s, a_t, b_c, b_s, b_t, K)
+
+
+def test_gemm_nvfp4_rejects_missing_tensor_scale_and_bad_shapes():
+    a = torch.zeros((128, 128), dtype=torch.uint8, device="cuda")
+    b = torch.zeros((256, 128), dtype=torch.uint8, device="cuda")
+    ts = torch.ones(1, dtype=torch.float32, device="cuda")
+    lib = W.load_library()
+    at = torch.zeros(W.atom_bytes(256, 16), dtype=torch.uint8, device="cuda")
+    d = torch.empty((128, 256), dtype=torch.bfloat16, device="cuda")
+    st = lib.wush_gemm_nvfp4(a.data_ptr(), at.data_ptr(), None, b.data_ptr(), at.data_ptr(), ts.data_ptr(),
+                             128, 256, 256, d.data_ptr(), None)
+    assert st == 1
+    a_bad = torch.zeros((100, 128), dtype=torch.uint8, device="cuda")
+    with pytest.raises(W.WushError):
+        W.wush_gemm_nvfp4(a_bad, at, ts, b, at, ts)
+
+
+@pytest.mark.parametrize("n_tok,d_in", [(256, 1024), (300, 416), (129, 4096 + 64)])
+def test_nvfp4_quantiser_writes_scale_atoms_directly(n_tok, d_in):
+    wl = workload("attn_mxfp4_4096", n_tok=n_tok, d_in=d_in, d_out=256, n_cal=512)
+    inp = make_inputs(wl)
+    b = O.build_transforms(inp.w, inp.xcal_bits, 16)
+    x = dev(inp.x_bits.view(np.int16)).view(torch.bfloat16)
+    T = dev(b["T_wush32"])
+    c, s, ts = W.wush_quant_act(x, T, 16, "nvfp4")
+    ca, at, tsa = W.wush_quant_act_nv_atoms(x, T)
+    cw, sw, tw = W.wush_quant_weight(dev(inp.w), dev(b["T_xvsh32"]), 16, "nvfp4")
+    cwa, atw, twa = W.wush_quant_weight_nv_atoms(dev(inp.w), dev(b["T_xvsh32"]))
+    torch.cuda.synchronize()
+    assert torch.equal(c, ca) and torch.equal(cw, cwa)
+    assert torch.equal(ts, tsa) and torch.equal(tw, twa)
+    assert np.array_equal(at.cpu().numpy(), O.scale_atoms(s.cpu().numpy()))
+    assert np.array_equal(atw.cpu().numpy(), O.scale_atoms(sw.cpu().numpy()))
+
+
+def test_nvfp4_layer_after_wush_quantisation():
+    """The NVFP4 layer end to end: both operands quantised by the library with the G = 16
+    WUSH transforms straight into scale atoms, then the NVFP4 GEMM; the oracle multiplies
+    the kernels' own codes, scales and tensor scales."""
+    wl = workload("attn_mxfp4_4096", n_tok=256, d_in=1024, d_out=512, n_cal=1024)
+    inp = make_inputs(wl)
+    b = O.build_transforms(inp.w, inp.xcal_bits, 16)
+    x = dev(inp.x_bits.view(np.int16)).view(torch.bfloat16)
+    cx, sx, tx = W.wush_quant_act(x, dev(b["T_wush32"]), 16, "nvfp4")
+    cw, sw, tw = W.wush_quant_weight(dev(inp.w), dev(b["T_xvsh32"]), 16, "nvfp4")
+    _, ax, _ = W.wush_quant_act_nv_atoms(x, dev(b["T_wush32"]))
+    _, aw, _ = W.wush_quant_weight_nv_atoms(dev(inp.w), dev(b["T_xvsh32"]))
+    d = W.wush_gemm_nvfp4(cx, ax, tx, cw, aw, tw)
+    torch.cuda.synchronize()
+    assert_gemm_nv_close(d.float().cpu().numpy(), cx.cpu().numpy(), sx.cpu().numpy(), float(tx.item()),
+                         cw.cpu().numpy(), sw.cpu().numpy(), float(tw.item()), wl.d_in)
+    ref = O.bf16_to_f64(inp.x_bits) @ inp.w.astype(np.float64).T
+    rel = np.linalg.norm(d.float().cpu().numpy() - ref) / np.linalg.norm(ref)
+    assert rel < 0.25, rel

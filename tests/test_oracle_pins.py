@@ -296,6 +296,21 @@ def test_gemm_mx_exact_small_cases():
     assert np.array_equal(d, np.full((M, N), K * 1.5 * -2.0))
 
 
+def test_gemm_nv_exact_small_cases():
+    """E2M1 1.0 everywhere.  A's E4M3 scales 2.0 (0x40) at tensor scale 0.25, B's 0.5
+    (0x30) at 3.0: every product is 0.5 * 1.5, so each output is 0.75 K.  Then A's groups
+    alternate 1.0 (0x38) and the smallest subnormal 2^-9 (0x01) with everything else 1:
+    each 16-wide group contributes 16 times its scale."""
+    M, N, K = 2, 3, 64
+    a = O.pack_nibbles(np.full((M, K), 2, np.uint8))
+    b = O.pack_nibbles(np.full((N, K), 2, np.uint8))
+    d = O.gemm_nv(a, np.full((M, K // 16), 0x40, np.uint8), 0.25, b, np.full((N, K // 16), 0x30, np.uint8), 3.0)
+    assert np.array_equal(d, np.full((M, N), 0.75 * K))
+    sa = np.tile(np.array([0x38, 0x01], np.uint8), (M, K // 32))
+    d = O.gemm_nv(a, sa, 1.0, b, np.full((N, K // 16), 0x38, np.uint8), 1.0)
+    assert np.array_equal(d, np.full((M, N), (K // 32) * (16.0 + 16.0 * 2.0 ** -9)))
+
+
 def test_gptq_block_second_column_takes_the_obs_correction():
     """Two columns, Hb = [[a, b], [b, c]] undamped: after column 0 is rounded, column 1
     moves by (w0 - q0) b / c (the optimal brain surgeon update), then is rounded."""
