@@ -592,42 +592,50 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
       const uint32_t tq = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(acc * Cfg::ACC_COLS);
       ScaleT sc[BPT];
       if (warp_live) tc_fence_after();
+      // one 64-column TMEM load per step: one G = 32 block, or two G = 16 blocks whose
+      // quantisation chains are independent, so the scheduler can interleave them
+      constexpr int BPL = 32 / G;                     // blocks per load
 #pragma unroll
-      for (int b = 0; b < BPT; ++b) {
-        float hl[2 * G];
-        if (warp_live) {
-          if constexpr (G == 32) tmem_ld64_sync(tq + static_cast<uint32_t>(b * 2 * G), hl);
-          else tmem_ld32_sync(tq + static_cast<uint32_t>(b * 2 * G), hl);
-        }
-        if (b == BPT - 1) {             // the whole accumulator buffer has been read
+      for (int bl = 0; bl < BPT / BPL; ++bl) {
+        float hl[64];
+        if (warp_live) tmem_ld64_sync(tq + static_cast<uint32_t>(bl * 64), hl);
+        if (bl == BPT / BPL - 1) {      // the whole accumulator buffer has been read
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(BAR(B_AEMPTY + acc));
         }
         if (!warp_live) continue;
 #pragma unroll
-        for (int jj = 0; jj < G; jj += 2) add2_rn(hl[jj], hl[jj + 1], hl[G + jj], hl[G + jj + 1]);  // hi + lo
-        const int blk = ct * BPT + b;
+        for (int u = 0; u < BPL; ++u) {
+          float* v = hl + u * 2 * G;
+#pragma unroll
+          for (int jj = 0; jj < G; jj += 2) add2_rn(v[jj], v[jj + 1], v[G + jj], v[G + jj + 1]);  // hi + lo
+        }
         if (Cfg::AMAX_ONLY) {
-          if (row_ok && blk < C) run_max = fmaxf(run_max, group_absmax<G>(hl));
+#pragma unroll
+          for (int u = 0; u < BPL; ++u)
+            if (row_ok && ct * BPT + bl * BPL + u < C) run_max = fmaxf(run_max, group_absmax<G>(hl + u * 2 * G));
           continue;
         }
-        if (Cfg::EMIT_Y && row_ok && blk < C) {
-          float4* yd = reinterpret_cast<float4*>(p.y_out + grow * p.d_in + static_cast<long long>(blk) * G);
+        uint32_t words[BPL][G / 8];
 #pragma unroll
-          for (int k = 0; k < G / 4; ++k) yd[k] = make_float4(hl[4 * k], hl[4 * k + 1], hl[4 * k + 2], hl[4 * k + 3]);
+        for (int u = 0; u < BPL; ++u) {
+          const float* v = hl + u * 2 * G;
+          const int b = bl * BPL + u;
+          const int blk = ct * BPT + b;
+          if (Cfg::EMIT_Y && row_ok && blk < C) {
+            float4* yd = reinterpret_cast<float4*>(p.y_out + grow * p.d_in + static_cast<long long>(blk) * G);
+#pragma unroll
+            for (int k = 0; k < G / 4; ++k) yd[k] = make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
+          }
+          if (Cfg::FMT == kMXFP4) sc[b] = static_cast<ScaleT>(quant_mx<G>(v, words[u]));
+          else if (Cfg::FMT == kNVFP4) sc[b] = static_cast<ScaleT>(quant_nv<G>(v, s_t, d6, words[u]));
+          else sc[b] = static_cast<ScaleT>(quant_int4<G>(v, words[u]));
         }
-        uint32_t words[G / 8];
-        if (Cfg::FMT == kMXFP4) sc[b] = static_cast<ScaleT>(quant_mx<G>(hl, words));
-        else if (Cfg::FMT == kNVFP4) sc[b] = static_cast<ScaleT>(quant_nv<G>(hl, s_t, d6, words));
-        else sc[b] = static_cast<ScaleT>(quant_int4<G>(hl, words));
-        const int c = (b * G) / 32;       // 16-byte chunk of this row's codes
-        const int pc = c ^ ((row >> SW_SHIFT) & (NCH - 1));
-        if constexpr (G == 32) {
-          *reinterpret_cast<uint4*>(cstage + row * (CH / 2) + pc * 16) = make_uint4(words[0], words[1], words[2], words[3]);
-        } else {                          // a G=16 block fills one 8-byte half of the chunk
-          *reinterpret_cast<uint2*>(cstage + row * (CH / 2) + pc * 16 + (b & 1) * 8) = make_uint2(words[0], words[1]);
-        }
+        // the load's 32 elements are one 16-byte chunk of this row's codes
+        const int pc = bl ^ ((row >> SW_SHIFT) & (NCH - 1));
+        const uint32_t* w = &words[0][0];
+        *reinterpret_cast<uint4*>(cstage + row * (CH / 2) + pc * 16) = make_uint4(w[0], w[1], w[2], w[3]);
       }
       if (Cfg::AMAX_ONLY) continue;
       // scales: this thread's row of the tile, straight from registers
@@ -721,7 +729,9 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
       for (int o = 16; o > 0; o >>= 1) run_max = fmaxf(run_max, __shfl_xor_sync(0xffffffffu, run_max, o));
       if (lane == 0 && run_max > 0.0f) atomicMax(p.amax_word, __float_as_uint(run_max));
     }
-    if (store_leader && p.codes_via_tma) bulk_wait_all();
+    // the last stores must have read their staging buffers before the CTA's shared
+    // memory goes away; their global writes complete with the grid
+    if (store_leader && p.codes_via_tma) bulk_wait_read_all();
   }
 
   tc_fence_before();
