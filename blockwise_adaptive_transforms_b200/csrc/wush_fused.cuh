@@ -611,31 +611,31 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
 #pragma unroll
           for (int jj = 0; jj < G; jj += 2) add2_rn(v[jj], v[jj + 1], v[G + jj], v[G + jj + 1]);  // hi + lo
         }
-        if (Cfg::AMAX_ONLY) {
+        if constexpr (Cfg::AMAX_ONLY) {
 #pragma unroll
           for (int u = 0; u < BPL; ++u)
             if (row_ok && ct * BPT + bl * BPL + u < C) run_max = fmaxf(run_max, group_absmax<G>(hl + u * 2 * G));
-          continue;
-        }
-        uint32_t words[BPL][G / 8];
+        } else {
+          uint32_t words[BPL][G / 8];
 #pragma unroll
-        for (int u = 0; u < BPL; ++u) {
-          const float* v = hl + u * 2 * G;
-          const int b = bl * BPL + u;
-          const int blk = ct * BPT + b;
-          if (Cfg::EMIT_Y && row_ok && blk < C) {
-            float4* yd = reinterpret_cast<float4*>(p.y_out + grow * p.d_in + static_cast<long long>(blk) * G);
+          for (int u = 0; u < BPL; ++u) {
+            const float* v = hl + u * 2 * G;
+            const int b = bl * BPL + u;
+            const int blk = ct * BPT + b;
+            if (Cfg::EMIT_Y && row_ok && blk < C) {
+              float4* yd = reinterpret_cast<float4*>(p.y_out + grow * p.d_in + static_cast<long long>(blk) * G);
 #pragma unroll
-            for (int k = 0; k < G / 4; ++k) yd[k] = make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
+              for (int k = 0; k < G / 4; ++k) yd[k] = make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
+            }
+            if (Cfg::FMT == kMXFP4) sc[b] = static_cast<ScaleT>(quant_mx<G>(v, words[u]));
+            else if (Cfg::FMT == kNVFP4) sc[b] = static_cast<ScaleT>(quant_nv<G>(v, s_t, d6, words[u]));
+            else sc[b] = static_cast<ScaleT>(quant_int4<G>(v, words[u]));
           }
-          if (Cfg::FMT == kMXFP4) sc[b] = static_cast<ScaleT>(quant_mx<G>(v, words[u]));
-          else if (Cfg::FMT == kNVFP4) sc[b] = static_cast<ScaleT>(quant_nv<G>(v, s_t, d6, words[u]));
-          else sc[b] = static_cast<ScaleT>(quant_int4<G>(v, words[u]));
+          // the load's 32 elements are one 16-byte chunk of this row's codes
+          const int pc = bl ^ ((row >> SW_SHIFT) & (NCH - 1));
+          const uint32_t* w = &words[0][0];
+          *reinterpret_cast<uint4*>(cstage + row * (CH / 2) + pc * 16) = make_uint4(w[0], w[1], w[2], w[3]);
         }
-        // the load's 32 elements are one 16-byte chunk of this row's codes
-        const int pc = bl ^ ((row >> SW_SHIFT) & (NCH - 1));
-        const uint32_t* w = &words[0][0];
-        *reinterpret_cast<uint4*>(cstage + row * (CH / 2) + pc * 16) = make_uint4(w[0], w[1], w[2], w[3]);
       }
       if (Cfg::AMAX_ONLY) continue;
       // scales: this thread's row of the tile, straight from registers
