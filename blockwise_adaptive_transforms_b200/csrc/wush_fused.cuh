@@ -658,11 +658,15 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
                     static_cast<uint32_t>(sc[4 * w4]) | (static_cast<uint32_t>(sc[4 * w4 + 1]) << 8) |
                     (static_cast<uint32_t>(sc[4 * w4 + 2]) << 16) | (static_cast<uint32_t>(sc[4 * w4 + 3]) << 24);
               } else {
-                for (int k = 4 * w4; k < nb; ++k) word[k - 4 * w4] = static_cast<uint8_t>(sc[k]);
+#pragma unroll
+                for (int k = 4 * w4; k < 4 * w4 + 4; ++k)   // compile-time indices keep sc in registers
+                  if (k < nb) word[k - 4 * w4] = static_cast<uint8_t>(sc[k]);
               }
             }
           } else {
-            for (int k = 0; k < nb; ++k) row_base[((col0 + k) >> 2) * 512 + ((col0 + k) & 3)] = static_cast<uint8_t>(sc[k]);
+#pragma unroll
+            for (int k = 0; k < BPT; ++k)
+              if (k < nb) row_base[((col0 + k) >> 2) * 512 + ((col0 + k) & 3)] = static_cast<uint8_t>(sc[k]);
           }
         }
       } else if (warp_live && row_ok) {
@@ -689,7 +693,9 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
             for (int k = 0; k < BPT; ++k) dst[k] = sc[k];
           }
         } else {
-          for (int k = 0; k < nb; ++k) dst[k] = sc[k];
+#pragma unroll
+          for (int k = 0; k < BPT; ++k)
+            if (k < nb) dst[k] = sc[k];
         }
       }
       if (warp_live && p.codes_via_tma) fence_proxy_async_smem();
