@@ -192,3 +192,43 @@ def test_nvfp4_layer_after_wush_quantisation():
     ref = O.bf16_to_f64(inp.x_bits) @ inp.w.astype(np.float64).T
     rel = np.linalg.norm(d.float().cpu().numpy() - ref) / np.linalg.norm(ref)
     assert rel < 0.25, rel
+
+
+@pytest.mark.parametrize("fmt", ["mxfp4", "nvfp4"])
+def test_gemm_at_the_benchmarked_shape(fmt):
+    """M = 1024, N = K = 4096 (the bench row), operands from the library's quantisers in
+    the scale-atom layout; 4096 sampled outputs against the oracle's product of the same
+    codes and scales (row-major scales from the row-major quantiser, which writes the same
+    codes)."""
+    M, N, K = 1024, 4096, 4096
+    g = torch.Generator().manual_seed(11)
+    x = torch.randn(M, K, generator=g).to(torch.bfloat16).cuda()
+    w = (torch.randn(N, K, generator=g) / K ** 0.5).cuda()
+    G = 32 if fmt == "mxfp4" else 16
+    T = (torch.eye(G) + 0.1 * torch.randn(K // G, G, G, generator=g)).cuda()
+    if fmt == "mxfp4":
+        cx, ax = W.wush_quant_act_mx_atoms(x, T)
+        cw, aw = W.wush_quant_weight_mx_atoms(w, T)
+        d = W.wush_gemm_mxfp4(cx, ax, cw, aw)
+        _, sx, _ = W.wush_quant_act(x, T, G, fmt)
+        _, sw, _ = W.wush_quant_weight(w, T, G, fmt)
+        ts_x = ts_w = None
+    else:
+        cx, ax, tx = W.wush_quant_act_nv_atoms(x, T)
+        cw, aw, tw = W.wush_quant_weight_nv_atoms(w, T)
+        d = W.wush_gemm_nvfp4(cx, ax, tx, cw, aw, tw)
+        _, sx, _ = W.wush_quant_act(x, T, G, fmt)
+        _, sw, _ = W.wush_quant_weight(w, T, G, fmt)
+        ts_x, ts_w = float(tx.item()), float(tw.item())
+    torch.cuda.synchronize()
+    st, bits = W.wush_device_status()
+    assert st == 0 and bits == 0, f"device error word {bits:#x}"
+    A = O.dequant(O.unpack_nibbles(cx.cpu().numpy()), sx.cpu().numpy(), fmt, G, ts_x)
+    B = O.dequant(O.unpack_nibbles(cw.cpu().numpy()), sw.cpu().numpy(), fmt, G, ts_w)
+    rng = np.random.default_rng(5)
+    mi, ni = rng.integers(0, M, 4096), rng.integers(0, N, 4096)
+    ref = np.einsum("ik,ik->i", A[mi], B[ni])
+    mag = np.einsum("ik,ik->i", np.abs(A[mi]), np.abs(B[ni]))
+    got = d.float().cpu().numpy()[mi, ni].astype(np.float64)
+    bound = 2.0 ** -8 * np.abs(ref) + (K + 2) * 2.0 ** -23 * mag + 1e-30
+    assert np.all(np.abs(got - ref) <= bound), np.max(np.abs(got - ref) / bound)
