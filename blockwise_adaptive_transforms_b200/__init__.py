@@ -22,7 +22,8 @@ __all__ = ["FMT", "WushError", "wush_quant_act", "wush_quant_weight", "wush_quan
            "EXPORTED_SYMBOLS", "output_shapes", "hadamard_matrix", "wush_dequant", "wush_gemm_mxfp4",
            "wush_mx_scales_to_atoms", "atom_bytes", "wush_quant_act_mx_atoms", "wush_quant_weight_mx_atoms",
            "wush_quant_act_shared_mx_atoms", "wush_gemm_nvfp4", "wush_quant_act_nv_atoms",
-           "wush_quant_weight_nv_atoms"]
+           "wush_quant_weight_nv_atoms", "wush_quant_act_nvfp4_amax", "wush_nvfp4_scale_from_amax",
+           "wush_quant_act_nvfp4_with_scale"]
 
 FMT = {"mxfp4": 0, "nvfp4": 1, "int4": 2}
 STATUS = {0: "WUSH_OK", 1: "WUSH_ERR_INVALID_ARG", 2: "WUSH_ERR_UNSUPPORTED", 3: "WUSH_ERR_MISALIGNED",
@@ -32,6 +33,7 @@ EXPORTED_SYMBOLS = ("wush_quant_act", "wush_quant_weight", "wush_quant_act_debug
                     "wush_dequant", "wush_gemm_mxfp4", "wush_mx_scales_to_atoms", "wush_quant_act_mx_atoms",
                     "wush_quant_weight_mx_atoms", "wush_quant_act_shared_mx_atoms",
                     "wush_gemm_nvfp4", "wush_quant_act_nv_atoms", "wush_quant_weight_nv_atoms",
+                    "wush_quant_act_nvfp4_amax", "wush_nvfp4_scale_from_amax", "wush_quant_act_nvfp4_with_scale",
                     "wush_build_transforms", "wush_device_status",
                     "wush_set_wait_limit_ns",
                     "wush_selftest_wait_timeout", "wush_status_string", "wush_version")
@@ -79,6 +81,12 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
     lib.wush_gemm_mxfp4.restype = ctypes.c_int
     lib.wush_gemm_nvfp4.argtypes = [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _P]
     lib.wush_gemm_nvfp4.restype = ctypes.c_int
+    lib.wush_quant_act_nvfp4_amax.argtypes = [_P, _P, _I64, _I64, _P, _P]
+    lib.wush_quant_act_nvfp4_amax.restype = ctypes.c_int
+    lib.wush_nvfp4_scale_from_amax.argtypes = [_P, _P]
+    lib.wush_nvfp4_scale_from_amax.restype = ctypes.c_int
+    lib.wush_quant_act_nvfp4_with_scale.argtypes = [_P, _P, _I64, _I64, _P, _P, _P, _P]
+    lib.wush_quant_act_nvfp4_with_scale.restype = ctypes.c_int
     lib.wush_mx_scales_to_atoms.argtypes = [_P, _I64, _I64, _P, _P]
     lib.wush_mx_scales_to_atoms.restype = ctypes.c_int
     lib.wush_build_transforms.argtypes = [_P, _P, _I64, _I64, _I64, _I32, ctypes.c_double, _I32,
@@ -325,6 +333,62 @@ def wush_quant_act_nv_atoms(x, T, codes=None, atoms=None, tensor_scale=None, str
 def wush_quant_weight_nv_atoms(w, T, codes=None, atoms=None, tensor_scale=None, stream=None):
     return _quant_atoms("wush_quant_weight_nv_atoms", w, torch.float32, T, codes, atoms, stream, G=16,
                         tensor_scale=tensor_scale)
+
+
+def _nv_stage_input(x, T):
+    _check_dev(x, "x", torch.bfloat16)
+    _check_dev(T, "T", torch.float32)
+    n, d = int(x.shape[0]), int(x.shape[1])
+    if d % 16 or tuple(T.shape) != (d // 16, 16, 16):
+        raise ValueError("NVFP4 needs d_in % 16 == 0 and T of shape [d_in/16][16][16]")
+    return n, d
+
+
+def wush_quant_act_nvfp4_amax(x, T, amax=None, stream=None):
+    """max |y| of this batch's G = 16 WUSH transform as a device fp32 tensor of one element
+    (the first NVFP4 stage; reduce it across ranks before fixing the scale)."""
+    lib = load_library()
+    n, d = _nv_stage_input(x, T)
+    if amax is None:
+        amax = torch.empty(1, dtype=torch.float32, device=x.device)
+    _check_dev(amax, "amax", torch.float32)
+    with torch.cuda.device(x.device):
+        st = lib.wush_quant_act_nvfp4_amax(_ptr(x), _ptr(T), n, d, _ptr(amax), _stream_handle(stream))
+    if st != 0:
+        raise WushError(st, "wush_quant_act_nvfp4_amax")
+    return amax
+
+
+def wush_nvfp4_scale_from_amax(amax, stream=None):
+    """In place: amax -> the tensor scale amax / 2688."""
+    lib = load_library()
+    _check_dev(amax, "amax", torch.float32)
+    with torch.cuda.device(amax.device):
+        st = lib.wush_nvfp4_scale_from_amax(_ptr(amax), _stream_handle(stream))
+    if st != 0:
+        raise WushError(st, "wush_nvfp4_scale_from_amax")
+    return amax
+
+
+def wush_quant_act_nvfp4_with_scale(x, T, tensor_scale, codes=None, scales=None, stream=None):
+    """NVFP4 codes and E4M3 scales of x under a given device tensor scale: (codes, scales)."""
+    lib = load_library()
+    n, d = _nv_stage_input(x, T)
+    _check_dev(tensor_scale, "tensor_scale", torch.float32)
+    if codes is None:
+        codes = torch.empty((n, d // 2), dtype=torch.uint8, device=x.device)
+    if scales is None:
+        scales = torch.empty((n, d // 16), dtype=torch.uint8, device=x.device)
+    _check_dev(codes, "codes", torch.uint8)
+    _check_dev(scales, "scales", torch.uint8)
+    if tuple(codes.shape) != (n, d // 2) or tuple(scales.shape) != (n, d // 16):
+        raise ValueError("output buffers have the wrong size")
+    with torch.cuda.device(x.device):
+        st = lib.wush_quant_act_nvfp4_with_scale(_ptr(x), _ptr(T), n, d, _ptr(codes), _ptr(scales),
+                                                 _ptr(tensor_scale), _stream_handle(stream))
+    if st != 0:
+        raise WushError(st, "wush_quant_act_nvfp4_with_scale")
+    return codes, scales
 
 
 def _gemm_args(a_codes, a_atoms, b_codes, b_atoms, out, vs):

@@ -120,9 +120,13 @@ int launch_pick_y(const CUtensorMap& map, const CUtensorMap& cmap, const wush::F
   return launch_fused<wush::FusedCfg<G, FMT, IN_F32, AMAX_ONLY, false, SHARED>>(map, cmap, p, s);
 }
 
+// NVFP4 stages: the whole call, the amax pass alone (for a max-reduction across ranks
+// before the scale is fixed), or the quantising pass with a given tensor scale
+enum NvMode { kNvAll = 0, kNvAmaxOnly = 1, kNvWithScale = 2 };
+
 template <bool IN_F32, bool SHARED>
 int dispatch(const CUtensorMap& map, const CUtensorMap& cmap, wush::FusedParams p, int G, int fmt, bool emit_y,
-             float* tensor_scale, cudaStream_t s) {
+             float* tensor_scale, cudaStream_t s, int nv_mode = kNvAll) {
   if (fmt == WUSH_MXFP4) return launch_pick_y<32, wush::kMXFP4, IN_F32, false, SHARED>(map, cmap, p, emit_y, s);
   if (fmt == WUSH_INT4) {
     if (G == 32) return launch_pick_y<32, wush::kINT4, IN_F32, false, SHARED>(map, cmap, p, emit_y, s);
@@ -130,32 +134,42 @@ int dispatch(const CUtensorMap& map, const CUtensorMap& cmap, wush::FusedParams 
   }
   // NVFP4: pass 1 finds amax|y| (float bits, running max in *tensor_scale), a one-thread
   // kernel turns it into s_t in place, pass 2 quantises with s_t.
-  if (cudaMemsetAsync(tensor_scale, 0, sizeof(float), s) != cudaSuccess) return WUSH_ERR_CUDA;
-  wush::FusedParams p1 = p;
-  p1.amax_word = reinterpret_cast<unsigned int*>(tensor_scale);
-  p1.codes_via_tma = 0;
-  int st = launch_fused<wush::FusedCfg<16, wush::kNVFP4, IN_F32, true, false, SHARED>>(map, cmap, p1, s);
-  if (st != WUSH_OK) return st;
-  wush::wush_nvfp4_tensor_scale_kernel<<<1, 32, 0, s>>>(tensor_scale);
-  if (cudaGetLastError() != cudaSuccess) return WUSH_ERR_CUDA;
+  if (nv_mode != kNvWithScale) {
+    if (cudaMemsetAsync(tensor_scale, 0, sizeof(float), s) != cudaSuccess) return WUSH_ERR_CUDA;
+    wush::FusedParams p1 = p;
+    p1.amax_word = reinterpret_cast<unsigned int*>(tensor_scale);
+    p1.codes_via_tma = 0;
+    int st = launch_fused<wush::FusedCfg<16, wush::kNVFP4, IN_F32, true, false, SHARED>>(map, cmap, p1, s);
+    if (st != WUSH_OK) return st;
+    if (nv_mode == kNvAmaxOnly) return WUSH_OK;
+    wush::wush_nvfp4_tensor_scale_kernel<<<1, 32, 0, s>>>(tensor_scale);
+    if (cudaGetLastError() != cudaSuccess) return WUSH_ERR_CUDA;
+  }
   p.tensor_scale = tensor_scale;
   return launch_pick_y<16, wush::kNVFP4, IN_F32, false, SHARED>(map, cmap, p, emit_y, s);
 }
 
 int quant_common(const void* in, bool in_f32, const float* T, int64_t rows, int64_t d_in, int G, int fmt,
                  uint8_t* codes, void* scales, float* tensor_scale, float* y_out, bool debug,
-                 wush_stream_t stream, bool shared_T = false, bool scale_atoms = false) {
+                 wush_stream_t stream, bool shared_T = false, bool scale_atoms = false, int nv_mode = kNvAll) {
   if (fmt != WUSH_MXFP4 && fmt != WUSH_NVFP4 && fmt != WUSH_INT4) return WUSH_ERR_UNSUPPORTED;
+  const bool amax_only = fmt == WUSH_NVFP4 && nv_mode == kNvAmaxOnly;   // no codes or scales written
   const bool g_ok = (fmt == WUSH_MXFP4 && G == 32) || (fmt == WUSH_NVFP4 && G == 16) ||
                     (fmt == WUSH_INT4 && (G == 16 || G == 32));
   if (!g_ok) return WUSH_ERR_UNSUPPORTED;
   if (rows < 0 || d_in <= 0 || d_in % G != 0) return WUSH_ERR_INVALID_ARG;
   if (rows > INT_MAX || d_in > INT_MAX) return WUSH_ERR_INVALID_ARG;
-  if (rows == 0) return WUSH_OK;   // empty batch: nothing to read or write, pointers unused
-  if (!in || !T || !codes || !scales) return WUSH_ERR_INVALID_ARG;
+  if (rows == 0) {                 // empty batch: nothing to read or write
+    if (!amax_only) return WUSH_OK;
+    if (!tensor_scale || !aligned(tensor_scale, 4)) return tensor_scale ? WUSH_ERR_MISALIGNED : WUSH_ERR_INVALID_ARG;
+    // an empty shard still contributes its amax (0) to a reduction across ranks
+    return cudaMemsetAsync(tensor_scale, 0, sizeof(float), reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? WUSH_OK : WUSH_ERR_CUDA;
+  }
+  if (!in || !T || (!amax_only && (!codes || !scales))) return WUSH_ERR_INVALID_ARG;
   if (fmt == WUSH_NVFP4 && !tensor_scale) return WUSH_ERR_INVALID_ARG;
   if (debug && !y_out) return WUSH_ERR_INVALID_ARG;
-  if (!aligned(in, 16) || !aligned(T, 16) || !aligned(codes, 16)) return WUSH_ERR_MISALIGNED;
+  if (!aligned(in, 16) || !aligned(T, 16) || (codes && !aligned(codes, 16))) return WUSH_ERR_MISALIGNED;
   if (fmt == WUSH_INT4 && !aligned(scales, 4)) return WUSH_ERR_MISALIGNED;
   if (scale_atoms && !aligned(scales, 16)) return WUSH_ERR_MISALIGNED;
   if (tensor_scale && !aligned(tensor_scale, 4)) return WUSH_ERR_MISALIGNED;
@@ -176,7 +190,7 @@ int quant_common(const void* in, bool in_f32, const float* T, int64_t rows, int6
   // the store map's swizzle matches the kernel's staging layout (64-byte rows: 64B
   // swizzle, 32-byte rows: 32B swizzle)
   CUtensorMap cmap = map;
-  const bool codes_tma = ((d_in / 2) % 16) == 0;
+  const bool codes_tma = !amax_only && ((d_in / 2) % 16) == 0;
   if (codes_tma) {
     st = encode_2d(&cmap, codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, rows, d_in / 2, ch / 2,
                    ch == 128 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B);
@@ -200,9 +214,9 @@ int quant_common(const void* in, bool in_f32, const float* T, int64_t rows, int6
   p.total_tiles = static_cast<int>(n_row_tiles * n_col_tiles);
   p.wait_limit_ns = g_wait_limit_ns.load(std::memory_order_relaxed);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (shared_T) return dispatch<false, true>(map, cmap, p, G, fmt, debug, tensor_scale, s);
-  return in_f32 ? dispatch<true, false>(map, cmap, p, G, fmt, debug, tensor_scale, s)
-                : dispatch<false, false>(map, cmap, p, G, fmt, debug, tensor_scale, s);
+  if (shared_T) return dispatch<false, true>(map, cmap, p, G, fmt, debug, tensor_scale, s, nv_mode);
+  return in_f32 ? dispatch<true, false>(map, cmap, p, G, fmt, debug, tensor_scale, s, nv_mode)
+                : dispatch<false, false>(map, cmap, p, G, fmt, debug, tensor_scale, s, nv_mode);
 }
 
 }  // namespace
@@ -401,6 +415,26 @@ int wush_quant_weight_nv_atoms(const float* w_f32, const float* T_blocks, int64_
                                uint8_t* scale_atoms, float* tensor_scale, wush_stream_t stream) {
   return quant_common(w_f32, true, T_blocks, d_out, d_in, 16, WUSH_NVFP4, codes, scale_atoms, tensor_scale, nullptr,
                       false, stream, false, true);
+}
+
+int wush_quant_act_nvfp4_amax(const void* x_bf16, const float* T_blocks, int64_t n_tok, int64_t d_in, float* amax,
+                              wush_stream_t stream) {
+  return quant_common(x_bf16, false, T_blocks, n_tok, d_in, 16, WUSH_NVFP4, nullptr, nullptr, amax, nullptr, false,
+                      stream, false, false, kNvAmaxOnly);
+}
+
+int wush_nvfp4_scale_from_amax(float* amax_to_scale, wush_stream_t stream) {
+  if (!amax_to_scale) return WUSH_ERR_INVALID_ARG;
+  if (!aligned(amax_to_scale, 4)) return WUSH_ERR_MISALIGNED;
+  wush::wush_nvfp4_tensor_scale_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(amax_to_scale);
+  return cudaGetLastError() == cudaSuccess ? WUSH_OK : WUSH_ERR_CUDA;
+}
+
+int wush_quant_act_nvfp4_with_scale(const void* x_bf16, const float* T_blocks, int64_t n_tok, int64_t d_in,
+                                    uint8_t* codes, uint8_t* scales, const float* tensor_scale,
+                                    wush_stream_t stream) {
+  return quant_common(x_bf16, false, T_blocks, n_tok, d_in, 16, WUSH_NVFP4, codes, scales,
+                      const_cast<float*>(tensor_scale), nullptr, false, stream, false, false, kNvWithScale);
 }
 
 int wush_build_transforms(const float* w_f32, const void* xcal_bf16, int64_t d_out, int64_t n_cal, int64_t d_in,

@@ -187,6 +187,25 @@ int wush_quant_weight_nv_atoms(const float* w_f32, const float* T_blocks, int64_
                                int64_t d_in, uint8_t* codes, uint8_t* scale_atoms,
                                float* tensor_scale, wush_stream_t stream);
 
+/* NVFP4 activations in stages, for a batch whose rows are split across ranks: the
+ * tensor scale s_t = amax / (6 * 448) must then come from the AbsMax over all ranks'
+ * transformed values (a max-reduction between the stages; the single-call
+ * wush_quant_act does all three steps on one device).
+ *   wush_quant_act_nvfp4_amax: *amax (device fp32) = max |y| over this batch (0 for an
+ *     empty batch), y = the G = 16 WUSH transform of x; writes no codes or scales.
+ *   wush_nvfp4_scale_from_amax: in place, *p = fl32(*p / 2688) (one thread).
+ *   wush_quant_act_nvfp4_with_scale: codes and E4M3 scales of x under the given device
+ *     fp32 tensor scale (read only) — the quantising pass of wush_quant_act.
+ * Same layouts, alignment and errors as wush_quant_act with fmt = NVFP4, G = 16; the
+ * three calls together give wush_quant_act's result bit for bit.  Asynchronous on
+ * `stream`, allocate nothing. */
+int wush_quant_act_nvfp4_amax(const void* x_bf16, const float* T_blocks, int64_t n_tok, int64_t d_in,
+                              float* amax, wush_stream_t stream);
+int wush_nvfp4_scale_from_amax(float* amax_to_scale, wush_stream_t stream);
+int wush_quant_act_nvfp4_with_scale(const void* x_bf16, const float* T_blocks, int64_t n_tok,
+                                    int64_t d_in, uint8_t* codes, uint8_t* scales,
+                                    const float* tensor_scale, wush_stream_t stream);
+
 /* Row-major one-byte scales [rows][C] (E8M0 or E4M3) -> the scale-atom layout the
  * block-scaled MMA reads:
  * rows padded to a multiple of 128 and C to a multiple of 4 (zero bytes); the atom of
