@@ -23,7 +23,7 @@ __all__ = ["FMT", "WushError", "wush_quant_act", "wush_quant_weight", "wush_quan
            "wush_mx_scales_to_atoms", "atom_bytes", "wush_quant_act_mx_atoms", "wush_quant_weight_mx_atoms",
            "wush_quant_act_shared_mx_atoms", "wush_gemm_nvfp4", "wush_quant_act_nv_atoms",
            "wush_quant_weight_nv_atoms", "wush_quant_act_nvfp4_amax", "wush_nvfp4_scale_from_amax",
-           "wush_quant_act_nvfp4_with_scale"]
+           "wush_quant_act_nvfp4_with_scale", "wush_set_small_batch_rows"]
 
 FMT = {"mxfp4": 0, "nvfp4": 1, "int4": 2}
 STATUS = {0: "WUSH_OK", 1: "WUSH_ERR_INVALID_ARG", 2: "WUSH_ERR_UNSUPPORTED", 3: "WUSH_ERR_MISALIGNED",
@@ -34,6 +34,7 @@ EXPORTED_SYMBOLS = ("wush_quant_act", "wush_quant_weight", "wush_quant_act_debug
                     "wush_quant_weight_mx_atoms", "wush_quant_act_shared_mx_atoms",
                     "wush_gemm_nvfp4", "wush_quant_act_nv_atoms", "wush_quant_weight_nv_atoms",
                     "wush_quant_act_nvfp4_amax", "wush_nvfp4_scale_from_amax", "wush_quant_act_nvfp4_with_scale",
+                    "wush_set_small_batch_rows",
                     "wush_build_transforms", "wush_device_status",
                     "wush_set_wait_limit_ns",
                     "wush_selftest_wait_timeout", "wush_status_string", "wush_version")
@@ -94,6 +95,8 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
     lib.wush_build_transforms.restype = ctypes.c_int
     lib.wush_device_status.argtypes = [_P, ctypes.POINTER(ctypes.c_uint32)]
     lib.wush_device_status.restype = ctypes.c_int
+    lib.wush_set_small_batch_rows.argtypes = [_I64]
+    lib.wush_set_small_batch_rows.restype = ctypes.c_int
     lib.wush_set_wait_limit_ns.argtypes = [_U64]
     lib.wush_set_wait_limit_ns.restype = ctypes.c_int
     lib.wush_selftest_wait_timeout.argtypes = [_U64, _P, ctypes.POINTER(ctypes.c_uint32)]
@@ -485,6 +488,13 @@ def wush_device_status(stream=None):
     bits = ctypes.c_uint32(0)
     st = load_library().wush_device_status(_stream_handle(stream), ctypes.byref(bits))
     return int(st), int(bits.value)
+
+
+def wush_set_small_batch_rows(rows: int) -> None:
+    """Activation batches of at most `rows` rows use the CUDA-core path (0: never; < 0: default)."""
+    st = load_library().wush_set_small_batch_rows(int(rows))
+    if st != 0:
+        raise WushError(st, "wush_set_small_batch_rows")
 
 
 def wush_set_wait_limit_ns(ns: int) -> None:

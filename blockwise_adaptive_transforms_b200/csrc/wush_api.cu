@@ -15,6 +15,7 @@
 #include "wush_build.cuh"
 #include "wush_dequant.cuh"
 #include "wush_gemm.cuh"
+#include "wush_small.cuh"
 
 namespace wush {
 // Waits on an mbarrier that no thread ever arrives on; the bounded wait must give up.
@@ -149,6 +150,42 @@ int dispatch(const CUtensorMap& map, const CUtensorMap& cmap, wush::FusedParams 
   return launch_pick_y<16, wush::kNVFP4, IN_F32, false, SHARED>(map, cmap, p, emit_y, s);
 }
 
+// Activation batches of at most this many rows take the CUDA-core path (wush_small.cuh);
+// 0 sends every batch to the fused tensor-core kernel.
+constexpr long long kDefaultSmallRows = 64;
+std::atomic<long long> g_small_rows{kDefaultSmallRows};
+
+template <int G, int FMT, bool AMAX_ONLY, bool SHARED>
+int launch_small(const void* x, const wush::FusedParams& p, bool emit_y, cudaStream_t s) {
+  const dim3 grid(static_cast<unsigned>(p.C), static_cast<unsigned>((p.n_rows + wush::kSmallRows - 1) / wush::kSmallRows));
+  const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
+  if (emit_y && !AMAX_ONLY)
+    wush::wush_small_kernel<G, FMT, AMAX_ONLY, true, SHARED><<<grid, wush::kSmallRows, 0, s>>>(xb, p);
+  else
+    wush::wush_small_kernel<G, FMT, AMAX_ONLY, false, SHARED><<<grid, wush::kSmallRows, 0, s>>>(xb, p);
+  return cudaGetLastError() == cudaSuccess ? WUSH_OK : WUSH_ERR_CUDA;
+}
+
+template <bool SHARED>
+int small_dispatch(const void* x, wush::FusedParams p, int G, int fmt, bool emit_y, float* tensor_scale,
+                   cudaStream_t s, int nv_mode) {
+  if (fmt == WUSH_MXFP4) return launch_small<32, wush::kMXFP4, false, SHARED>(x, p, emit_y, s);
+  if (fmt == WUSH_INT4)
+    return G == 32 ? launch_small<32, wush::kINT4, false, SHARED>(x, p, emit_y, s)
+                   : launch_small<16, wush::kINT4, false, SHARED>(x, p, emit_y, s);
+  if (nv_mode != kNvWithScale) {   // NVFP4: amax pass, tensor scale, quantising pass
+    if (cudaMemsetAsync(tensor_scale, 0, sizeof(float), s) != cudaSuccess) return WUSH_ERR_CUDA;
+    wush::FusedParams p1 = p;
+    p1.amax_word = reinterpret_cast<unsigned int*>(tensor_scale);
+    const int st = launch_small<16, wush::kNVFP4, true, SHARED>(x, p1, false, s);
+    if (st != WUSH_OK || nv_mode == kNvAmaxOnly) return st;
+    wush::wush_nvfp4_tensor_scale_kernel<<<1, 32, 0, s>>>(tensor_scale);
+    if (cudaGetLastError() != cudaSuccess) return WUSH_ERR_CUDA;
+  }
+  p.tensor_scale = tensor_scale;
+  return launch_small<16, wush::kNVFP4, false, SHARED>(x, p, emit_y, s);
+}
+
 int quant_common(const void* in, bool in_f32, const float* T, int64_t rows, int64_t d_in, int G, int fmt,
                  uint8_t* codes, void* scales, float* tensor_scale, float* y_out, bool debug,
                  wush_stream_t stream, bool shared_T = false, bool scale_atoms = false, int nv_mode = kNvAll) {
@@ -174,6 +211,20 @@ int quant_common(const void* in, bool in_f32, const float* T, int64_t rows, int6
   if (scale_atoms && !aligned(scales, 16)) return WUSH_ERR_MISALIGNED;
   if (tensor_scale && !aligned(tensor_scale, 4)) return WUSH_ERR_MISALIGNED;
   if (debug && !aligned(y_out, 16)) return WUSH_ERR_MISALIGNED;
+
+  if (!in_f32 && !scale_atoms && rows <= g_small_rows.load(std::memory_order_relaxed)) {
+    wush::FusedParams p{};
+    p.T = T;
+    p.codes = codes;
+    p.scales = scales;
+    p.y_out = y_out;
+    p.n_rows = rows;
+    p.d_in = static_cast<int>(d_in);
+    p.C = static_cast<int>(d_in / G);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    return shared_T ? small_dispatch<true>(in, p, G, fmt, debug, tensor_scale, s, nv_mode)
+                    : small_dispatch<false>(in, p, G, fmt, debug, tensor_scale, s, nv_mode);
+  }
 
   const int ch = in_f32 ? 64 : WUSH_ACT_TILE_CH;   // channels per tile, as in FusedCfg
   const long long n_row_tiles = (rows + 127) / 128;
@@ -435,6 +486,13 @@ int wush_quant_act_nvfp4_with_scale(const void* x_bf16, const float* T_blocks, i
                                     wush_stream_t stream) {
   return quant_common(x_bf16, false, T_blocks, n_tok, d_in, 16, WUSH_NVFP4, codes, scales,
                       const_cast<float*>(tensor_scale), nullptr, false, stream, false, false, kNvWithScale);
+}
+
+int wush_set_small_batch_rows(int64_t rows) {
+  if (rows < 0) rows = kDefaultSmallRows;
+  if (rows > (1 << 20)) return WUSH_ERR_INVALID_ARG;
+  g_small_rows.store(rows, std::memory_order_relaxed);
+  return WUSH_OK;
 }
 
 int wush_build_transforms(const float* w_f32, const void* xcal_bf16, int64_t d_out, int64_t n_cal, int64_t d_in,

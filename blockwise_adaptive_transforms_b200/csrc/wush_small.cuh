@@ -1,0 +1,85 @@
+// Decode-sized batches on CUDA cores: the same per-block transform and group
+// quantisation as the fused tensor-core kernel (paper-graph-ui analysis, section 3.2
+// "Online Activation Transform + Quantize Kernel": per token t and block i,
+// y[t, iG + r] = sum_c T_i[r, c] x[t, iG + c], then RTN AbsMax quantisation of the
+// group), for batches of a few to ~100 token rows.  There the fused kernel's fixed
+// latency (TMA set-up, transform split into bf16 hi/lo panels, MMA pipeline fill) is most
+// of the call; here one CTA takes one block i and up to 128 rows, stages T_i (fp32) in
+// shared memory, and each thread forms its row's group with fp32 FMAs (sequential over c,
+// so y is within a few fp32 ulps of the exact sum) and quantises it with the fused
+// kernel's group quantisers.  Rows of the same CTA read T_i as shared-memory broadcasts.
+#pragma once
+#include <cstdint>
+#include <cuda_bf16.h>
+#include "wush_fused.cuh"
+
+namespace wush {
+
+constexpr int kSmallRows = 128;   // rows (threads) per CTA
+
+template <int G, int FMT, bool AMAX_ONLY, bool EMIT_Y, bool SHARED_T>
+__global__ void __launch_bounds__(kSmallRows)
+    wush_small_kernel(const __nv_bfloat16* __restrict__ x, const FusedParams p) {
+  __shared__ __align__(16) float Ts[G * G];
+  const int blk = static_cast<int>(blockIdx.x);
+  const long long row = static_cast<long long>(blockIdx.y) * kSmallRows + threadIdx.x;
+  const bool valid = row < p.n_rows;
+  const float4* tg = reinterpret_cast<const float4*>(p.T + (SHARED_T ? 0ll : static_cast<long long>(blk) * G * G));
+  for (int k = threadIdx.x; k < G * G / 4; k += kSmallRows) reinterpret_cast<float4*>(Ts)[k] = tg[k];
+  __syncthreads();
+
+  float y[G];
+  if (valid) {
+    float xv[G];
+    const uint4* xs = reinterpret_cast<const uint4*>(x + row * p.d_in + static_cast<long long>(blk) * G);
+#pragma unroll
+    for (int k = 0; k < G / 8; ++k) {   // 8 bf16 per 16-byte load; bf16 -> fp32 is exact
+      const uint4 u = xs[k];
+      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        xv[8 * k + 2 * j] = __uint_as_float(w[j] << 16);
+        xv[8 * k + 2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < G; ++r) {
+      float acc = 0.0f;
+#pragma unroll
+      for (int c = 0; c < G; ++c) acc = __fmaf_rn(Ts[r * G + c], xv[c], acc);
+      y[r] = acc;
+    }
+  } else {
+#pragma unroll
+    for (int r = 0; r < G; ++r) y[r] = 0.0f;
+  }
+
+  if constexpr (AMAX_ONLY) {
+    float m = group_absmax<G>(y);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if ((threadIdx.x & 31) == 0 && m > 0.0f) atomicMax(p.amax_word, __float_as_uint(m));
+    return;
+  }
+  if (!valid) return;
+  if (EMIT_Y) {
+    float4* yd = reinterpret_cast<float4*>(p.y_out + row * p.d_in + static_cast<long long>(blk) * G);
+#pragma unroll
+    for (int k = 0; k < G / 4; ++k) yd[k] = make_float4(y[4 * k], y[4 * k + 1], y[4 * k + 2], y[4 * k + 3]);
+  }
+  uint32_t words[G / 8];
+  uint8_t* cdst = p.codes + row * (p.d_in / 2) + static_cast<long long>(blk) * (G / 2);
+  if constexpr (FMT == kMXFP4) {
+    static_cast<uint8_t*>(p.scales)[row * p.C + blk] = static_cast<uint8_t>(quant_mx<G>(y, words));
+  } else if constexpr (FMT == kNVFP4) {
+    const float s_t = *p.tensor_scale;
+    static_cast<uint8_t*>(p.scales)[row * p.C + blk] =
+        static_cast<uint8_t>(quant_nv<G>(y, s_t, __fmul_rn(6.0f, s_t), words));
+  } else {
+    static_cast<float*>(p.scales)[row * p.C + blk] = quant_int4<G>(y, words);
+  }
+  if constexpr (G == 32) *reinterpret_cast<uint4*>(cdst) = make_uint4(words[0], words[1], words[2], words[3]);
+  else *reinterpret_cast<uint2*>(cdst) = make_uint2(words[0], words[1]);
+}
+
+}  // namespace wush

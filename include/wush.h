@@ -250,6 +250,16 @@ int wush_build_transforms(const float* w_f32, const void* xcal_bf16, int64_t d_o
  * `bits` is not NULL it receives the raw word. */
 int wush_device_status(wush_stream_t stream, uint32_t* bits);
 
+/* Activation batches (bf16 input, row-major scales) of at most `rows` rows take a
+ * CUDA-core path instead of the fused tensor-core kernel: one CTA per block and 128 rows,
+ * T_i staged in shared memory, y = T_i x in fp32 FMAs, then the same group quantisers
+ * (codes, scales and NVFP4 tensor scale in the same layouts; y differs from the tensor-core
+ * path's by fp32 rounding only).  At decode sizes the fused kernel's fixed start-up
+ * latency dominates.  rows = 0 sends every batch to the fused kernel; rows < 0 restores
+ * the default (64).  Applies to later calls on every device; returns WUSH_OK, or
+ * WUSH_ERR_INVALID_ARG above 2^20 rows. */
+int wush_set_small_batch_rows(int64_t rows);
+
 /* Sets the bound of every in-kernel wait for later launches, in nanoseconds
  * (0 restores the default of 2 s).  Returns WUSH_OK. */
 int wush_set_wait_limit_ns(uint64_t ns);

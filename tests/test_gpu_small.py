@@ -1,0 +1,101 @@
+"""The CUDA-core path for decode-sized activation batches vs the fp64 oracle (needs a B200).
+
+Batches of at most `wush_set_small_batch_rows` rows (default 64) skip the fused
+tensor-core kernel.  Each case checks rule 1 (the oracle's quantiser on the kernel's own
+fp32 y gives the kernel's codes and scales bit for bit), that y is the fp32-FMA transform
+(within G * 2^-23 of |T_i||x| of the float64 product), rule 2 end to end, and the same
+two rules for the fused kernel forced onto the same batch (the two paths' y differ by
+rounding, so for NVFP4 even their tensor scales may differ: each is held to the oracle).
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import wush_oracle as O
+from workloads import make_inputs, workload
+import blockwise_adaptive_transforms_b200 as W
+from parity_rules import assert_bit_exact, assert_end_to_end
+
+pytestmark = pytest.mark.gpu
+
+CASES = [  # workload, fmt, G, d_in (ragged block counts)
+    ("attn_mxfp4_4096", "mxfp4", 32, 1056),
+    ("mlp_down_nvfp4_14336", "nvfp4", 16, 1040),
+    ("int4_sweep_4096", "int4", 32, 1056),
+    ("int4_sweep_4096", "int4", 16, 1040),
+]
+
+
+@pytest.fixture(autouse=True)
+def _default_threshold():
+    W.wush_set_small_batch_rows(-1)
+    yield
+    W.wush_set_small_batch_rows(-1)
+
+
+def _data(name, fmt, G, d_in, n_tok):
+    over = dict(n_tok=n_tok, d_in=d_in, d_out=2048, n_cal=512)   # transforms from a realistically wide layer
+    if name == "int4_sweep_4096":
+        over["G"] = G
+    wl = workload(name, **over)
+    inp = make_inputs(wl)
+    b = O.build_transforms(inp.w, inp.xcal_bits, G)
+    x = torch.from_numpy(np.ascontiguousarray(inp.x_bits).view(np.int16)).cuda().view(torch.bfloat16)
+    return inp, b, x, torch.from_numpy(b["T_wush32"]).cuda()
+
+
+def _ts(ts):
+    return None if ts is None else float(ts.item())
+
+
+@pytest.mark.parametrize("n_tok", [1, 7, 64])
+@pytest.mark.parametrize("name,fmt,G,d_in", CASES)
+def test_small_batches_against_the_oracle(name, fmt, G, d_in, n_tok):
+    inp, b, x, T = _data(name, fmt, G, d_in, n_tok)
+    c, s, ts, y = W.wush_quant_act_debug(x, T, G, fmt)
+    c2, s2, ts2 = W.wush_quant_act(x, T, G, fmt)
+    torch.cuda.synchronize()
+    st, bits = W.wush_device_status()
+    assert st == 0 and bits == 0, f"device error word {bits:#x}"
+    assert torch.equal(c, c2) and torch.equal(s, s2)
+    assert_bit_exact(c.cpu().numpy(), s.cpu().numpy(), _ts(ts), y.cpu().numpy(), fmt, G)
+    x64 = O.bf16_to_f64(inp.x_bits)
+    y_ref = O.block_transform(x64, b["T_wush32"].astype(np.float64))
+    bound = O.block_transform(np.abs(x64), np.abs(b["T_wush32"].astype(np.float64)))
+    assert np.all(np.abs(y.cpu().numpy() - y_ref) <= G * 2.0 ** -23 * bound + 1e-300)
+    assert_end_to_end(c.cpu().numpy(), s.cpu().numpy(), _ts(ts), y_ref, fmt, G)
+
+    # the fused tensor-core kernel on the same batch
+    W.wush_set_small_batch_rows(0)
+    cf, sf, tsf, yf = W.wush_quant_act_debug(x, T, G, fmt)
+    torch.cuda.synchronize()
+    assert_bit_exact(cf.cpu().numpy(), sf.cpu().numpy(), _ts(tsf), yf.cpu().numpy(), fmt, G)
+    assert_end_to_end(cf.cpu().numpy(), sf.cpu().numpy(), _ts(tsf), y_ref, fmt, G)
+
+
+def test_shared_matrix_small_batch_equals_per_block_copies():
+    inp, b, x, _ = _data("attn_mxfp4_4096", "mxfp4", 32, 1024, 5)
+    H = W.hadamard_matrix(32)
+    c, s, _ = W.wush_quant_act_shared(x, H, 32, "mxfp4")
+    c2, s2, _ = W.wush_quant_act(x, H.repeat(32, 1, 1).contiguous(), 32, "mxfp4")
+    torch.cuda.synchronize()
+    assert torch.equal(c, c2) and torch.equal(s, s2)
+
+
+def test_nvfp4_stages_take_the_small_path_too():
+    inp, b, x, T = _data("mlp_down_nvfp4_14336", "nvfp4", 16, 1024, 40)
+    c, s, ts = W.wush_quant_act(x, T, 16, "nvfp4")
+    a0 = W.wush_quant_act_nvfp4_amax(x[:17], T)
+    a1 = W.wush_quant_act_nvfp4_amax(x[17:], T)
+    amax = torch.maximum(a0, a1)
+    W.wush_nvfp4_scale_from_amax(amax)
+    c0, s0 = W.wush_quant_act_nvfp4_with_scale(x[:17], T, amax)
+    c1, s1 = W.wush_quant_act_nvfp4_with_scale(x[17:], T, amax)
+    torch.cuda.synchronize()
+    assert torch.equal(amax, ts)
+    assert torch.equal(torch.cat([c0, c1]), c) and torch.equal(torch.cat([s0, s1]), s)
+
+
+def test_threshold_setter_rejects_huge_values():
+    with pytest.raises(W.WushError):
+        W.wush_set_small_batch_rows(1 << 21)
