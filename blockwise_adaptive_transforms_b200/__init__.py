@@ -23,7 +23,8 @@ __all__ = ["FMT", "WushError", "wush_quant_act", "wush_quant_weight", "wush_quan
            "wush_mx_scales_to_atoms", "atom_bytes", "wush_quant_act_mx_atoms", "wush_quant_weight_mx_atoms",
            "wush_quant_act_shared_mx_atoms", "wush_gemm_nvfp4", "wush_quant_act_nv_atoms",
            "wush_quant_weight_nv_atoms", "wush_quant_act_nvfp4_amax", "wush_nvfp4_scale_from_amax",
-           "wush_quant_act_nvfp4_with_scale", "wush_set_small_batch_rows"]
+           "wush_quant_act_nvfp4_with_scale", "wush_set_small_batch_rows", "wush_quant_act_nvfp4_onepass",
+           "nvfp4_workspace"]
 
 FMT = {"mxfp4": 0, "nvfp4": 1, "int4": 2}
 STATUS = {0: "WUSH_OK", 1: "WUSH_ERR_INVALID_ARG", 2: "WUSH_ERR_UNSUPPORTED", 3: "WUSH_ERR_MISALIGNED",
@@ -34,7 +35,7 @@ EXPORTED_SYMBOLS = ("wush_quant_act", "wush_quant_weight", "wush_quant_act_debug
                     "wush_quant_weight_mx_atoms", "wush_quant_act_shared_mx_atoms",
                     "wush_gemm_nvfp4", "wush_quant_act_nv_atoms", "wush_quant_weight_nv_atoms",
                     "wush_quant_act_nvfp4_amax", "wush_nvfp4_scale_from_amax", "wush_quant_act_nvfp4_with_scale",
-                    "wush_set_small_batch_rows",
+                    "wush_set_small_batch_rows", "wush_quant_act_nvfp4_onepass",
                     "wush_build_transforms", "wush_device_status",
                     "wush_set_wait_limit_ns",
                     "wush_selftest_wait_timeout", "wush_status_string", "wush_version")
@@ -95,6 +96,8 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
     lib.wush_build_transforms.restype = ctypes.c_int
     lib.wush_device_status.argtypes = [_P, ctypes.POINTER(ctypes.c_uint32)]
     lib.wush_device_status.restype = ctypes.c_int
+    lib.wush_quant_act_nvfp4_onepass.argtypes = [_P, _P, _I64, _I64, _P, _P, _P, _P, _P]
+    lib.wush_quant_act_nvfp4_onepass.restype = ctypes.c_int
     lib.wush_set_small_batch_rows.argtypes = [_I64]
     lib.wush_set_small_batch_rows.restype = ctypes.c_int
     lib.wush_set_wait_limit_ns.argtypes = [_U64]
@@ -392,6 +395,36 @@ def wush_quant_act_nvfp4_with_scale(x, T, tensor_scale, codes=None, scales=None,
     if st != 0:
         raise WushError(st, "wush_quant_act_nvfp4_with_scale")
     return codes, scales
+
+
+def nvfp4_workspace(device=None):
+    """A zeroed workspace for wush_quant_act_nvfp4_onepass (16 bytes of device memory)."""
+    return torch.zeros(4, dtype=torch.int32, device=device if device is not None else "cuda")
+
+
+def wush_quant_act_nvfp4_onepass(x, T, workspace, codes=None, scales=None, tensor_scale=None, stream=None):
+    """NVFP4 activations of a decode-sized batch in one launch: (codes, scales, tensor_scale).
+    ``workspace``: from nvfp4_workspace(); zero before the first call, left zero by each."""
+    lib = load_library()
+    n, d = _nv_stage_input(x, T)
+    _check_dev(workspace, "workspace", torch.int32)
+    if codes is None:
+        codes = torch.empty((n, d // 2), dtype=torch.uint8, device=x.device)
+    if scales is None:
+        scales = torch.empty((n, d // 16), dtype=torch.uint8, device=x.device)
+    if tensor_scale is None:
+        tensor_scale = torch.empty(1, dtype=torch.float32, device=x.device)
+    for t, name, dt in ((codes, "codes", torch.uint8), (scales, "scales", torch.uint8),
+                        (tensor_scale, "tensor_scale", torch.float32)):
+        _check_dev(t, name, dt)
+    if tuple(codes.shape) != (n, d // 2) or tuple(scales.shape) != (n, d // 16) or workspace.numel() < 4:
+        raise ValueError("output or workspace buffers have the wrong size")
+    with torch.cuda.device(x.device):
+        st = lib.wush_quant_act_nvfp4_onepass(_ptr(x), _ptr(T), n, d, _ptr(codes), _ptr(scales), _ptr(tensor_scale),
+                                              _ptr(workspace), _stream_handle(stream))
+    if st != 0:
+        raise WushError(st, "wush_quant_act_nvfp4_onepass")
+    return codes, scales, tensor_scale
 
 
 def _gemm_args(a_codes, a_atoms, b_codes, b_atoms, out, vs):

@@ -488,6 +488,49 @@ int wush_quant_act_nvfp4_with_scale(const void* x_bf16, const float* T_blocks, i
                       const_cast<float*>(tensor_scale), nullptr, false, stream, false, false, kNvWithScale);
 }
 
+int wush_quant_act_nvfp4_onepass(const void* x_bf16, const float* T_blocks, int64_t n_tok, int64_t d_in,
+                                 uint8_t* codes, uint8_t* scales, float* tensor_scale, uint32_t* workspace,
+                                 wush_stream_t stream) {
+  if (n_tok < 0 || d_in <= 0 || d_in % 16 != 0 || n_tok > INT_MAX || d_in > INT_MAX) return WUSH_ERR_INVALID_ARG;
+  if (n_tok == 0) return WUSH_OK;
+  if (!x_bf16 || !T_blocks || !codes || !scales || !tensor_scale || !workspace) return WUSH_ERR_INVALID_ARG;
+  if (!aligned(x_bf16, 16) || !aligned(T_blocks, 16) || !aligned(codes, 16) || !aligned(tensor_scale, 4) ||
+      !aligned(workspace, 16))
+    return WUSH_ERR_MISALIGNED;
+  const long long C = d_in / 16;
+  const long long gy = (n_tok + wush::kSmallRows - 1) / wush::kSmallRows;
+  int dev = 0, sms = 0, per_sm = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return WUSH_ERR_CUDA;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return WUSH_ERR_CUDA;
+  auto kern = wush::wush_small_nvfp4_onepass_kernel<false, false>;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, wush::kSmallRows, 0) != cudaSuccess)
+    return WUSH_ERR_CUDA;
+  // the CTAs wait on one another: the whole grid must be resident at once
+  if (C * gy > static_cast<long long>(per_sm) * sms || gy > 65535) return WUSH_ERR_UNSUPPORTED;
+  wush::FusedParams p{};
+  p.T = T_blocks;
+  p.codes = codes;
+  p.scales = scales;
+  p.tensor_scale = tensor_scale;
+  p.n_rows = n_tok;
+  p.d_in = static_cast<int>(d_in);
+  p.C = static_cast<int>(C);
+  p.wait_limit_ns = g_wait_limit_ns.load(std::memory_order_relaxed);
+  cudaLaunchConfig_t lc = {};
+  lc.gridDim = dim3(static_cast<unsigned>(C), static_cast<unsigned>(gy));
+  lc.blockDim = dim3(wush::kSmallRows);
+  lc.stream = reinterpret_cast<cudaStream_t>(stream);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  lc.attrs = attr;
+  lc.numAttrs = 1;
+  if (cudaLaunchKernelEx(&lc, kern, static_cast<const __nv_bfloat16*>(x_bf16), p,
+                         reinterpret_cast<unsigned int*>(workspace)) != cudaSuccess)
+    return WUSH_ERR_CUDA;
+  return cudaGetLastError() == cudaSuccess ? WUSH_OK : WUSH_ERR_CUDA;
+}
+
 int wush_set_small_batch_rows(int64_t rows) {
   if (rows < 0) rows = kDefaultSmallRows;
   if (rows > (1 << 20)) return WUSH_ERR_INVALID_ARG;

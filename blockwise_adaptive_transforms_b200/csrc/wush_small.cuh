@@ -17,18 +17,17 @@ namespace wush {
 
 constexpr int kSmallRows = 128;   // rows (threads) per CTA
 
-template <int G, int FMT, bool AMAX_ONLY, bool EMIT_Y, bool SHARED_T>
-__global__ void __launch_bounds__(kSmallRows)
-    wush_small_kernel(const __nv_bfloat16* __restrict__ x, const FusedParams p) {
-  __shared__ __align__(16) float Ts[G * G];
+// Stages T_i in shared memory and forms this thread's row group y = T_i x (zeros for rows
+// past the batch).  Every thread of the CTA must call it (it synchronises the CTA).
+template <int G, bool SHARED_T>
+__device__ __forceinline__ void small_transform(const __nv_bfloat16* __restrict__ x, const FusedParams& p,
+                                                float* Ts, float (&y)[G], bool& valid, long long& row) {
   const int blk = static_cast<int>(blockIdx.x);
-  const long long row = static_cast<long long>(blockIdx.y) * kSmallRows + threadIdx.x;
-  const bool valid = row < p.n_rows;
+  row = static_cast<long long>(blockIdx.y) * kSmallRows + threadIdx.x;
+  valid = row < p.n_rows;
   const float4* tg = reinterpret_cast<const float4*>(p.T + (SHARED_T ? 0ll : static_cast<long long>(blk) * G * G));
   for (int k = threadIdx.x; k < G * G / 4; k += kSmallRows) reinterpret_cast<float4*>(Ts)[k] = tg[k];
   __syncthreads();
-
-  float y[G];
   if (valid) {
     float xv[G];
     const uint4* xs = reinterpret_cast<const uint4*>(x + row * p.d_in + static_cast<long long>(blk) * G);
@@ -53,6 +52,17 @@ __global__ void __launch_bounds__(kSmallRows)
 #pragma unroll
     for (int r = 0; r < G; ++r) y[r] = 0.0f;
   }
+}
+
+template <int G, int FMT, bool AMAX_ONLY, bool EMIT_Y, bool SHARED_T>
+__global__ void __launch_bounds__(kSmallRows)
+    wush_small_kernel(const __nv_bfloat16* __restrict__ x, const FusedParams p) {
+  __shared__ __align__(16) float Ts[G * G];
+  const int blk = static_cast<int>(blockIdx.x);
+  float y[G];
+  bool valid;
+  long long row;
+  small_transform<G, SHARED_T>(x, p, Ts, y, valid, row);
 
   if constexpr (AMAX_ONLY) {
     float m = group_absmax<G>(y);
@@ -80,6 +90,77 @@ __global__ void __launch_bounds__(kSmallRows)
   }
   if constexpr (G == 32) *reinterpret_cast<uint4*>(cdst) = make_uint4(words[0], words[1], words[2], words[3]);
   else *reinterpret_cast<uint2*>(cdst) = make_uint2(words[0], words[1]);
+}
+
+// NVFP4 in one launch for decode-sized batches.  The tensor scale s_t = amax / 2688 needs
+// max |y| over the whole batch before any group can be quantised, so the CTAs meet once:
+// each folds its maximum into ws[0] (float bits, atomicMax), counts itself into ws[1], and
+// waits (bounded in time) until ws[1] reaches the grid size; then every CTA quantises
+// with the same s_t, and the last CTA to leave (ws[2]) puts the three words back to zero.
+// The CTAs wait on one another, so the host launches this only as a cooperative launch
+// whose grid is resident at once.  ws: three words, zero before the launch, zero after a
+// launch that completed without error.
+template <bool EMIT_Y, bool SHARED_T>
+__global__ void __launch_bounds__(kSmallRows)
+    wush_small_nvfp4_onepass_kernel(const __nv_bfloat16* __restrict__ x, const FusedParams p, unsigned int* ws) {
+  __shared__ __align__(16) float Ts[16 * 16];
+  __shared__ float warp_max[kSmallRows / 32];
+  __shared__ float s_amax;
+  __shared__ int s_ok;
+  const int blk = static_cast<int>(blockIdx.x);
+  float y[16];
+  bool valid;
+  long long row;
+  small_transform<16, SHARED_T>(x, p, Ts, y, valid, row);
+
+  float m = group_absmax<16>(y);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if ((threadIdx.x & 31) == 0) warp_max[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float cm = warp_max[0];
+#pragma unroll
+    for (int w = 1; w < kSmallRows / 32; ++w) cm = fmaxf(cm, warp_max[w]);
+    const unsigned int total = gridDim.x * gridDim.y;
+    if (cm > 0.0f) atomicMax(&ws[0], __float_as_uint(cm));
+    __threadfence();
+    atomicAdd(&ws[1], 1u);
+    const uint64_t t0 = global_timer_ns();
+    int ok = 1;
+    while (atomicAdd(&ws[1], 0u) < total) {
+      __nanosleep(64);
+      if (global_timer_ns() - t0 > p.wait_limit_ns) {   // a CTA never arrived
+        atomicOr(&g_wush_device_error, 128u);
+        ok = 0;
+        break;
+      }
+    }
+    __threadfence();
+    s_amax = __uint_as_float(atomicAdd(&ws[0], 0u));
+    s_ok = ok;
+    if (ok && atomicAdd(&ws[2], 1u) == total - 1) {     // every CTA has read the maximum
+      ws[0] = 0u;
+      ws[1] = 0u;
+      ws[2] = 0u;
+      __threadfence();
+    }
+  }
+  __syncthreads();
+  if (!s_ok) return;
+  const float s_t = __fdiv_rn(s_amax, 2688.0f);
+  if (blk == 0 && blockIdx.y == 0 && threadIdx.x == 0) *const_cast<float*>(p.tensor_scale) = s_t;
+  if (!valid) return;
+  if (EMIT_Y) {
+    float4* yd = reinterpret_cast<float4*>(p.y_out + row * p.d_in + static_cast<long long>(blk) * 16);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) yd[k] = make_float4(y[4 * k], y[4 * k + 1], y[4 * k + 2], y[4 * k + 3]);
+  }
+  uint32_t words[2];
+  static_cast<uint8_t*>(p.scales)[row * p.C + blk] =
+      static_cast<uint8_t>(quant_nv<16>(y, s_t, __fmul_rn(6.0f, s_t), words));
+  *reinterpret_cast<uint2*>(p.codes + row * (p.d_in / 2) + static_cast<long long>(blk) * 8) =
+      make_uint2(words[0], words[1]);
 }
 
 }  // namespace wush

@@ -55,7 +55,8 @@
  *                          non-sm_100 device)
  * Bits of the device error word (wush_device_status): 1/2/4/8/16 a wait of the TMA
  * producer / MMA issuer / converter / epilogue / final drain expired, 32 the wait
- * self-test expired (expected), 64 a Cholesky pivot was not positive.
+ * self-test expired (expected), 64 a Cholesky pivot was not positive, 128 a CTA of the
+ * one-launch NVFP4 path waited in vain for the rest of its grid.
  * rows == 0 (with a supported fmt/G and a valid d_in) returns WUSH_OK without launching
  * anything; its pointers are then not checked and may be NULL.
  */
@@ -249,6 +250,25 @@ int wush_build_transforms(const float* w_f32, const void* xcal_bf16, int64_t d_o
  * WUSH_ERR_DEVICE_TIMEOUT (WUSH_ERR_CUDA if the runtime reports an error).  If
  * `bits` is not NULL it receives the raw word. */
 int wush_device_status(wush_stream_t stream, uint32_t* bits);
+
+/* NVFP4 activations of a decode-sized batch in ONE launch (the staged or single-call
+ * NVFP4 paths take three: amax pass, tensor scale, quantising pass).  The CTAs (one per
+ * 16-channel block and 128 rows, on CUDA cores as in wush_set_small_batch_rows) fold their
+ * max |y| into workspace[0], count themselves into workspace[1] and wait — bounded by the
+ * wait limit, error bit 128 on expiry — until the whole grid has arrived, then quantise
+ * with s_t = amax / 2688; the last CTA to leave returns the words to zero.  Outputs and
+ * layouts as wush_quant_act with fmt = NVFP4, G = 16 (codes and scales bit-identical to
+ * it whenever both take the CUDA-core path).
+ * workspace: device memory of at least 16 bytes, 16-byte aligned, ZERO before the first
+ * call; every call that completes without a device error leaves it zero again.  Calls
+ * that may overlap (other streams) need workspaces of their own.
+ * The grid (d_in/16 x ceil(n_tok/128) CTAs) must be resident on the device at once; it is
+ * launched cooperatively, and a larger batch returns WUSH_ERR_UNSUPPORTED (use
+ * wush_quant_act).  Other errors as wush_quant_act; the workspace must be 16-byte aligned.
+ * The pages have no counterpart: it is a latency path for small batches. */
+int wush_quant_act_nvfp4_onepass(const void* x_bf16, const float* T_blocks, int64_t n_tok,
+                                 int64_t d_in, uint8_t* codes, uint8_t* scales,
+                                 float* tensor_scale, uint32_t* workspace, wush_stream_t stream);
 
 /* Activation batches (bf16 input, row-major scales) of at most `rows` rows take a
  * CUDA-core path instead of the fused tensor-core kernel: one CTA per block and 128 rows,
