@@ -24,7 +24,7 @@ __all__ = ["FMT", "WushError", "wush_quant_act", "wush_quant_weight", "wush_quan
            "wush_quant_act_shared_mx_atoms", "wush_gemm_nvfp4", "wush_quant_act_nv_atoms",
            "wush_quant_weight_nv_atoms", "wush_quant_act_nvfp4_amax", "wush_nvfp4_scale_from_amax",
            "wush_quant_act_nvfp4_with_scale", "wush_set_small_batch_rows", "wush_quant_act_nvfp4_onepass",
-           "nvfp4_workspace"]
+           "nvfp4_workspace", "wush_quant_act_nvfp4_onepass_noalloc"]
 
 FMT = {"mxfp4": 0, "nvfp4": 1, "int4": 2}
 STATUS = {0: "WUSH_OK", 1: "WUSH_ERR_INVALID_ARG", 2: "WUSH_ERR_UNSUPPORTED", 3: "WUSH_ERR_MISALIGNED",
@@ -36,6 +36,7 @@ EXPORTED_SYMBOLS = ("wush_quant_act", "wush_quant_weight", "wush_quant_act_debug
                     "wush_gemm_nvfp4", "wush_quant_act_nv_atoms", "wush_quant_weight_nv_atoms",
                     "wush_quant_act_nvfp4_amax", "wush_nvfp4_scale_from_amax", "wush_quant_act_nvfp4_with_scale",
                     "wush_set_small_batch_rows", "wush_quant_act_nvfp4_onepass",
+                    "wush_quant_act_nvfp4_onepass_noalloc",
                     "wush_build_transforms", "wush_device_status",
                     "wush_set_wait_limit_ns",
                     "wush_selftest_wait_timeout", "wush_status_string", "wush_version")
@@ -98,6 +99,8 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
     lib.wush_device_status.restype = ctypes.c_int
     lib.wush_quant_act_nvfp4_onepass.argtypes = [_P, _P, _I64, _I64, _P, _P, _P, _P, _P]
     lib.wush_quant_act_nvfp4_onepass.restype = ctypes.c_int
+    lib.wush_quant_act_nvfp4_onepass_noalloc.argtypes = [_P, _P, _I64, _I64, _P, _P, _P, _P]
+    lib.wush_quant_act_nvfp4_onepass_noalloc.restype = ctypes.c_int
     lib.wush_set_small_batch_rows.argtypes = [_I64]
     lib.wush_set_small_batch_rows.restype = ctypes.c_int
     lib.wush_set_wait_limit_ns.argtypes = [_U64]
@@ -424,6 +427,30 @@ def wush_quant_act_nvfp4_onepass(x, T, workspace, codes=None, scales=None, tenso
                                               _ptr(workspace), _stream_handle(stream))
     if st != 0:
         raise WushError(st, "wush_quant_act_nvfp4_onepass")
+    return codes, scales, tensor_scale
+
+
+def wush_quant_act_nvfp4_onepass_noalloc(x, T, codes=None, scales=None, tensor_scale=None, stream=None):
+    """As wush_quant_act_nvfp4_onepass on the library's own static scratch (no workspace;
+    calls that may overlap race).  Returns (codes, scales, tensor_scale)."""
+    lib = load_library()
+    n, d = _nv_stage_input(x, T)
+    if codes is None:
+        codes = torch.empty((n, d // 2), dtype=torch.uint8, device=x.device)
+    if scales is None:
+        scales = torch.empty((n, d // 16), dtype=torch.uint8, device=x.device)
+    if tensor_scale is None:
+        tensor_scale = torch.empty(1, dtype=torch.float32, device=x.device)
+    for t, name, dt in ((codes, "codes", torch.uint8), (scales, "scales", torch.uint8),
+                        (tensor_scale, "tensor_scale", torch.float32)):
+        _check_dev(t, name, dt)
+    if tuple(codes.shape) != (n, d // 2) or tuple(scales.shape) != (n, d // 16):
+        raise ValueError("output buffers have the wrong size")
+    with torch.cuda.device(x.device):
+        st = lib.wush_quant_act_nvfp4_onepass_noalloc(_ptr(x), _ptr(T), n, d, _ptr(codes), _ptr(scales),
+                                                      _ptr(tensor_scale), _stream_handle(stream))
+    if st != 0:
+        raise WushError(st, "wush_quant_act_nvfp4_onepass_noalloc")
     return codes, scales, tensor_scale
 
 

@@ -30,6 +30,14 @@ __global__ void wush_selftest_wait_kernel(unsigned long long limit_ns) {
   __syncthreads();
   if (threadIdx.x == 0) wait_bounded(smem_addr(&bar), 0u, &abort_word, 32u, limit_ns);
 }
+// Scratch of wush_quant_act_nvfp4_onepass_noalloc: 256 bytes, of which the one-launch
+// NVFP4 kernel uses the first three words.  Zero at module load; every call that ends
+// without a device error leaves it zero.
+constexpr int kNoAllocScratchWords = 64;
+constexpr int kOnepassWorkspaceWords = 3;
+static __device__ __align__(256) unsigned int g_noalloc_scratch[kNoAllocScratchWords];
+static_assert(kOnepassWorkspaceWords <= kNoAllocScratchWords, "scratch too small for the one-launch workspace");
+
 }  // namespace wush
 
 #ifndef WUSH_USE_PDL
@@ -529,6 +537,27 @@ int wush_quant_act_nvfp4_onepass(const void* x_bf16, const float* T_blocks, int6
                          reinterpret_cast<unsigned int*>(workspace)) != cudaSuccess)
     return WUSH_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? WUSH_OK : WUSH_ERR_CUDA;
+}
+
+int wush_quant_act_nvfp4_onepass_noalloc(const void* x_bf16, const float* T_blocks, int64_t n_tok, int64_t d_in,
+                                         uint8_t* codes, uint8_t* scales, float* tensor_scale, wush_stream_t stream) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return WUSH_ERR_CUDA;
+  if (dev < 0 || dev >= 64) return WUSH_ERR_UNSUPPORTED;
+  static std::mutex mu;
+  static void* scratch[64] = {};
+  void* ws = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    if (!scratch[dev]) {   // once per device, with that device current
+      void* a = nullptr;
+      if (cudaGetSymbolAddress(&a, wush::g_noalloc_scratch) != cudaSuccess || !a) return WUSH_ERR_CUDA;
+      scratch[dev] = a;
+    }
+    ws = scratch[dev];
+  }
+  return wush_quant_act_nvfp4_onepass(x_bf16, T_blocks, n_tok, d_in, codes, scales, tensor_scale,
+                                      static_cast<uint32_t*>(ws), stream);
 }
 
 int wush_set_small_batch_rows(int64_t rows) {

@@ -270,6 +270,24 @@ int wush_quant_act_nvfp4_onepass(const void* x_bf16, const float* T_blocks, int6
                                  int64_t d_in, uint8_t* codes, uint8_t* scales,
                                  float* tensor_scale, uint32_t* workspace, wush_stream_t stream);
 
+/* The one-launch NVFP4 path without a caller workspace: it uses a 256-byte file-scope
+ * static device array of the library (3 words of it), whose address is taken once per
+ * device with cudaGetSymbolAddress; nothing is allocated.  The scratch is zero when the
+ * library is loaded and every call that completes without a device error leaves it zero;
+ * after a call that records error bit 128 it is not zero any more and this entry point
+ * must not be used again in the process (wush_quant_act_nvfp4_onepass with a fresh
+ * workspace still works).  All calls share the one scratch per device: calls that may
+ * overlap (several streams, several host threads) race and give wrong results — use
+ * wush_quant_act_nvfp4_onepass with a workspace each there.  Make the first call on each
+ * device before any stream capture (it resolves the scratch address).  Requests the
+ * one-launch path cannot take (a grid of d_in/16 x ceil(n_tok/128) CTAs that is not
+ * resident at once) return WUSH_ERR_UNSUPPORTED; a current device ordinal above 63 also
+ * returns WUSH_ERR_UNSUPPORTED; otherwise as wush_quant_act_nvfp4_onepass.
+ * The pages have no counterpart: it only spares the caller a workspace allocation. */
+int wush_quant_act_nvfp4_onepass_noalloc(const void* x_bf16, const float* T_blocks, int64_t n_tok,
+                                         int64_t d_in, uint8_t* codes, uint8_t* scales,
+                                         float* tensor_scale, wush_stream_t stream);
+
 /* Activation batches (bf16 input, row-major scales) of at most `rows` rows take a
  * CUDA-core path instead of the fused tensor-core kernel: one CTA per block and 128 rows,
  * T_i staged in shared memory, y = T_i x in fp32 FMAs, then the same group quantisers
