@@ -159,9 +159,15 @@ int dispatch(const CUtensorMap& map, const CUtensorMap& cmap, wush::FusedParams 
 }
 
 // Activation batches of at most this many rows take the CUDA-core path (wush_small.cuh);
-// 0 sends every batch to the fused tensor-core kernel.
-constexpr long long kDefaultSmallRows = 64;
-std::atomic<long long> g_small_rows{kDefaultSmallRows};
+// 0 sends every batch to the fused tensor-core kernel, -1 selects the per-format default
+// (measured crossovers at d_in = 4096: MXFP4 between 64 and 128 rows, INT4 and NVFP4
+// between 256 and 512).
+std::atomic<long long> g_small_rows{-1};
+long long small_rows_limit(int fmt) {
+  const long long v = g_small_rows.load(std::memory_order_relaxed);
+  if (v >= 0) return v;
+  return fmt == WUSH_MXFP4 ? 64 : 256;
+}
 
 template <int G, int FMT, bool AMAX_ONLY, bool SHARED>
 int launch_small(const void* x, const wush::FusedParams& p, bool emit_y, cudaStream_t s) {
@@ -220,8 +226,10 @@ int quant_common(const void* in, bool in_f32, const float* T, int64_t rows, int6
   if (tensor_scale && !aligned(tensor_scale, 4)) return WUSH_ERR_MISALIGNED;
   if (debug && !aligned(y_out, 16)) return WUSH_ERR_MISALIGNED;
 
-  if (!in_f32 && !scale_atoms && rows <= g_small_rows.load(std::memory_order_relaxed)) {
+  if (!in_f32 && rows <= small_rows_limit(fmt)) {
     wush::FusedParams p{};
+    p.scale_atoms = scale_atoms ? 1 : 0;
+    p.atom_cols = static_cast<int>((d_in / G + 3) / 4);
     p.T = T;
     p.codes = codes;
     p.scales = scales;
@@ -561,7 +569,7 @@ int wush_quant_act_nvfp4_onepass_noalloc(const void* x_bf16, const float* T_bloc
 }
 
 int wush_set_small_batch_rows(int64_t rows) {
-  if (rows < 0) rows = kDefaultSmallRows;
+  if (rows < 0) rows = -1;
   if (rows > (1 << 20)) return WUSH_ERR_INVALID_ARG;
   g_small_rows.store(rows, std::memory_order_relaxed);
   return WUSH_OK;

@@ -79,12 +79,19 @@ __global__ void __launch_bounds__(kSmallRows)
   }
   uint32_t words[G / 8];
   uint8_t* cdst = p.codes + row * (p.d_in / 2) + static_cast<long long>(blk) * (G / 2);
+  // one-byte scales go row-major or, for the block-scaled GEMM, to the scale-atom layout:
+  // row 128 r + i + 32 j, column 4 c + k at byte (r * atom_cols + c) * 512 + 16 i + 4 j + k
+  uint8_t* sdst = static_cast<uint8_t*>(p.scales) + row * p.C + blk;
+  if (FMT != kINT4 && p.scale_atoms) {
+    const int rr = static_cast<int>(row & 127);
+    sdst = static_cast<uint8_t*>(p.scales) + ((row >> 7) * p.atom_cols + (blk >> 2)) * 512 + (rr & 31) * 16 +
+           (rr >> 5) * 4 + (blk & 3);
+  }
   if constexpr (FMT == kMXFP4) {
-    static_cast<uint8_t*>(p.scales)[row * p.C + blk] = static_cast<uint8_t>(quant_mx<G>(y, words));
+    *sdst = static_cast<uint8_t>(quant_mx<G>(y, words));
   } else if constexpr (FMT == kNVFP4) {
     const float s_t = *p.tensor_scale;
-    static_cast<uint8_t*>(p.scales)[row * p.C + blk] =
-        static_cast<uint8_t>(quant_nv<G>(y, s_t, __fmul_rn(6.0f, s_t), words));
+    *sdst = static_cast<uint8_t>(quant_nv<G>(y, s_t, __fmul_rn(6.0f, s_t), words));
   } else {
     static_cast<float*>(p.scales)[row * p.C + blk] = quant_int4<G>(y, words);
   }

@@ -288,14 +288,16 @@ int wush_quant_act_nvfp4_onepass_noalloc(const void* x_bf16, const float* T_bloc
                                          int64_t d_in, uint8_t* codes, uint8_t* scales,
                                          float* tensor_scale, wush_stream_t stream);
 
-/* Activation batches (bf16 input, row-major scales) of at most `rows` rows take a
+/* Activation batches (bf16 input; row-major scales or the scale-atom layout) of at most
+ * `rows` rows take a
  * CUDA-core path instead of the fused tensor-core kernel: one CTA per block and 128 rows,
  * T_i staged in shared memory, y = T_i x in fp32 FMAs, then the same group quantisers
  * (codes, scales and NVFP4 tensor scale in the same layouts; y differs from the tensor-core
  * path's by fp32 rounding only).  At decode sizes the fused kernel's fixed start-up
  * latency dominates.  rows = 0 sends every batch to the fused kernel; rows < 0 restores
- * the default (64).  Applies to later calls on every device; returns WUSH_OK, or
- * WUSH_ERR_INVALID_ARG above 2^20 rows. */
+ * the default, which depends on the format (MXFP4 64 rows, INT4 and NVFP4 256: the
+ * measured crossovers at d_in = 4096); rows > 0 applies to every format.  Applies to later
+ * calls on every device; returns WUSH_OK, or WUSH_ERR_INVALID_ARG above 2^20 rows. */
 int wush_set_small_batch_rows(int64_t rows);
 
 /* Sets the bound of every in-kernel wait for later launches, in nanoseconds

@@ -17,6 +17,15 @@ from blockwise_adaptive_transforms_b200 import sharded
 pytestmark = pytest.mark.gpu
 
 
+@pytest.fixture(autouse=True)
+def _fused_path():
+    # shards and the whole batch must take the same path (the CUDA-core path for small
+    # batches rounds y differently); its own stage test is in test_gpu_small.py
+    W.wush_set_small_batch_rows(0)
+    yield
+    W.wush_set_small_batch_rows(-1)
+
+
 def _layer(n_tok, d_in):
     wl = workload("mlp_down_nvfp4_14336", n_tok=n_tok, d_in=d_in, d_out=256, n_cal=512)
     inp = make_inputs(wl)

@@ -1,6 +1,6 @@
 """The CUDA-core path for decode-sized activation batches vs the fp64 oracle (needs a B200).
 
-Batches of at most `wush_set_small_batch_rows` rows (default 64) skip the fused
+Batches of at most `wush_set_small_batch_rows` rows (default 64 MXFP4, 256 otherwise) skip the fused
 tensor-core kernel.  Each case checks rule 1 (the oracle's quantiser on the kernel's own
 fp32 y gives the kernel's codes and scales bit for bit), that y is the fp32-FMA transform
 (within G * 2^-23 of |T_i||x| of the float64 product), rule 2 end to end, and the same
@@ -99,3 +99,22 @@ def test_nvfp4_stages_take_the_small_path_too():
 def test_threshold_setter_rejects_huge_values():
     with pytest.raises(W.WushError):
         W.wush_set_small_batch_rows(1 << 21)
+
+
+@pytest.mark.parametrize("fmt,n_tok,d_in", [("mxfp4", 40, 1056), ("nvfp4", 200, 1040)])
+def test_small_batches_write_scale_atoms(fmt, n_tok, d_in):
+    """The scale-atom quantisers take the same path as the row-major ones for the same
+    batch: same codes, and the atoms hold the row-major scales in the atom layout."""
+    G = 32 if fmt == "mxfp4" else 16
+    name = "attn_mxfp4_4096" if fmt == "mxfp4" else "mlp_down_nvfp4_14336"
+    inp, b, x, T = _data(name, fmt, G, d_in, n_tok)
+    c, s, ts = W.wush_quant_act(x, T, G, fmt)
+    if fmt == "mxfp4":
+        ca, at = W.wush_quant_act_mx_atoms(x, T)
+    else:
+        ca, at, tsa = W.wush_quant_act_nv_atoms(x, T)
+    torch.cuda.synchronize()
+    assert torch.equal(c, ca)
+    if fmt == "nvfp4":
+        assert torch.equal(ts, tsa)
+    assert np.array_equal(at.cpu().numpy(), O.scale_atoms(s.cpu().numpy()))
