@@ -19,6 +19,7 @@ from __future__ import annotations
 import argparse
 import hashlib
 import json
+import re
 import os
 import statistics
 import sys
@@ -75,11 +76,19 @@ def job_throughput(world: int, steps: int, bytes_per_step: int, elapsed_s: float
     return world * steps * bytes_per_step / elapsed_s / 1e9
 
 
+def _code_only(text: str) -> str:
+    """The source without comments and blank lines: what the compiled kernel depends on."""
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    return "\n".join(line.rstrip() for line in text.splitlines() if line.strip())
+
+
 def kernel_source_hash() -> str:
+    """SHA-256 (16 hex digits) of the fused kernel's sources, comments excluded."""
     h = hashlib.sha256()
     for rel in KERNEL_SOURCES:
-        with open(os.path.join(ROOT, rel), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, rel), encoding="utf-8") as f:
+            h.update(_code_only(f.read()).encode())
     return h.hexdigest()[:16]
 
 

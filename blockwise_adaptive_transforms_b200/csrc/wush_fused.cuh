@@ -12,15 +12,18 @@
 //  * warp 0 streams the input tiles with TMA (128-byte swizzle) through a STAGES-deep
 //    mbarrier ring and bulk-copies each column tile's fp32 matrices into a transform
 //    slot; warps 2-3 split them in place into bf16 hi and lo, stacked along N (for fp32
-//    weights they also split each staged weight tile into bf16 hi + lo operands);
+//    weights warps 2-3 and 8-11 also split each staged weight tile into bf16 hi + lo
+//    operands);
 //  * warp 1 issues tcgen05.mma (M=128, N=2G, K=16) into fp32 TMEM accumulators,
 //    double-buffered: one MMA per block and K-step yields X*T_hi^T and X*T_lo^T side
 //    by side (fp32 weights add W_lo*T_hi^T into the first half; the dropped W_lo*T_lo
 //    term is below 2^-16 relative).  Each tcgen05.mma costs the issuing thread ~50
 //    cycles whatever N is, so stacking hi|lo halves the issue work of the tile;
-//  * warps 4-11 read the accumulators with tcgen05.ld (one token row per thread),
-//    add the hi and lo halves, compute the AbsMax scale, round and pack, stage the
-//    tile's codes in shared memory for one TMA store and write one scale word per row.
+//  * two epilogue groups (warps 4-7 and 8-11; one group, warps 4-7, for fp32 weights)
+//    take alternate tiles: they read the accumulators with tcgen05.ld (one token row
+//    per thread, 64 columns per load), add the hi and lo halves, compute the AbsMax
+//    scale, round and pack, stage the tile's codes in shared memory for one TMA store and
+//    write the row's scales (row-major, or in the block-scaled MMA's scale-atom layout).
 //  * every wait is an mbarrier try_wait with a suspend-time hint, so waiting warps do
 //    not take issue slots from the working ones.
 #pragma once
