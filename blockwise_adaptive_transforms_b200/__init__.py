@@ -24,7 +24,7 @@ __all__ = ["FMT", "WushError", "wush_quant_act", "wush_quant_weight", "wush_quan
            "wush_quant_act_shared_mx_atoms", "wush_gemm_nvfp4", "wush_quant_act_nv_atoms",
            "wush_quant_weight_nv_atoms", "wush_quant_act_nvfp4_amax", "wush_nvfp4_scale_from_amax",
            "wush_quant_act_nvfp4_with_scale", "wush_set_small_batch_rows", "wush_quant_act_nvfp4_onepass",
-           "nvfp4_workspace", "wush_quant_act_nvfp4_onepass_noalloc"]
+           "nvfp4_workspace", "wush_quant_act_nvfp4_onepass_noalloc", "wush_set_gemm_cta_pairs"]
 
 FMT = {"mxfp4": 0, "nvfp4": 1, "int4": 2}
 STATUS = {0: "WUSH_OK", 1: "WUSH_ERR_INVALID_ARG", 2: "WUSH_ERR_UNSUPPORTED", 3: "WUSH_ERR_MISALIGNED",
@@ -36,7 +36,7 @@ EXPORTED_SYMBOLS = ("wush_quant_act", "wush_quant_weight", "wush_quant_act_debug
                     "wush_gemm_nvfp4", "wush_quant_act_nv_atoms", "wush_quant_weight_nv_atoms",
                     "wush_quant_act_nvfp4_amax", "wush_nvfp4_scale_from_amax", "wush_quant_act_nvfp4_with_scale",
                     "wush_set_small_batch_rows", "wush_quant_act_nvfp4_onepass",
-                    "wush_quant_act_nvfp4_onepass_noalloc",
+                    "wush_quant_act_nvfp4_onepass_noalloc", "wush_set_gemm_cta_pairs",
                     "wush_build_transforms", "wush_device_status",
                     "wush_set_wait_limit_ns",
                     "wush_selftest_wait_timeout", "wush_status_string", "wush_version")
@@ -101,6 +101,8 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
     lib.wush_quant_act_nvfp4_onepass.restype = ctypes.c_int
     lib.wush_quant_act_nvfp4_onepass_noalloc.argtypes = [_P, _P, _I64, _I64, _P, _P, _P, _P]
     lib.wush_quant_act_nvfp4_onepass_noalloc.restype = ctypes.c_int
+    lib.wush_set_gemm_cta_pairs.argtypes = [_I32]
+    lib.wush_set_gemm_cta_pairs.restype = ctypes.c_int
     lib.wush_set_small_batch_rows.argtypes = [_I64]
     lib.wush_set_small_batch_rows.restype = ctypes.c_int
     lib.wush_set_wait_limit_ns.argtypes = [_U64]
@@ -548,6 +550,11 @@ def wush_device_status(stream=None):
     bits = ctypes.c_uint32(0)
     st = load_library().wush_device_status(_stream_handle(stream), ctypes.byref(bits))
     return int(st), int(bits.value)
+
+
+def wush_set_gemm_cta_pairs(enable: bool) -> None:
+    """FP4 GEMMs with M % 256 == 0 on CTA pairs, or (default) always on single CTAs."""
+    load_library().wush_set_gemm_cta_pairs(1 if enable else 0)
 
 
 def wush_set_small_batch_rows(rows: int) -> None:

@@ -77,6 +77,20 @@ int encode_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dt, int el
   return r == CUDA_SUCCESS ? WUSH_OK : WUSH_ERR_CUDA;
 }
 
+// 2-D row-major uint8 [rows][cols] tensor, box {box_cols, box_rows}, no swizzle.
+int encode_u8_plain(CUtensorMap* map, const void* base, int64_t rows, int64_t cols, int box_cols, int box_rows) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return WUSH_ERR_CUDA;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols)};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t estr[2] = {1u, 1u};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? WUSH_OK : WUSH_ERR_CUDA;
+}
+
 // 2-D row-major uint8 [rows][cols] tensor, box {box_cols, box_rows}, 128-byte swizzle.
 int encode_u8_sw128(CUtensorMap* map, const void* base, int64_t rows, int64_t cols, int box_cols, int box_rows) {
   auto enc = tensor_map_encoder();
@@ -378,6 +392,72 @@ int wush_mx_scales_to_atoms(const uint8_t* scales, int64_t rows, int64_t C, uint
 
 namespace {
 
+// Opt-in (wush_set_gemm_cta_pairs): for M a multiple of 256, pairs of CTAs share M = 256
+// MMAs (wush_gemm_fp4_pair_kernel).  Off by default: on B200 it measured 4-11 % slower
+// than single CTAs at the benchmarked shapes.
+std::atomic<int> g_gemm_pairs{0};
+
+template <bool NV>
+int gemm_fp4_pair(const uint8_t* a_codes, const uint8_t* a_atoms, const float* a_ts, const uint8_t* b_codes,
+                  const uint8_t* b_atoms, const float* b_ts, int64_t M, int64_t N, int64_t K, void* d_bf16,
+                  wush_stream_t stream) {
+  using Cfg = wush::GemmPairCfg<NV>;
+  CUtensorMap ma, mb, msa, msb;
+  int st = encode_u8_sw128(&ma, a_codes, M, K / 2, 128, Cfg::BM);
+  if (st != WUSH_OK) return st;
+  st = encode_u8_sw128(&mb, b_codes, N, K / 2, 128, Cfg::BN / 2);
+  if (st != WUSH_OK) return st;
+  // scale atoms as rows of 128 bytes: a stage's atoms of one 128-row block are 4 * APS rows
+  const long long c_pad = (K / Cfg::VS + 3) / 4 * 4;
+  st = encode_u8_plain(&msa, a_atoms, M * c_pad / 128, 128, 128, 4 * Cfg::ATOMS_PER_STAGE);
+  if (st != WUSH_OK) return st;
+  st = encode_u8_plain(&msb, b_atoms, N * c_pad / 128, 128, 128, 4 * Cfg::ATOMS_PER_STAGE);
+  if (st != WUSH_OK) return st;
+  wush::GemmParams p{};
+  p.sfa = a_atoms;
+  p.sfb = b_atoms;
+  p.ts_a = a_ts;
+  p.ts_b = b_ts;
+  p.d = static_cast<__nv_bfloat16*>(d_bf16);
+  p.M = static_cast<int>(M);
+  p.N = static_cast<int>(N);
+  p.K = static_cast<int>(K);
+  p.tiles_m = static_cast<int>(M / Cfg::PAIR_M);
+  p.tiles_n = static_cast<int>(N / Cfg::BN);
+  p.wait_limit_ns = g_wait_limit_ns.load(std::memory_order_relaxed);
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return WUSH_ERR_CUDA;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return WUSH_ERR_CUDA;
+  static std::atomic<unsigned long long> configured{0ull};
+  const unsigned long long bit = 1ull << (dev & 63);
+  if (!(configured.load(std::memory_order_acquire) & bit)) {
+    if (cudaFuncSetAttribute(wush::wush_gemm_fp4_pair_kernel<Cfg>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             Cfg::SMEM_BYTES) != cudaSuccess)
+      return WUSH_ERR_CUDA;
+    configured.fetch_or(bit, std::memory_order_acq_rel);
+  }
+  const long long tiles = static_cast<long long>(p.tiles_m) * p.tiles_n;
+  if (tiles > INT_MAX / 2) return WUSH_ERR_INVALID_ARG;
+  const long long pairs = tiles < sms / 2 ? tiles : sms / 2;
+  cudaLaunchConfig_t lc = {};
+  lc.gridDim = dim3(static_cast<unsigned>(2 * pairs));
+  lc.blockDim = dim3(Cfg::THREADS);
+  lc.dynamicSmemBytes = Cfg::SMEM_BYTES;
+  lc.stream = reinterpret_cast<cudaStream_t>(stream);
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  lc.attrs = attr;
+  lc.numAttrs = WUSH_USE_PDL ? 2 : 1;
+  if (cudaLaunchKernelEx(&lc, wush::wush_gemm_fp4_pair_kernel<Cfg>, ma, mb, msa, msb, p) != cudaSuccess)
+    return WUSH_ERR_CUDA;
+  return cudaGetLastError() == cudaSuccess ? WUSH_OK : WUSH_ERR_CUDA;
+}
+
 // One launch of the block-scaled FP4 GEMM (MXFP4 or NVFP4 operands).
 template <bool NV>
 int gemm_fp4(const uint8_t* a_codes, const uint8_t* a_atoms, const float* a_ts, const uint8_t* b_codes,
@@ -394,6 +474,8 @@ int gemm_fp4(const uint8_t* a_codes, const uint8_t* a_atoms, const float* a_ts, 
       !aligned(d_bf16, 16))
     return WUSH_ERR_MISALIGNED;
   if (NV && (!aligned(a_ts, 4) || !aligned(b_ts, 4))) return WUSH_ERR_MISALIGNED;
+  if (M % 256 == 0 && g_gemm_pairs.load(std::memory_order_relaxed))
+    return gemm_fp4_pair<NV>(a_codes, a_atoms, a_ts, b_codes, b_atoms, b_ts, M, N, K, d_bf16, stream);
   CUtensorMap ma, mb;
   int st = encode_u8_sw128(&ma, a_codes, M, K / 2, 128, Cfg::BM);
   if (st != WUSH_OK) return st;
@@ -566,6 +648,11 @@ int wush_quant_act_nvfp4_onepass_noalloc(const void* x_bf16, const float* T_bloc
   }
   return wush_quant_act_nvfp4_onepass(x_bf16, T_blocks, n_tok, d_in, codes, scales, tensor_scale,
                                       static_cast<uint32_t*>(ws), stream);
+}
+
+int wush_set_gemm_cta_pairs(int enable) {
+  g_gemm_pairs.store(enable ? 1 : 0, std::memory_order_relaxed);
+  return WUSH_OK;
 }
 
 int wush_set_small_batch_rows(int64_t rows) {

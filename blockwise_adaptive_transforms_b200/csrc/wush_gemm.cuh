@@ -287,6 +287,284 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
   }
 }
 
+// ---------------------------------------------------------------- CTA-pair variant
+// The same GEMM on pairs of CTAs (a cluster of two on two SMs) sharing one M = 256 MMA:
+// CTA v of the pair holds rows [128 v, 128 v + 128) of the pair's A tile and rows
+// [128 v, 128 v + 128) of its 256-row B tile (B split along N), plus its rows' A scale
+// atoms and the whole B tile's scale atoms; its TMEM accumulator holds its 128 rows x all
+// 256 columns.  Each SM thus streams 32 KB of operands per 256-K stage instead of 48 KB
+// for the same multiply-adds, which is what bounds the one-CTA kernel (operand bytes in
+// flight per SM against L2 latency).  Both CTAs' TMA loads complete on the even CTA's
+// full barrier; only the even CTA waits on it, copies the scale atoms into both CTAs'
+// TMEM and issues the MMAs; its commits reach both CTAs' barriers; the odd CTA's
+// epilogue warps arrive on the even CTA's accumulator-empty barrier.  No load is
+// multicast.
+template <bool NV_>
+struct GemmPairCfg {
+  static constexpr bool NV = NV_;
+  static constexpr int VS = NV ? 16 : 32;
+  static constexpr int BM = 128, BN = 256, BK = 256;   // per CTA: 128 rows, all 256 columns
+  static constexpr int PAIR_M = 2 * BM;
+  static constexpr int ATOM_K = 4 * VS;
+  static constexpr int ATOMS_PER_STAGE = BK / ATOM_K;  // MX 2, NV 4
+  static constexpr int STAGES = NV ? 5 : 6;
+  static constexpr int A_BYTES = BM * BK / 2;          // 16 KB
+  static constexpr int B_BYTES = (BN / 2) * BK / 2;    // 16 KB: this CTA's half of B
+  static constexpr int SFA_BYTES = ATOMS_PER_STAGE * 512;
+  static constexpr int SFB_BYTES = 2 * ATOMS_PER_STAGE * 512;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
+  static constexpr int OFF_A = 0, OFF_B = A_BYTES, OFF_SFA = A_BYTES + B_BYTES, OFF_SFB = OFF_SFA + SFA_BYTES;
+  static constexpr int OFF_BAR = STAGES * STAGE_BYTES;
+  static constexpr int N_BARS = 2 * STAGES + 3;        // full[S], empty[S], afull, aempty, drain
+  static constexpr int OFF_MISC = OFF_BAR + 8 * N_BARS;
+  static constexpr int SMEM_BYTES = OFF_MISC + 64 + 1024;
+  static constexpr int THREADS = 8 * 32;               // producer, MMA, 2 idle, 4 epilogue warps
+  static constexpr int TMEM_COLS = 512;
+  static constexpr int SF_COL0 = 256, SFB_COL = 4 * ATOMS_PER_STAGE, SF_SLOT_COLS = 12 * ATOMS_PER_STAGE;
+  static_assert(STAGE_BYTES % 1024 == 0, "stage alignment");
+  static_assert(SF_COL0 + STAGES * SF_SLOT_COLS <= TMEM_COLS, "TMEM columns");
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+};
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// shared::cluster address of the same shared-memory location in CTA `rank` of the cluster
+__device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+// TMA 2-D load into this CTA's shared memory whose bytes complete on a barrier of either
+// CTA of the pair (given as a shared::cluster address)
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* map, uint32_t bar_cluster,
+                                                 int32_t x, int32_t y, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster), "r"(x), "r"(y), "l"(policy)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem), "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish_pair() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+// 32 lanes x 128 bits from each CTA's shared memory into the same TMEM address of each CTA
+__device__ __forceinline__ void tmem_cp_pair_32x128b_x4(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+__device__ __forceinline__ void umma_pair_fp4(bool nv, uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                              uint32_t idesc, uint32_t sfa_tmem, uint32_t sfb_tmem,
+                                              uint32_t accumulate) {
+  if (nv)
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(
+            d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+        : "memory");
+  else
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(
+            d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+        : "memory");
+}
+// completion of this thread's earlier tcgen05 operations arrives once on the barrier at
+// the same shared-memory offset in both CTAs of the pair
+__device__ __forceinline__ void umma_commit_pair(uint32_t bar) {
+  const uint16_t mask = 3;
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(bar),
+      "h"(mask)
+      : "memory");
+}
+
+template <class Cfg>
+__global__ void __launch_bounds__(Cfg::THREADS, 1)
+    wush_gemm_fp4_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
+                              const __grid_constant__ CUtensorMap tmap_sfa,
+                              const __grid_constant__ CUtensorMap tmap_sfb, const GemmParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_addr(smem);
+  const uint32_t bar0 = sbase + Cfg::OFF_BAR;
+  auto BAR = [&](int i) -> uint32_t { return bar0 + 8u * static_cast<uint32_t>(i); };
+  constexpr int STAGES = Cfg::STAGES;
+  constexpr uint32_t APS = Cfg::ATOMS_PER_STAGE;
+  const int B_FULL = 0, B_EMPTY = STAGES, B_AFULL = 2 * STAGES, B_AEMPTY = 2 * STAGES + 1, B_DRAIN = 2 * STAGES + 2;
+  volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + Cfg::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::OFF_MISC + 4);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();           // 0: issues the MMAs, 1: its partner
+  const int pair = static_cast<int>(blockIdx.x >> 1), n_pairs = static_cast<int>(gridDim.x >> 1);
+  const uint64_t lim = p.wait_limit_ns;
+  const int n_tiles = p.tiles_m * p.tiles_n;         // pair tiles of 256 x 256
+  const int k_stages = p.K / Cfg::BK;
+  const int k_chunks = p.K / Cfg::ATOM_K;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(BAR(B_FULL + s), 1);
+      mbar_init(BAR(B_EMPTY + s), 1);
+    }
+    mbar_init(BAR(B_AFULL), 1);
+    mbar_init(BAR(B_AEMPTY), 2 * 4);                 // four epilogue warps in each CTA
+    mbar_init(BAR(B_DRAIN), 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+    tma_prefetch_desc(&tmap_a);
+    tma_prefetch_desc(&tmap_b);
+    tma_prefetch_desc(&tmap_sfa);
+    tma_prefetch_desc(&tmap_sfb);
+  }
+  grid_dependency_wait();
+  grid_launch_dependents();
+  if (warp == 1) {                                    // the same warp of both CTAs
+    tmem_alloc_pair(smem_addr(const_cast<uint32_t*>(tmem_slot)), Cfg::TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync_all();                                 // both CTAs' barriers exist before any remote use
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer (both CTAs)
+    if (lane == 0) {
+      const uint64_t pol = l2_policy_evict_first();
+      int stage = 0;
+      uint32_t phase = 0;
+      for (int tile = pair; tile < n_tiles && !*abort_flag; tile += n_pairs) {
+        const int tm = tile % p.tiles_m, tn = tile / p.tiles_m;
+        const int a_row = tm * Cfg::PAIR_M + static_cast<int>(rank) * Cfg::BM;
+        const int b_row = tn * Cfg::BN + static_cast<int>(rank) * (Cfg::BN / 2);
+        const int a_blk = tm * 2 + static_cast<int>(rank);     // this CTA's 128-row scale block
+        for (int ks = 0; ks < k_stages; ++ks) {
+          if (!wait_bounded(BAR(B_EMPTY + stage), phase ^ 1u, abort_flag, 1u, lim)) break;
+          const uint32_t dst = sbase + stage * Cfg::STAGE_BYTES;
+          const uint32_t fb = mapa_shared(BAR(B_FULL + stage), 0);   // the even CTA's full barrier
+          if (rank == 0) mbar_arrive_expect_tx(BAR(B_FULL + stage), 2u * Cfg::STAGE_BYTES);
+          tma_load_2d_pair(dst + Cfg::OFF_A, &tmap_a, fb, ks * 128, a_row, 0ull);
+          tma_load_2d_pair(dst + Cfg::OFF_B, &tmap_b, fb, ks * 128, b_row, pol);
+          // scale atoms as 128-byte rows: APS atoms of this CTA's A block, APS of each B half
+          tma_load_2d_pair(dst + Cfg::OFF_SFA, &tmap_sfa, fb, 0,
+                           static_cast<int>((a_blk * k_chunks + APS * ks) * 4), 0ull);
+          for (int h = 0; h < 2; ++h)
+            tma_load_2d_pair(dst + Cfg::OFF_SFB + h * APS * 512, &tmap_sfb, fb, 0,
+                             static_cast<int>(((2 * tn + h) * k_chunks + APS * ks) * 4), 0ull);
+          if (++stage == STAGES) stage = 0, phase ^= 1u;
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer (even CTA)
+    if (lane == 0 && rank == 0) {
+      int stage = 0, it = 0;
+      uint32_t phase = 0;
+      for (int tile = pair; tile < n_tiles; tile += n_pairs, ++it) {
+        if (!wait_bounded(BAR(B_AEMPTY), static_cast<uint32_t>((it & 1) ^ 1), abort_flag, 2u, lim)) break;
+        tc_fence_after();
+        bool ok = true;
+        for (int ks = 0; ks < k_stages; ++ks) {
+          if (!wait_bounded(BAR(B_FULL + stage), phase, abort_flag, 2u, lim)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t st = sbase + stage * Cfg::STAGE_BYTES;
+          const uint32_t sf_cols = tmem_base + static_cast<uint32_t>(Cfg::SF_COL0 + stage * Cfg::SF_SLOT_COLS);
+#pragma unroll
+          for (int a = 0; a < Cfg::ATOMS_PER_STAGE; ++a) {
+            tmem_cp_pair_32x128b_x4(sf_cols + 4 * a, desc_sf_atom(st + Cfg::OFF_SFA + a * 512));
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+              tmem_cp_pair_32x128b_x4(sf_cols + Cfg::SFB_COL + 8 * a + 4 * h,
+                                      desc_sf_atom(st + Cfg::OFF_SFB + h * Cfg::ATOMS_PER_STAGE * 512 + a * 512));
+          }
+          const uint64_t da = desc_k_sw128(st + Cfg::OFF_A);
+          const uint64_t db = desc_k_sw128(st + Cfg::OFF_B);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int a = Cfg::NV ? j : (j >> 1);
+            const uint32_t sub = Cfg::NV ? 0u : static_cast<uint32_t>(2 * (j & 1));
+            const uint32_t sfa = (sf_cols + 4 * a) | (sub << 30);
+            const uint32_t sfb = (sf_cols + Cfg::SFB_COL + 8 * a) | (sub << 30);
+            umma_pair_fp4(Cfg::NV, tmem_base, da + ((j * 32) >> 4), db + ((j * 32) >> 4),
+                          idesc_mxf4(Cfg::PAIR_M, Cfg::BN, sub, !Cfg::NV), sfa, sfb, (ks > 0 || j > 0) ? 1u : 0u);
+          }
+          umma_commit_pair(BAR(B_EMPTY + stage));
+          if (++stage == STAGES) stage = 0, phase ^= 1u;
+        }
+        if (!ok) break;
+        umma_commit_pair(BAR(B_AFULL));
+      }
+      umma_commit_pair(BAR(B_DRAIN));
+    }
+    if (lane == 0) {   // both CTAs: every MMA writing this CTA's TMEM has finished
+      volatile int no_abort = 0;
+      wait_bounded(BAR(B_DRAIN), 0u, &no_abort, 16u, lim);
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ epilogue (4 warps, both CTAs)
+    const int quad = warp & 3;
+    const int row_in_tile = quad * 32 + lane;
+    const float alpha = Cfg::NV ? __fmul_rn(*p.ts_a, *p.ts_b) : 1.0f;
+    const uint32_t aempty_leader = mapa_shared(BAR(B_AEMPTY), 0);
+    int it = 0;
+    bool live = true;
+    for (int tile = pair; tile < n_tiles; tile += n_pairs, ++it) {
+      const int tm = tile % p.tiles_m, tn = tile / p.tiles_m;
+      if (live && !wait_bounded(BAR(B_AFULL), static_cast<uint32_t>(it & 1), abort_flag, 8u, lim)) live = false;
+      const bool warp_live = __all_sync(0xffffffffu, live) && !*abort_flag;
+      if (warp_live) tc_fence_after();
+      const long long row = static_cast<long long>(tm) * Cfg::PAIR_M + rank * Cfg::BM + row_in_tile;
+      __nv_bfloat16* drow = p.d + row * p.N + static_cast<long long>(tn) * Cfg::BN;
+#pragma unroll 1
+      for (int ch = 0; ch < Cfg::BN / 32; ++ch) {
+        float v[32];
+        if (warp_live) tmem_ld32_sync(tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(32 * ch), v);
+        if (!warp_live) continue;
+        uint32_t packed[16];
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+          const __nv_bfloat162 b2 = Cfg::NV ? __floats2bfloat162_rn(v[2 * k] * alpha, v[2 * k + 1] * alpha)
+                                            : __floats2bfloat162_rn(v[2 * k], v[2 * k + 1]);
+          packed[k] = *reinterpret_cast<const uint32_t*>(&b2);
+        }
+        uint4* dst = reinterpret_cast<uint4*>(drow + 32 * ch);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) dst[k] = make_uint4(packed[4 * k], packed[4 * k + 1], packed[4 * k + 2], packed[4 * k + 3]);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(aempty_leader);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();                                 // no remote arrive or commit is still on its way
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, Cfg::TMEM_COLS);
+  }
+}
+
 // Row-major one-byte scales [rows][C] -> tcgen05 scale atoms (rows padded to a multiple
 // of 128 with zero bytes, C to a multiple of 4).
 __global__ void wush_scales_to_atoms_kernel(const uint8_t* __restrict__ src, long long rows, int C,

@@ -251,6 +251,13 @@ int wush_build_transforms(const float* w_f32, const void* xcal_bf16, int64_t d_o
  * `bits` is not NULL it receives the raw word. */
 int wush_device_status(wush_stream_t stream, uint32_t* bits);
 
+/* enable != 0: the FP4 GEMMs with M % 256 == 0 run on pairs of CTAs (clusters of two SMs
+ * sharing M = 256 block-scaled MMAs, B split between them along N); enable = 0 (the
+ * default) keeps every call on single CTAs, which measured faster on B200 at the
+ * benchmarked shapes.  Same results either way up to the order of fp32 accumulation.
+ * Applies to later calls; returns WUSH_OK. */
+int wush_set_gemm_cta_pairs(int enable);
+
 /* NVFP4 activations of a decode-sized batch in ONE launch (the staged or single-call
  * NVFP4 paths take three: amax pass, tensor scale, quantising pass).  The CTAs (one per
  * 16-channel block and 128 rows, on CUDA cores as in wush_set_small_batch_rows) fold their

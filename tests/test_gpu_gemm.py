@@ -232,3 +232,37 @@ def test_gemm_at_the_benchmarked_shape(fmt):
     got = d.float().cpu().numpy()[mi, ni].astype(np.float64)
     bound = 2.0 ** -8 * np.abs(ref) + (K + 2) * 2.0 ** -23 * mag + 1e-30
     assert np.all(np.abs(got - ref) <= bound), np.max(np.abs(got - ref) / bound)
+
+
+@pytest.mark.parametrize("nv", [False, True])
+@pytest.mark.parametrize("M,N,K", [(256, 256, 256), (512, 768, 1024), (1024, 512, 4096)])
+def test_cta_pair_kernel_equals_the_oracle_and_the_single_cta_kernel(M, N, K, nv):
+    """The opt-in CTA-pair GEMM (M % 256 == 0): within the oracle bound, and equal to the
+    single-CTA kernel up to fp32 accumulation order (both checked against the bound)."""
+    if nv:
+        a_c, a_s = random_nv_operand(M, K, 5)
+        b_c, b_s = random_nv_operand(N, K, 6)
+        ta = torch.tensor([0.5], dtype=torch.float32, device="cuda")
+        tb = torch.tensor([1.25], dtype=torch.float32, device="cuda")
+        run = lambda: W.wush_gemm_nvfp4(dev(a_c), W.wush_mx_scales_to_atoms(dev(a_s)), ta, dev(b_c),
+                                        W.wush_mx_scales_to_atoms(dev(b_s)), tb)
+    else:
+        a_c, a_s = random_operand(M, K, 5)
+        b_c, b_s = random_operand(N, K, 6)
+        run = lambda: W.wush_gemm_mxfp4(dev(a_c), W.wush_mx_scales_to_atoms(dev(a_s)), dev(b_c),
+                                        W.wush_mx_scales_to_atoms(dev(b_s)))
+    try:
+        W.wush_set_gemm_cta_pairs(True)
+        d_pair = run()
+        W.wush_set_gemm_cta_pairs(False)
+        d_single = run()
+        torch.cuda.synchronize()
+    finally:
+        W.wush_set_gemm_cta_pairs(False)
+    st, bits = W.wush_device_status()
+    assert st == 0 and bits == 0, f"device error word {bits:#x}"
+    for d in (d_pair, d_single):
+        if nv:
+            assert_gemm_nv_close(d.float().cpu().numpy(), a_c, a_s, 0.5, b_c, b_s, 1.25, K)
+        else:
+            assert_gemm_close(d.float().cpu().numpy(), a_c, a_s, b_c, b_s, K)
