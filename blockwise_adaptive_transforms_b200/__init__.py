@@ -24,7 +24,8 @@ __all__ = ["FMT", "WushError", "wush_quant_act", "wush_quant_weight", "wush_quan
            "wush_quant_act_shared_mx_atoms", "wush_gemm_nvfp4", "wush_quant_act_nv_atoms",
            "wush_quant_weight_nv_atoms", "wush_quant_act_nvfp4_amax", "wush_nvfp4_scale_from_amax",
            "wush_quant_act_nvfp4_with_scale", "wush_set_small_batch_rows", "wush_quant_act_nvfp4_onepass",
-           "nvfp4_workspace", "wush_quant_act_nvfp4_onepass_noalloc", "wush_set_gemm_cta_pairs"]
+           "nvfp4_workspace", "wush_quant_act_nvfp4_onepass_noalloc", "wush_set_gemm_cta_pairs",
+           "wush_last_error_detail"]
 
 FMT = {"mxfp4": 0, "nvfp4": 1, "int4": 2}
 STATUS = {0: "WUSH_OK", 1: "WUSH_ERR_INVALID_ARG", 2: "WUSH_ERR_UNSUPPORTED", 3: "WUSH_ERR_MISALIGNED",
@@ -39,13 +40,21 @@ EXPORTED_SYMBOLS = ("wush_quant_act", "wush_quant_weight", "wush_quant_act_debug
                     "wush_quant_act_nvfp4_onepass_noalloc", "wush_set_gemm_cta_pairs",
                     "wush_build_transforms", "wush_device_status",
                     "wush_set_wait_limit_ns",
-                    "wush_selftest_wait_timeout", "wush_status_string", "wush_version")
+                    "wush_selftest_wait_timeout", "wush_status_string", "wush_last_error_detail",
+                    "wush_version")
 
 
 class WushError(RuntimeError):
+    """A non-zero wush_status; for WUSH_ERR_CUDA `detail` names the failing CUDA call.
+
+    Raised on the thread that made the call, so the library's per-thread record of the
+    failure is still the one for this call."""
+
     def __init__(self, status: int, where: str):
         self.status = status
-        super().__init__(f"{where}: {wush_status_string(status)} (status {status})")
+        self.detail = wush_last_error_detail() if status == 4 else ""
+        extra = f" [{self.detail}]" if self.detail else ""
+        super().__init__(f"{where}: {wush_status_string(status)} (status {status}){extra}")
 
 
 _LIB = None
@@ -111,6 +120,8 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
     lib.wush_selftest_wait_timeout.restype = ctypes.c_int
     lib.wush_status_string.argtypes = [ctypes.c_int]
     lib.wush_status_string.restype = ctypes.c_char_p
+    lib.wush_last_error_detail.argtypes = [ctypes.c_char_p, ctypes.c_size_t]
+    lib.wush_last_error_detail.restype = ctypes.c_int
     lib.wush_version.argtypes = []
     lib.wush_version.restype = ctypes.c_int
     if path is None:
@@ -120,6 +131,14 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
 
 def wush_status_string(status: int) -> str:
     return load_library().wush_status_string(int(status)).decode()
+
+
+def wush_last_error_detail() -> str:
+    """The failing CUDA call behind this thread's last WUSH_ERR_CUDA (empty text if none)."""
+    lib = load_library()
+    buf = ctypes.create_string_buffer(512)
+    lib.wush_last_error_detail(buf, len(buf))
+    return buf.value.decode(errors="replace")
 
 
 def wush_version() -> int:

@@ -8,6 +8,8 @@
 #include <atomic>
 #include <climits>
 #include <cstdint>
+#include <cstdio>
+#include <cstring>
 #include <mutex>
 
 #include "wush.h"
@@ -49,6 +51,36 @@ namespace {
 constexpr unsigned long long kDefaultWaitLimitNs = 2000000000ull;
 std::atomic<unsigned long long> g_wait_limit_ns{kDefaultWaitLimitNs};
 
+// The failing call behind the last WUSH_ERR_CUDA returned on this host thread: what was
+// called, where, and the runtime's (or the driver's) error code.
+struct CudaFailure {
+  const char* what = nullptr;
+  int line = 0;
+  int code = 0;
+  bool driver = false;
+};
+thread_local CudaFailure t_cuda_failure;
+
+int cuda_fail(int code, const char* what, int line, bool driver = false) {
+  t_cuda_failure.what = what;
+  t_cuda_failure.line = line;
+  t_cuda_failure.code = code;
+  t_cuda_failure.driver = driver;
+  return WUSH_ERR_CUDA;
+}
+
+// status of the kernel launch just issued on this thread
+int launch_status(int line) {
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? WUSH_OK : cuda_fail(e, "kernel launch", line);
+}
+
+#define WUSH_CUDA_CHECK(call)                                                    \
+  do {                                                                           \
+    const cudaError_t wush_e_ = (call);                                          \
+    if (wush_e_ != cudaSuccess) return cuda_fail(wush_e_, #call, __LINE__);     \
+  } while (0)
+
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
     void* p = nullptr;
@@ -61,26 +93,59 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   return fn;
 }
 
+PFN_cuCtxGetCurrent_v4000 context_getter() {
+  static PFN_cuCtxGetCurrent_v4000 fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return static_cast<PFN_cuCtxGetCurrent_v4000>(nullptr);
+    return reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p);
+  }();
+  return fn;
+}
+
+// Driver-API calls (the tensor-map encoder) act on the context current on the calling host
+// thread.  The runtime binds the current device's primary context to a thread lazily, at
+// its first call there that needs one, so a thread whose first CUDA work is a call into
+// this library may have no context yet; bind it before the first driver call.
+int ensure_context() {
+  auto get = context_getter();
+  if (!get) return cuda_fail(0, "cudaGetDriverEntryPoint(cuCtxGetCurrent)", __LINE__, true);
+  CUcontext c = nullptr;
+  const CUresult r = get(&c);
+  if (r != CUDA_SUCCESS) return cuda_fail(r, "cuCtxGetCurrent", __LINE__, true);
+  if (c) return WUSH_OK;
+  int dev = 0;
+  WUSH_CUDA_CHECK(cudaGetDevice(&dev));
+  WUSH_CUDA_CHECK(cudaSetDevice(dev));   // initialises the primary context and makes it current
+  return WUSH_OK;
+}
+
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
 // 2-D row-major [rows][cols] tensor, box {box_cols, 128 rows}.
 int encode_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dt, int elem_bytes, int64_t rows,
               int64_t cols, int box_cols, CUtensorMapSwizzle swz) {
+  const int ctx = ensure_context();
+  if (ctx != WUSH_OK) return ctx;
   auto enc = tensor_map_encoder();
-  if (!enc) return WUSH_ERR_CUDA;
+  if (!enc) return cuda_fail(0, "cudaGetDriverEntryPoint(cuTensorMapEncodeTiled)", __LINE__, true);
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
   cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * static_cast<cuuint64_t>(elem_bytes)};
   cuuint32_t box[2] = {static_cast<cuuint32_t>(box_cols), 128u};
   cuuint32_t estr[2] = {1u, 1u};
   CUresult r = enc(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                    swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS ? WUSH_OK : WUSH_ERR_CUDA;
+  return r == CUDA_SUCCESS ? WUSH_OK : cuda_fail(r, "cuTensorMapEncodeTiled", __LINE__, true);
 }
 
 // 2-D row-major uint8 [rows][cols] tensor, box {box_cols, box_rows}, no swizzle.
 int encode_u8_plain(CUtensorMap* map, const void* base, int64_t rows, int64_t cols, int box_cols, int box_rows) {
+  const int ctx = ensure_context();
+  if (ctx != WUSH_OK) return ctx;
   auto enc = tensor_map_encoder();
-  if (!enc) return WUSH_ERR_CUDA;
+  if (!enc) return cuda_fail(0, "cudaGetDriverEntryPoint(cuTensorMapEncodeTiled)", __LINE__, true);
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
   cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols)};
   cuuint32_t box[2] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(box_rows)};
@@ -88,13 +153,15 @@ int encode_u8_plain(CUtensorMap* map, const void* base, int64_t rows, int64_t co
   CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS ? WUSH_OK : WUSH_ERR_CUDA;
+  return r == CUDA_SUCCESS ? WUSH_OK : cuda_fail(r, "cuTensorMapEncodeTiled", __LINE__, true);
 }
 
 // 2-D row-major uint8 [rows][cols] tensor, box {box_cols, box_rows}, 128-byte swizzle.
 int encode_u8_sw128(CUtensorMap* map, const void* base, int64_t rows, int64_t cols, int box_cols, int box_rows) {
+  const int ctx = ensure_context();
+  if (ctx != WUSH_OK) return ctx;
   auto enc = tensor_map_encoder();
-  if (!enc) return WUSH_ERR_CUDA;
+  if (!enc) return cuda_fail(0, "cudaGetDriverEntryPoint(cuTensorMapEncodeTiled)", __LINE__, true);
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
   cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols)};
   cuuint32_t box[2] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(box_rows)};
@@ -102,20 +169,19 @@ int encode_u8_sw128(CUtensorMap* map, const void* base, int64_t rows, int64_t co
   CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS ? WUSH_OK : WUSH_ERR_CUDA;
+  return r == CUDA_SUCCESS ? WUSH_OK : cuda_fail(r, "cuTensorMapEncodeTiled", __LINE__, true);
 }
 
 template <class Cfg>
 int launch_fused(const CUtensorMap& map, const CUtensorMap& cmap, wush::FusedParams p, cudaStream_t stream) {
   int dev = 0, sms = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return WUSH_ERR_CUDA;
-  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return WUSH_ERR_CUDA;
+  WUSH_CUDA_CHECK(cudaGetDevice(&dev));
+  WUSH_CUDA_CHECK(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
   static std::atomic<unsigned long long> configured{0ull};   // one bit per device ordinal
   const unsigned long long bit = 1ull << (dev & 63);
   if (!(configured.load(std::memory_order_acquire) & bit)) {
-    if (cudaFuncSetAttribute(wush::wush_fused_kernel<Cfg>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             Cfg::SMEM_BYTES) != cudaSuccess)
-      return WUSH_ERR_CUDA;
+    WUSH_CUDA_CHECK(cudaFuncSetAttribute(wush::wush_fused_kernel<Cfg>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES));
     configured.fetch_or(bit, std::memory_order_acq_rel);
   }
   const int grid = p.total_tiles < sms ? p.total_tiles : sms;
@@ -132,8 +198,8 @@ int launch_fused(const CUtensorMap& map, const CUtensorMap& cmap, wush::FusedPar
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   lc.attrs = attr;
   lc.numAttrs = WUSH_USE_PDL ? 1 : 0;
-  if (cudaLaunchKernelEx(&lc, wush::wush_fused_kernel<Cfg>, map, cmap, p) != cudaSuccess) return WUSH_ERR_CUDA;
-  return cudaGetLastError() == cudaSuccess ? WUSH_OK : WUSH_ERR_CUDA;
+  WUSH_CUDA_CHECK(cudaLaunchKernelEx(&lc, wush::wush_fused_kernel<Cfg>, map, cmap, p));
+  return launch_status(__LINE__);
 }
 
 template <int G, int FMT, bool IN_F32, bool AMAX_ONLY, bool SHARED>
@@ -158,7 +224,7 @@ int dispatch(const CUtensorMap& map, const CUtensorMap& cmap, wush::FusedParams 
   // NVFP4: pass 1 finds amax|y| (float bits, running max in *tensor_scale), a one-thread
   // kernel turns it into s_t in place, pass 2 quantises with s_t.
   if (nv_mode != kNvWithScale) {
-    if (cudaMemsetAsync(tensor_scale, 0, sizeof(float), s) != cudaSuccess) return WUSH_ERR_CUDA;
+    WUSH_CUDA_CHECK(cudaMemsetAsync(tensor_scale, 0, sizeof(float), s));
     wush::FusedParams p1 = p;
     p1.amax_word = reinterpret_cast<unsigned int*>(tensor_scale);
     p1.codes_via_tma = 0;
@@ -166,7 +232,7 @@ int dispatch(const CUtensorMap& map, const CUtensorMap& cmap, wush::FusedParams 
     if (st != WUSH_OK) return st;
     if (nv_mode == kNvAmaxOnly) return WUSH_OK;
     wush::wush_nvfp4_tensor_scale_kernel<<<1, 32, 0, s>>>(tensor_scale);
-    if (cudaGetLastError() != cudaSuccess) return WUSH_ERR_CUDA;
+    WUSH_CUDA_CHECK(cudaGetLastError());
   }
   p.tensor_scale = tensor_scale;
   return launch_pick_y<16, wush::kNVFP4, IN_F32, false, SHARED>(map, cmap, p, emit_y, s);
@@ -191,7 +257,7 @@ int launch_small(const void* x, const wush::FusedParams& p, bool emit_y, cudaStr
     wush::wush_small_kernel<G, FMT, AMAX_ONLY, true, SHARED><<<grid, wush::kSmallRows, 0, s>>>(xb, p);
   else
     wush::wush_small_kernel<G, FMT, AMAX_ONLY, false, SHARED><<<grid, wush::kSmallRows, 0, s>>>(xb, p);
-  return cudaGetLastError() == cudaSuccess ? WUSH_OK : WUSH_ERR_CUDA;
+  return launch_status(__LINE__);
 }
 
 template <bool SHARED>
@@ -202,13 +268,13 @@ int small_dispatch(const void* x, wush::FusedParams p, int G, int fmt, bool emit
     return G == 32 ? launch_small<32, wush::kINT4, false, SHARED>(x, p, emit_y, s)
                    : launch_small<16, wush::kINT4, false, SHARED>(x, p, emit_y, s);
   if (nv_mode != kNvWithScale) {   // NVFP4: amax pass, tensor scale, quantising pass
-    if (cudaMemsetAsync(tensor_scale, 0, sizeof(float), s) != cudaSuccess) return WUSH_ERR_CUDA;
+    WUSH_CUDA_CHECK(cudaMemsetAsync(tensor_scale, 0, sizeof(float), s));
     wush::FusedParams p1 = p;
     p1.amax_word = reinterpret_cast<unsigned int*>(tensor_scale);
     const int st = launch_small<16, wush::kNVFP4, true, SHARED>(x, p1, false, s);
     if (st != WUSH_OK || nv_mode == kNvAmaxOnly) return st;
     wush::wush_nvfp4_tensor_scale_kernel<<<1, 32, 0, s>>>(tensor_scale);
-    if (cudaGetLastError() != cudaSuccess) return WUSH_ERR_CUDA;
+    WUSH_CUDA_CHECK(cudaGetLastError());
   }
   p.tensor_scale = tensor_scale;
   return launch_small<16, wush::kNVFP4, false, SHARED>(x, p, emit_y, s);
@@ -228,8 +294,8 @@ int quant_common(const void* in, bool in_f32, const float* T, int64_t rows, int6
     if (!amax_only) return WUSH_OK;
     if (!tensor_scale || !aligned(tensor_scale, 4)) return tensor_scale ? WUSH_ERR_MISALIGNED : WUSH_ERR_INVALID_ARG;
     // an empty shard still contributes its amax (0) to a reduction across ranks
-    return cudaMemsetAsync(tensor_scale, 0, sizeof(float), reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
-               ? WUSH_OK : WUSH_ERR_CUDA;
+    WUSH_CUDA_CHECK(cudaMemsetAsync(tensor_scale, 0, sizeof(float), reinterpret_cast<cudaStream_t>(stream)));
+    return WUSH_OK;
   }
   if (!in || !T || (!amax_only && (!codes || !scales))) return WUSH_ERR_INVALID_ARG;
   if (fmt == WUSH_NVFP4 && !tensor_scale) return WUSH_ERR_INVALID_ARG;
@@ -355,8 +421,8 @@ int wush_dequant(const uint8_t* codes, const void* scales, const float* tensor_s
       (tensor_scale && !aligned(tensor_scale, 4)))
     return WUSH_ERR_MISALIGNED;
   int dev = 0, sms = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return WUSH_ERR_CUDA;
-  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return WUSH_ERR_CUDA;
+  WUSH_CUDA_CHECK(cudaGetDevice(&dev));
+  WUSH_CUDA_CHECK(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
   const long long n_words = rows * (d_in / 8);
   const long long want = (n_words + 255) / 256;
   const int grid = static_cast<int>(want < 8LL * sms ? want : 8LL * sms);
@@ -368,7 +434,7 @@ int wush_dequant(const uint8_t* codes, const void* scales, const float* tensor_s
     wush::wush_dequant_kernel<wush::kNVFP4><<<grid, 256, 0, s>>>(codes, scales, tensor_scale, rows, di, G, out);
   else
     wush::wush_dequant_kernel<wush::kINT4><<<grid, 256, 0, s>>>(codes, scales, tensor_scale, rows, di, G, out);
-  return cudaGetLastError() == cudaSuccess ? WUSH_OK : WUSH_ERR_CUDA;
+  return launch_status(__LINE__);
 }
 
 int wush_mx_scales_to_atoms(const uint8_t* scales, int64_t rows, int64_t C, uint8_t* atoms, wush_stream_t stream) {
@@ -379,13 +445,13 @@ int wush_mx_scales_to_atoms(const uint8_t* scales, int64_t rows, int64_t C, uint
   const int C_pad = static_cast<int>((C + 3) / 4 * 4);
   const long long n = rows_pad * C_pad;
   int dev = 0, sms = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return WUSH_ERR_CUDA;
-  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return WUSH_ERR_CUDA;
+  WUSH_CUDA_CHECK(cudaGetDevice(&dev));
+  WUSH_CUDA_CHECK(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
   const long long want = (n + 255) / 256;
   const int grid = static_cast<int>(want < 8LL * sms ? want : 8LL * sms);
   wush::wush_scales_to_atoms_kernel<<<grid, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
       scales, rows, static_cast<int>(C), atoms, rows_pad, C_pad);
-  return cudaGetLastError() == cudaSuccess ? WUSH_OK : WUSH_ERR_CUDA;
+  return launch_status(__LINE__);
 }
 
 }  // extern "C"
@@ -426,14 +492,13 @@ int gemm_fp4_pair(const uint8_t* a_codes, const uint8_t* a_atoms, const float* a
   p.tiles_n = static_cast<int>(N / Cfg::BN);
   p.wait_limit_ns = g_wait_limit_ns.load(std::memory_order_relaxed);
   int dev = 0, sms = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return WUSH_ERR_CUDA;
-  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return WUSH_ERR_CUDA;
+  WUSH_CUDA_CHECK(cudaGetDevice(&dev));
+  WUSH_CUDA_CHECK(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
   static std::atomic<unsigned long long> configured{0ull};
   const unsigned long long bit = 1ull << (dev & 63);
   if (!(configured.load(std::memory_order_acquire) & bit)) {
-    if (cudaFuncSetAttribute(wush::wush_gemm_fp4_pair_kernel<Cfg>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             Cfg::SMEM_BYTES) != cudaSuccess)
-      return WUSH_ERR_CUDA;
+    WUSH_CUDA_CHECK(cudaFuncSetAttribute(wush::wush_gemm_fp4_pair_kernel<Cfg>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES));
     configured.fetch_or(bit, std::memory_order_acq_rel);
   }
   const long long tiles = static_cast<long long>(p.tiles_m) * p.tiles_n;
@@ -453,9 +518,8 @@ int gemm_fp4_pair(const uint8_t* a_codes, const uint8_t* a_atoms, const float* a
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   lc.attrs = attr;
   lc.numAttrs = WUSH_USE_PDL ? 2 : 1;
-  if (cudaLaunchKernelEx(&lc, wush::wush_gemm_fp4_pair_kernel<Cfg>, ma, mb, msa, msb, p) != cudaSuccess)
-    return WUSH_ERR_CUDA;
-  return cudaGetLastError() == cudaSuccess ? WUSH_OK : WUSH_ERR_CUDA;
+  WUSH_CUDA_CHECK(cudaLaunchKernelEx(&lc, wush::wush_gemm_fp4_pair_kernel<Cfg>, ma, mb, msa, msb, p));
+  return launch_status(__LINE__);
 }
 
 // One launch of the block-scaled FP4 GEMM (MXFP4 or NVFP4 operands).
@@ -494,14 +558,13 @@ int gemm_fp4(const uint8_t* a_codes, const uint8_t* a_atoms, const float* a_ts, 
   p.tiles_n = static_cast<int>(N / Cfg::BN);
   p.wait_limit_ns = g_wait_limit_ns.load(std::memory_order_relaxed);
   int dev = 0, sms = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return WUSH_ERR_CUDA;
-  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return WUSH_ERR_CUDA;
+  WUSH_CUDA_CHECK(cudaGetDevice(&dev));
+  WUSH_CUDA_CHECK(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
   static std::atomic<unsigned long long> configured{0ull};
   const unsigned long long bit = 1ull << (dev & 63);
   if (!(configured.load(std::memory_order_acquire) & bit)) {
-    if (cudaFuncSetAttribute(wush::wush_gemm_fp4_kernel<Cfg>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             Cfg::SMEM_BYTES) != cudaSuccess)
-      return WUSH_ERR_CUDA;
+    WUSH_CUDA_CHECK(cudaFuncSetAttribute(wush::wush_gemm_fp4_kernel<Cfg>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES));
     configured.fetch_or(bit, std::memory_order_acq_rel);
   }
   const long long tiles = static_cast<long long>(p.tiles_m) * p.tiles_n;
@@ -517,8 +580,8 @@ int gemm_fp4(const uint8_t* a_codes, const uint8_t* a_atoms, const float* a_ts, 
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   lc.attrs = attr;
   lc.numAttrs = WUSH_USE_PDL ? 1 : 0;
-  if (cudaLaunchKernelEx(&lc, wush::wush_gemm_fp4_kernel<Cfg>, ma, mb, p) != cudaSuccess) return WUSH_ERR_CUDA;
-  return cudaGetLastError() == cudaSuccess ? WUSH_OK : WUSH_ERR_CUDA;
+  WUSH_CUDA_CHECK(cudaLaunchKernelEx(&lc, wush::wush_gemm_fp4_kernel<Cfg>, ma, mb, p));
+  return launch_status(__LINE__);
 }
 
 }  // namespace
@@ -576,7 +639,7 @@ int wush_nvfp4_scale_from_amax(float* amax_to_scale, wush_stream_t stream) {
   if (!amax_to_scale) return WUSH_ERR_INVALID_ARG;
   if (!aligned(amax_to_scale, 4)) return WUSH_ERR_MISALIGNED;
   wush::wush_nvfp4_tensor_scale_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(amax_to_scale);
-  return cudaGetLastError() == cudaSuccess ? WUSH_OK : WUSH_ERR_CUDA;
+  return launch_status(__LINE__);
 }
 
 int wush_quant_act_nvfp4_with_scale(const void* x_bf16, const float* T_blocks, int64_t n_tok, int64_t d_in,
@@ -598,11 +661,10 @@ int wush_quant_act_nvfp4_onepass(const void* x_bf16, const float* T_blocks, int6
   const long long C = d_in / 16;
   const long long gy = (n_tok + wush::kSmallRows - 1) / wush::kSmallRows;
   int dev = 0, sms = 0, per_sm = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return WUSH_ERR_CUDA;
-  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return WUSH_ERR_CUDA;
+  WUSH_CUDA_CHECK(cudaGetDevice(&dev));
+  WUSH_CUDA_CHECK(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
   auto kern = wush::wush_small_nvfp4_onepass_kernel<false, false>;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, wush::kSmallRows, 0) != cudaSuccess)
-    return WUSH_ERR_CUDA;
+  WUSH_CUDA_CHECK(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, wush::kSmallRows, 0));
   // the CTAs wait on one another: the whole grid must be resident at once
   if (C * gy > static_cast<long long>(per_sm) * sms || gy > 65535) return WUSH_ERR_UNSUPPORTED;
   wush::FusedParams p{};
@@ -623,16 +685,15 @@ int wush_quant_act_nvfp4_onepass(const void* x_bf16, const float* T_blocks, int6
   attr[0].val.cooperative = 1;
   lc.attrs = attr;
   lc.numAttrs = 1;
-  if (cudaLaunchKernelEx(&lc, kern, static_cast<const __nv_bfloat16*>(x_bf16), p,
-                         reinterpret_cast<unsigned int*>(workspace)) != cudaSuccess)
-    return WUSH_ERR_CUDA;
-  return cudaGetLastError() == cudaSuccess ? WUSH_OK : WUSH_ERR_CUDA;
+  WUSH_CUDA_CHECK(cudaLaunchKernelEx(&lc, kern, static_cast<const __nv_bfloat16*>(x_bf16), p,
+                         reinterpret_cast<unsigned int*>(workspace)));
+  return launch_status(__LINE__);
 }
 
 int wush_quant_act_nvfp4_onepass_noalloc(const void* x_bf16, const float* T_blocks, int64_t n_tok, int64_t d_in,
                                          uint8_t* codes, uint8_t* scales, float* tensor_scale, wush_stream_t stream) {
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return WUSH_ERR_CUDA;
+  WUSH_CUDA_CHECK(cudaGetDevice(&dev));
   if (dev < 0 || dev >= 64) return WUSH_ERR_UNSUPPORTED;
   static std::mutex mu;
   static void* scratch[64] = {};
@@ -641,7 +702,8 @@ int wush_quant_act_nvfp4_onepass_noalloc(const void* x_bf16, const float* T_bloc
     std::lock_guard<std::mutex> lock(mu);
     if (!scratch[dev]) {   // once per device, with that device current
       void* a = nullptr;
-      if (cudaGetSymbolAddress(&a, wush::g_noalloc_scratch) != cudaSuccess || !a) return WUSH_ERR_CUDA;
+      WUSH_CUDA_CHECK(cudaGetSymbolAddress(&a, wush::g_noalloc_scratch));
+      if (!a) return cuda_fail(cudaErrorInvalidSymbol, "cudaGetSymbolAddress", __LINE__);
       scratch[dev] = a;
     }
     ws = scratch[dev];
@@ -689,26 +751,23 @@ int wush_build_transforms(const float* w_f32, const void* xcal_bf16, int64_t d_o
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (G == 32) {
     constexpr int bytes = wush::BuildSmem<32>::BYTES;
-    if (cudaFuncSetAttribute(wush::wush_build_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) !=
-        cudaSuccess)
-      return WUSH_ERR_CUDA;
+    WUSH_CUDA_CHECK(
+        cudaFuncSetAttribute(wush::wush_build_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes));
     wush::wush_build_kernel<32><<<p.C, wush::kBuildThreads, bytes, s>>>(p);
   } else {
     constexpr int bytes = wush::BuildSmem<16>::BYTES;
-    if (cudaFuncSetAttribute(wush::wush_build_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) !=
-        cudaSuccess)
-      return WUSH_ERR_CUDA;
+    WUSH_CUDA_CHECK(
+        cudaFuncSetAttribute(wush::wush_build_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes));
     wush::wush_build_kernel<16><<<p.C, wush::kBuildThreads, bytes, s>>>(p);
   }
-  return cudaGetLastError() == cudaSuccess ? WUSH_OK : WUSH_ERR_CUDA;
+  return launch_status(__LINE__);
 }
 
 int wush_device_status(wush_stream_t stream, uint32_t* bits) {
-  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return WUSH_ERR_CUDA;
+  WUSH_CUDA_CHECK(cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)));
   unsigned int word = 0u, zero = 0u;
-  if (cudaMemcpyFromSymbol(&word, wush::g_wush_device_error, sizeof(word)) != cudaSuccess) return WUSH_ERR_CUDA;
-  if (word && cudaMemcpyToSymbol(wush::g_wush_device_error, &zero, sizeof(zero)) != cudaSuccess)
-    return WUSH_ERR_CUDA;
+  WUSH_CUDA_CHECK(cudaMemcpyFromSymbol(&word, wush::g_wush_device_error, sizeof(word)));
+  if (word) WUSH_CUDA_CHECK(cudaMemcpyToSymbol(wush::g_wush_device_error, &zero, sizeof(zero)));
   if (bits) *bits = word;
   return word ? WUSH_ERR_DEVICE_TIMEOUT : WUSH_OK;
 }
@@ -721,7 +780,7 @@ int wush_set_wait_limit_ns(uint64_t ns) {
 int wush_selftest_wait_timeout(uint64_t limit_ns, wush_stream_t stream, uint32_t* bits) {
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   wush::wush_selftest_wait_kernel<<<1, 32, 0, s>>>(limit_ns);
-  if (cudaGetLastError() != cudaSuccess) return WUSH_ERR_CUDA;
+  WUSH_CUDA_CHECK(cudaGetLastError());
   uint32_t word = 0;
   const int st = wush_device_status(stream, &word);
   if (bits) *bits = word;
@@ -738,6 +797,27 @@ const char* wush_status_string(int status) {
     case WUSH_ERR_DEVICE_TIMEOUT: return "WUSH_ERR_DEVICE_TIMEOUT: an in-kernel wait expired";
     default: return "unknown wush status";
   }
+}
+
+int wush_last_error_detail(char* buf, size_t len) {
+  const CudaFailure f = t_cuda_failure;
+  char tmp[512];
+  if (!f.what) {
+    snprintf(tmp, sizeof(tmp), "no CUDA failure recorded on this thread");
+  } else if (f.driver) {
+    snprintf(tmp, sizeof(tmp), "%s (wush_api.cu:%d) failed: CUresult %d", f.what, f.line, f.code);
+  } else {
+    const cudaError_t e = static_cast<cudaError_t>(f.code);
+    snprintf(tmp, sizeof(tmp), "%s (wush_api.cu:%d) failed: %s: %s", f.what, f.line, cudaGetErrorName(e),
+             cudaGetErrorString(e));
+  }
+  const int n = static_cast<int>(strlen(tmp));
+  if (buf && len) {
+    const size_t k = static_cast<size_t>(n) < len - 1 ? static_cast<size_t>(n) : len - 1;
+    memcpy(buf, tmp, k);
+    buf[k] = '\0';
+  }
+  return n;
 }
 
 int wush_version(void) { return 100; }

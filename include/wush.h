@@ -63,6 +63,7 @@
 #ifndef WUSH_H_
 #define WUSH_H_
 
+#include <stddef.h>
 #include <stdint.h>
 
 #ifdef __cplusplus
@@ -319,6 +320,15 @@ int wush_selftest_wait_timeout(uint64_t limit_ns, wush_stream_t stream, uint32_t
 
 /* Human-readable name of a wush_status value (static string, never NULL). */
 const char* wush_status_string(int status);
+
+/* The call behind the last WUSH_ERR_CUDA that a wush_* function returned on the calling
+ * host thread: its name, the source line in the library, and the CUDA runtime's error
+ * name and message (or the driver's CUresult for a tensor-map encoding).  The record is
+ * per host thread and is overwritten by the next such failure on that thread; it is not
+ * cleared by calls that succeed.  Writes at most len - 1 characters and a terminating NUL
+ * into buf (nothing if buf is NULL or len is 0) and returns the full length of the
+ * message.  Never fails. */
+int wush_last_error_detail(char* buf, size_t len);
 
 /* Library ABI version (major * 10000 + minor * 100 + patch). */
 int wush_version(void);

@@ -139,3 +139,32 @@ def test_builder_argument_checks(lib):
     assert b(A16 + 2, A16, 64, 64, 256, 32, 0.01, 1, A16, A16, None, None, None, None) == MISALIGNED
     assert b(A16, A1, 64, 64, 256, 32, 0.01, 1, A16, A16, None, None, None, None) == MISALIGNED
     assert b(A16, A16, 64, 64, 256, 32, 0.01, 1, A16, A16, A4, None, None, None) == MISALIGNED
+
+
+def test_error_detail_buffer_contract(lib):
+    # nothing has failed on this (fresh) thread yet
+    import threading
+    out = {}
+
+    def fresh():
+        out["n"] = lib.wush_last_error_detail(None, 0)
+        buf = ctypes.create_string_buffer(8)
+        out["short"] = (lib.wush_last_error_detail(buf, len(buf)), buf.value)
+
+    t = threading.Thread(target=fresh)
+    t.start()
+    t.join()
+    assert out["n"] == len("no CUDA failure recorded on this thread")
+    n, text = out["short"]
+    assert n == out["n"] and text == b"no CUDA"        # truncated to len - 1, NUL-terminated
+
+
+@pytest.mark.skipif(__import__("torch").cuda.is_available(), reason="needs a machine without a GPU")
+def test_cuda_failure_names_the_failing_call(lib):
+    # without a device the status query's stream synchronisation fails in the runtime
+    bits = ctypes.c_uint32(0)
+    assert lib.wush_device_status(None, ctypes.byref(bits)) == 4
+    detail = W.wush_last_error_detail()
+    assert detail.startswith("cudaStreamSynchronize(") and "failed: cudaError" in detail, detail
+    e = W.WushError(4, "wush_device_status")
+    assert e.detail == detail and detail in str(e)
