@@ -59,6 +59,7 @@ struct FusedParams {
   int codes_via_tma;        // 1: codes leave through the TMA store map (needs d_in % 32 == 0)
   int scale_atoms;          // MXFP4 only: 1 = scales in the block-scaled MMA's scale-atom layout
   int atom_cols;            // scale atoms per 128-row block (C padded to 4, / 4)
+  int prefetch_tiles;       // input tiles per CTA warmed in L2 before the dependency wait
   unsigned long long wait_limit_ns;
 };
 
@@ -309,6 +310,22 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
     fence_barrier_init();
     tma_prefetch_desc(&tmap_in);
     if (p.codes_via_tma) tma_prefetch_desc(&tmap_codes);
+    // Warm L2 with the CTA's first input tiles and its first column tile's matrices while
+    // the previous kernel in the stream drains.  A prefetch hands no data to this CTA and
+    // L2 is the point of coherence, so the loads issued after the dependency wait still
+    // see everything the previous kernel wrote.
+    for (int k = 0; k < p.prefetch_tiles && t_begin + k < t_end; ++k) {
+      const int t = t_begin + k;
+      const int ct = t / nrt, rt = t - ct * nrt;
+#pragma unroll
+      for (int s = 0; s < Cfg::SUB; ++s) tma_prefetch_l2_2d(&tmap_in, ct * CH + 64 * s, rt * 128);
+    }
+    if (p.prefetch_tiles > 0 && t_begin < t_end) {
+      const int ct = t_begin / nrt;
+      const int nblk = Cfg::SHARED_T ? 1 : min(BPT, p.C - ct * BPT);
+      bulk_prefetch_l2(p.T + (Cfg::SHARED_T ? 0ll : static_cast<long long>(ct) * BPT * G * G),
+                       static_cast<uint32_t>(nblk * G * G * 4));
+    }
   }
   // Launched with programmatic stream serialisation: everything above overlapped the end
   // of the previous kernel in the stream; its results are visible only after this wait.
