@@ -151,6 +151,26 @@ def _stream_handle(stream) -> int:
     return int(stream.cuda_stream) if hasattr(stream, "cuda_stream") else int(stream)
 
 
+def _launch_stream(stream, device) -> torch.cuda.Stream:
+    """The stream a call launches on: ``stream`` (a torch stream or a raw handle), else the
+    current stream of the input's device."""
+    if torch.device(device).type != "cuda":
+        raise TypeError("inputs must be CUDA tensors")
+    if stream is None:
+        return torch.cuda.current_stream(device)
+    if isinstance(stream, torch.cuda.Stream):
+        return stream
+    return torch.cuda.ExternalStream(int(stream), device=device)
+
+
+def _empty(shape, dtype, s, zero=False):
+    """An output buffer allocated (and, if asked, zero-filled) on the launch stream s, so
+    that torch's caching allocator orders its reuse after the launch and no fill on
+    another stream races the kernel."""
+    with torch.cuda.stream(s):
+        return (torch.zeros if zero else torch.empty)(shape, dtype=dtype, device=s.device)
+
+
 def _fmt_code(fmt) -> int:
     return FMT[fmt] if isinstance(fmt, str) else int(fmt)
 
@@ -170,14 +190,14 @@ def _check_dev(t: torch.Tensor, name: str, dtype=None):
         raise ValueError(f"{name} must be contiguous")
 
 
-def _alloc_outputs(ref: torch.Tensor, rows: int, d_in: int, G: int, fmt, codes, scales, tensor_scale):
+def _alloc_outputs(s, rows: int, d_in: int, G: int, fmt, codes, scales, tensor_scale):
     cs, ss, sdt = output_shapes(rows, d_in, G, fmt)
     if codes is None:
-        codes = torch.empty(cs, dtype=torch.uint8, device=ref.device)
+        codes = _empty(cs, torch.uint8, s)
     if scales is None:
-        scales = torch.empty(ss, dtype=sdt, device=ref.device)
+        scales = _empty(ss, sdt, s)
     if tensor_scale is None and _fmt_code(fmt) == FMT["nvfp4"]:
-        tensor_scale = torch.empty(1, dtype=torch.float32, device=ref.device)
+        tensor_scale = _empty(1, torch.float32, s)
     _check_dev(codes, "codes", torch.uint8)
     _check_dev(scales, "scales", sdt)
     if tuple(codes.shape) != cs or tuple(scales.shape) != ss:
@@ -203,12 +223,13 @@ def _call(fn_name, inp, in_dtype, T, G, fmt, codes, scales, tensor_scale, y, str
     t_shape = (G, G) if shared else (d_in // G, G, G)
     if tuple(T.shape) != t_shape:
         raise ValueError(f"T must have shape {t_shape}")
-    codes, scales, tensor_scale = _alloc_outputs(inp, rows, d_in, G, fmt, codes, scales, tensor_scale)
+    s = _launch_stream(stream, inp.device)
+    codes, scales, tensor_scale = _alloc_outputs(s, rows, d_in, G, fmt, codes, scales, tensor_scale)
     args = [_ptr(inp), _ptr(T), rows, d_in, int(G), _fmt_code(fmt), _ptr(codes), _ptr(scales),
             _ptr(tensor_scale)]
     if y is not None:
         args.append(_ptr(y))
-    args.append(_stream_handle(stream))
+    args.append(s.cuda_stream)
     with torch.cuda.device(inp.device):
         st = getattr(lib, fn_name)(*args)
     if st != 0:
@@ -226,9 +247,9 @@ def wush_quant_weight(w, T, G, fmt, codes=None, scales=None, tensor_scale=None, 
     return _call("wush_quant_weight", w, torch.float32, T, G, fmt, codes, scales, tensor_scale, None, stream)
 
 
-def _y_buffer(inp, y):
+def _y_buffer(inp, y, stream):
     if y is None:
-        y = torch.empty(inp.shape, dtype=torch.float32, device=inp.device)
+        y = _empty(inp.shape, torch.float32, _launch_stream(stream, inp.device))
     _check_dev(y, "y_out", torch.float32)
     if tuple(y.shape) != tuple(inp.shape):
         raise ValueError("y_out must have the input's shape")
@@ -237,13 +258,13 @@ def _y_buffer(inp, y):
 
 def wush_quant_act_debug(x, T, G, fmt, y_out=None, stream=None):
     """As wush_quant_act, also returning the fp32 transformed values y the kernel quantised."""
-    y = _y_buffer(x, y_out)
+    y = _y_buffer(x, y_out, stream)
     c, s, ts = _call("wush_quant_act_debug", x, torch.bfloat16, T, G, fmt, None, None, None, y, stream)
     return c, s, ts, y
 
 
 def wush_quant_weight_debug(w, T, G, fmt, y_out=None, stream=None):
-    y = _y_buffer(w, y_out)
+    y = _y_buffer(w, y_out, stream)
     c, s, ts = _call("wush_quant_weight_debug", w, torch.float32, T, G, fmt, None, None, None, y, stream)
     return c, s, ts, y
 
@@ -255,7 +276,7 @@ def wush_quant_act_shared(x, T, G, fmt, codes=None, scales=None, tensor_scale=No
 
 
 def wush_quant_act_shared_debug(x, T, G, fmt, y_out=None, stream=None):
-    y = _y_buffer(x, y_out)
+    y = _y_buffer(x, y_out, stream)
     c, s, ts = _call("wush_quant_act_shared_debug", x, torch.bfloat16, T, G, fmt, None, None, None, y, stream,
                      shared=True)
     return c, s, ts, y
@@ -274,14 +295,15 @@ def wush_dequant(codes, scales, tensor_scale, G, fmt, out=None, stream=None):
         raise ValueError(f"scales must have shape {ss}")
     if tensor_scale is not None:
         _check_dev(tensor_scale, "tensor_scale", torch.float32)
+    s = _launch_stream(stream, codes.device)
     if out is None:
-        out = torch.empty((rows, d_in), dtype=torch.float32, device=codes.device)
+        out = _empty((rows, d_in), torch.float32, s)
     _check_dev(out, "out", torch.float32)
     if tuple(out.shape) != (rows, d_in):
         raise ValueError("out must be [rows][d_in]")
     with torch.cuda.device(codes.device):
         st = lib.wush_dequant(_ptr(codes), _ptr(scales), _ptr(tensor_scale), rows, d_in, int(G), _fmt_code(fmt),
-                              _ptr(out), _stream_handle(stream))
+                              _ptr(out), s.cuda_stream)
     if st != 0:
         raise WushError(st, "wush_dequant")
     return out
@@ -297,13 +319,14 @@ def wush_mx_scales_to_atoms(scales, out=None, stream=None):
     lib = load_library()
     _check_dev(scales, "scales", torch.uint8)
     rows, C = int(scales.shape[0]), int(scales.shape[1])
+    s = _launch_stream(stream, scales.device)
     if out is None:
-        out = torch.empty(atom_bytes(rows, C), dtype=torch.uint8, device=scales.device)
+        out = _empty(atom_bytes(rows, C), torch.uint8, s)
     _check_dev(out, "atoms", torch.uint8)
     if out.numel() < atom_bytes(rows, C):
         raise ValueError("atoms buffer too small")
     with torch.cuda.device(scales.device):
-        st = lib.wush_mx_scales_to_atoms(_ptr(scales), rows, C, _ptr(out), _stream_handle(stream))
+        st = lib.wush_mx_scales_to_atoms(_ptr(scales), rows, C, _ptr(out), s.cuda_stream)
     if st != 0:
         raise WushError(st, "wush_mx_scales_to_atoms")
     return out
@@ -319,10 +342,11 @@ def _quant_atoms(fn_name, inp, in_dtype, T, codes, atoms, stream, shared=False, 
     t_shape = (G, G) if shared else (d_in // G, G, G)
     if tuple(T.shape) != t_shape:
         raise ValueError(f"T must have shape {t_shape}")
+    s = _launch_stream(stream, inp.device)
     if codes is None:
-        codes = torch.empty((rows, d_in // 2), dtype=torch.uint8, device=inp.device)
+        codes = _empty((rows, d_in // 2), torch.uint8, s)
     if atoms is None:
-        atoms = torch.zeros(atom_bytes(rows, d_in // G), dtype=torch.uint8, device=inp.device)
+        atoms = _empty(atom_bytes(rows, d_in // G), torch.uint8, s, zero=True)
     _check_dev(codes, "codes", torch.uint8)
     _check_dev(atoms, "scale atoms", torch.uint8)
     if tuple(codes.shape) != (rows, d_in // 2) or atoms.numel() < atom_bytes(rows, d_in // G):
@@ -330,11 +354,11 @@ def _quant_atoms(fn_name, inp, in_dtype, T, codes, atoms, stream, shared=False, 
     args = [_ptr(inp), _ptr(T), rows, d_in, _ptr(codes), _ptr(atoms)]
     if G == 16:
         if tensor_scale is None:
-            tensor_scale = torch.empty(1, dtype=torch.float32, device=inp.device)
+            tensor_scale = _empty(1, torch.float32, s)
         _check_dev(tensor_scale, "tensor_scale", torch.float32)
         args.append(_ptr(tensor_scale))
     with torch.cuda.device(inp.device):
-        st = getattr(lib, fn_name)(*args, _stream_handle(stream))
+        st = getattr(lib, fn_name)(*args, s.cuda_stream)
     if st != 0:
         raise WushError(st, fn_name)
     return (codes, atoms) if G == 32 else (codes, atoms, tensor_scale)
@@ -379,11 +403,12 @@ def wush_quant_act_nvfp4_amax(x, T, amax=None, stream=None):
     (the first NVFP4 stage; reduce it across ranks before fixing the scale)."""
     lib = load_library()
     n, d = _nv_stage_input(x, T)
+    s = _launch_stream(stream, x.device)
     if amax is None:
-        amax = torch.empty(1, dtype=torch.float32, device=x.device)
+        amax = _empty(1, torch.float32, s)
     _check_dev(amax, "amax", torch.float32)
     with torch.cuda.device(x.device):
-        st = lib.wush_quant_act_nvfp4_amax(_ptr(x), _ptr(T), n, d, _ptr(amax), _stream_handle(stream))
+        st = lib.wush_quant_act_nvfp4_amax(_ptr(x), _ptr(T), n, d, _ptr(amax), s.cuda_stream)
     if st != 0:
         raise WushError(st, "wush_quant_act_nvfp4_amax")
     return amax
@@ -393,8 +418,9 @@ def wush_nvfp4_scale_from_amax(amax, stream=None):
     """In place: amax -> the tensor scale amax / 2688."""
     lib = load_library()
     _check_dev(amax, "amax", torch.float32)
+    s = _launch_stream(stream, amax.device)
     with torch.cuda.device(amax.device):
-        st = lib.wush_nvfp4_scale_from_amax(_ptr(amax), _stream_handle(stream))
+        st = lib.wush_nvfp4_scale_from_amax(_ptr(amax), s.cuda_stream)
     if st != 0:
         raise WushError(st, "wush_nvfp4_scale_from_amax")
     return amax
@@ -405,25 +431,30 @@ def wush_quant_act_nvfp4_with_scale(x, T, tensor_scale, codes=None, scales=None,
     lib = load_library()
     n, d = _nv_stage_input(x, T)
     _check_dev(tensor_scale, "tensor_scale", torch.float32)
+    s = _launch_stream(stream, x.device)
     if codes is None:
-        codes = torch.empty((n, d // 2), dtype=torch.uint8, device=x.device)
+        codes = _empty((n, d // 2), torch.uint8, s)
     if scales is None:
-        scales = torch.empty((n, d // 16), dtype=torch.uint8, device=x.device)
+        scales = _empty((n, d // 16), torch.uint8, s)
     _check_dev(codes, "codes", torch.uint8)
     _check_dev(scales, "scales", torch.uint8)
     if tuple(codes.shape) != (n, d // 2) or tuple(scales.shape) != (n, d // 16):
         raise ValueError("output buffers have the wrong size")
     with torch.cuda.device(x.device):
         st = lib.wush_quant_act_nvfp4_with_scale(_ptr(x), _ptr(T), n, d, _ptr(codes), _ptr(scales),
-                                                 _ptr(tensor_scale), _stream_handle(stream))
+                                                 _ptr(tensor_scale), s.cuda_stream)
     if st != 0:
         raise WushError(st, "wush_quant_act_nvfp4_with_scale")
     return codes, scales
 
 
-def nvfp4_workspace(device=None):
-    """A zeroed workspace for wush_quant_act_nvfp4_onepass (16 bytes of device memory)."""
-    return torch.zeros(4, dtype=torch.int32, device=device if device is not None else "cuda")
+def nvfp4_workspace(device=None, stream=None):
+    """A zeroed workspace for wush_quant_act_nvfp4_onepass (16 bytes of device memory),
+    allocated and zeroed on ``stream`` (default: the device's current stream)."""
+    dev = torch.device(device if device is not None else "cuda")
+    if dev.index is None:
+        dev = torch.device("cuda", torch.cuda.current_device())
+    return _empty(4, torch.int32, _launch_stream(stream, dev), zero=True)
 
 
 def wush_quant_act_nvfp4_onepass(x, T, workspace, codes=None, scales=None, tensor_scale=None, stream=None):
@@ -432,12 +463,13 @@ def wush_quant_act_nvfp4_onepass(x, T, workspace, codes=None, scales=None, tenso
     lib = load_library()
     n, d = _nv_stage_input(x, T)
     _check_dev(workspace, "workspace", torch.int32)
+    s = _launch_stream(stream, x.device)
     if codes is None:
-        codes = torch.empty((n, d // 2), dtype=torch.uint8, device=x.device)
+        codes = _empty((n, d // 2), torch.uint8, s)
     if scales is None:
-        scales = torch.empty((n, d // 16), dtype=torch.uint8, device=x.device)
+        scales = _empty((n, d // 16), torch.uint8, s)
     if tensor_scale is None:
-        tensor_scale = torch.empty(1, dtype=torch.float32, device=x.device)
+        tensor_scale = _empty(1, torch.float32, s)
     for t, name, dt in ((codes, "codes", torch.uint8), (scales, "scales", torch.uint8),
                         (tensor_scale, "tensor_scale", torch.float32)):
         _check_dev(t, name, dt)
@@ -445,7 +477,7 @@ def wush_quant_act_nvfp4_onepass(x, T, workspace, codes=None, scales=None, tenso
         raise ValueError("output or workspace buffers have the wrong size")
     with torch.cuda.device(x.device):
         st = lib.wush_quant_act_nvfp4_onepass(_ptr(x), _ptr(T), n, d, _ptr(codes), _ptr(scales), _ptr(tensor_scale),
-                                              _ptr(workspace), _stream_handle(stream))
+                                              _ptr(workspace), s.cuda_stream)
     if st != 0:
         raise WushError(st, "wush_quant_act_nvfp4_onepass")
     return codes, scales, tensor_scale
@@ -456,12 +488,13 @@ def wush_quant_act_nvfp4_onepass_noalloc(x, T, codes=None, scales=None, tensor_s
     calls that may overlap race).  Returns (codes, scales, tensor_scale)."""
     lib = load_library()
     n, d = _nv_stage_input(x, T)
+    s = _launch_stream(stream, x.device)
     if codes is None:
-        codes = torch.empty((n, d // 2), dtype=torch.uint8, device=x.device)
+        codes = _empty((n, d // 2), torch.uint8, s)
     if scales is None:
-        scales = torch.empty((n, d // 16), dtype=torch.uint8, device=x.device)
+        scales = _empty((n, d // 16), torch.uint8, s)
     if tensor_scale is None:
-        tensor_scale = torch.empty(1, dtype=torch.float32, device=x.device)
+        tensor_scale = _empty(1, torch.float32, s)
     for t, name, dt in ((codes, "codes", torch.uint8), (scales, "scales", torch.uint8),
                         (tensor_scale, "tensor_scale", torch.float32)):
         _check_dev(t, name, dt)
@@ -469,13 +502,13 @@ def wush_quant_act_nvfp4_onepass_noalloc(x, T, codes=None, scales=None, tensor_s
         raise ValueError("output buffers have the wrong size")
     with torch.cuda.device(x.device):
         st = lib.wush_quant_act_nvfp4_onepass_noalloc(_ptr(x), _ptr(T), n, d, _ptr(codes), _ptr(scales),
-                                                      _ptr(tensor_scale), _stream_handle(stream))
+                                                      _ptr(tensor_scale), s.cuda_stream)
     if st != 0:
         raise WushError(st, "wush_quant_act_nvfp4_onepass_noalloc")
     return codes, scales, tensor_scale
 
 
-def _gemm_args(a_codes, a_atoms, b_codes, b_atoms, out, vs):
+def _gemm_args(a_codes, a_atoms, b_codes, b_atoms, out, vs, s):
     for t, n in ((a_codes, "a_codes"), (b_codes, "b_codes"), (a_atoms, "a_atoms"), (b_atoms, "b_atoms")):
         _check_dev(t, n, torch.uint8)
     M, K2 = int(a_codes.shape[0]), int(a_codes.shape[1])
@@ -486,7 +519,7 @@ def _gemm_args(a_codes, a_atoms, b_codes, b_atoms, out, vs):
     if a_atoms.numel() < atom_bytes(M, K // vs) or b_atoms.numel() < atom_bytes(N, K // vs):
         raise ValueError("scale atom buffers too small")
     if out is None:
-        out = torch.empty((M, N), dtype=torch.bfloat16, device=a_codes.device)
+        out = _empty((M, N), torch.bfloat16, s)
     _check_dev(out, "out", torch.bfloat16)
     if tuple(out.shape) != (M, N):
         raise ValueError("out must be [M][N]")
@@ -496,10 +529,11 @@ def _gemm_args(a_codes, a_atoms, b_codes, b_atoms, out, vs):
 def wush_gemm_mxfp4(a_codes, a_atoms, b_codes, b_atoms, out=None, stream=None):
     """bf16 [M][N] = A B^T from MXFP4 codes ([M][K/2], [N][K/2]) and scale atoms."""
     lib = load_library()
-    M, N, K, out = _gemm_args(a_codes, a_atoms, b_codes, b_atoms, out, 32)
+    s = _launch_stream(stream, a_codes.device)
+    M, N, K, out = _gemm_args(a_codes, a_atoms, b_codes, b_atoms, out, 32, s)
     with torch.cuda.device(a_codes.device):
         st = lib.wush_gemm_mxfp4(_ptr(a_codes), _ptr(a_atoms), _ptr(b_codes), _ptr(b_atoms), M, N, K, _ptr(out),
-                                 _stream_handle(stream))
+                                 s.cuda_stream)
     if st != 0:
         raise WushError(st, "wush_gemm_mxfp4")
     return out
@@ -509,12 +543,13 @@ def wush_gemm_nvfp4(a_codes, a_atoms, a_tensor_scale, b_codes, b_atoms, b_tensor
     """bf16 [M][N] = s_A s_B A B^T from NVFP4 codes, E4M3 scale atoms and the two fp32
     tensor scales (device tensors of one element)."""
     lib = load_library()
-    M, N, K, out = _gemm_args(a_codes, a_atoms, b_codes, b_atoms, out, 16)
+    s = _launch_stream(stream, a_codes.device)
+    M, N, K, out = _gemm_args(a_codes, a_atoms, b_codes, b_atoms, out, 16, s)
     _check_dev(a_tensor_scale, "a_tensor_scale", torch.float32)
     _check_dev(b_tensor_scale, "b_tensor_scale", torch.float32)
     with torch.cuda.device(a_codes.device):
         st = lib.wush_gemm_nvfp4(_ptr(a_codes), _ptr(a_atoms), _ptr(a_tensor_scale), _ptr(b_codes), _ptr(b_atoms),
-                                 _ptr(b_tensor_scale), M, N, K, _ptr(out), _stream_handle(stream))
+                                 _ptr(b_tensor_scale), M, N, K, _ptr(out), s.cuda_stream)
     if st != 0:
         raise WushError(st, "wush_gemm_nvfp4")
     return out
@@ -548,17 +583,18 @@ def wush_build_transforms(w, xcal, G, lam=0.01, use_hadamard=True, want_f64=Fals
         raise ValueError("d_in must be a multiple of G")
     C = d_in // G
     dev = w.device
-    Tw = torch.empty((C, G, G), dtype=torch.float32, device=dev)
-    Tx = torch.empty_like(Tw)
+    s = _launch_stream(stream, dev)
+    Tw = _empty((C, G, G), torch.float32, s)
+    Tx = _empty((C, G, G), torch.float32, s)
     Tw64 = Tx64 = s64 = None
     if want_f64:
-        Tw64 = torch.empty((C, G, G), dtype=torch.float64, device=dev)
-        Tx64 = torch.empty_like(Tw64)
-        s64 = torch.empty((C, G), dtype=torch.float64, device=dev)
+        Tw64 = _empty((C, G, G), torch.float64, s)
+        Tx64 = _empty((C, G, G), torch.float64, s)
+        s64 = _empty((C, G), torch.float64, s)
     with torch.cuda.device(dev):
         st = lib.wush_build_transforms(_ptr(w), _ptr(xcal), d_out, n_cal, d_in, int(G), float(lam),
                                        1 if use_hadamard else 0, _ptr(Tw), _ptr(Tx), _ptr(Tw64),
-                                       _ptr(Tx64), _ptr(s64), _stream_handle(stream))
+                                       _ptr(Tx64), _ptr(s64), s.cuda_stream)
     if st != 0:
         raise WushError(st, "wush_build_transforms")
     return (Tw, Tx, Tw64, Tx64, s64) if want_f64 else (Tw, Tx)

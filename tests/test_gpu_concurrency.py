@@ -88,3 +88,21 @@ def test_first_cuda_work_of_a_fresh_thread_is_a_fused_call():
     assert not errors, errors
     s.synchronize()
     assert torch.equal(codes, expected[0]) and torch.equal(scales, expected[1])
+
+
+def test_outputs_are_made_on_the_launch_stream():
+    # The current stream is kept busy while the call launches on a side stream.  The
+    # scale-atom buffer's zero fill must run on the launch stream, ahead of the kernel;
+    # on the busy stream it would land after the kernel and wipe the scales.
+    x, T = _case(7, 200, 1024, 32)
+    codes, atoms = W.wush_quant_act_mx_atoms(x, T)
+    torch.cuda.synchronize()
+    side = torch.cuda.Stream()
+    torch.cuda._sleep(50_000_000)              # ~25 ms of spinning on the current stream
+    c2, a2 = W.wush_quant_act_mx_atoms(x, T, stream=side)
+    side.synchronize()
+    torch.cuda.synchronize()
+    assert torch.equal(c2, codes) and torch.equal(a2, atoms)
+    ws = W.nvfp4_workspace(stream=side)
+    side.synchronize()
+    assert ws.device == x.device and torch.count_nonzero(ws).item() == 0
