@@ -207,6 +207,23 @@ int launch_fused(const CUtensorMap& map, const CUtensorMap& cmap, wush::FusedPar
   return launch_status(__LINE__);
 }
 
+// A launch with programmatic stream serialisation, for kernels that call
+// griddepcontrol.wait before their first global read.
+template <typename... KArgs, typename... Args>
+int launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, cudaStream_t s, Args... args) {
+  cudaLaunchConfig_t lc = {};
+  lc.gridDim = grid;
+  lc.blockDim = block;
+  lc.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  lc.attrs = attr;
+  lc.numAttrs = WUSH_USE_PDL ? 1 : 0;
+  WUSH_CUDA_CHECK(cudaLaunchKernelEx(&lc, kern, args...));
+  return launch_status(__LINE__);
+}
+
 template <int G, int FMT, bool IN_F32, bool AMAX_ONLY, bool SHARED>
 int launch_pick_y(const CUtensorMap& map, const CUtensorMap& cmap, const wush::FusedParams& p, bool emit_y,
                   cudaStream_t s) {
@@ -229,15 +246,16 @@ int dispatch(const CUtensorMap& map, const CUtensorMap& cmap, wush::FusedParams 
   // NVFP4: pass 1 finds amax|y| (float bits, running max in *tensor_scale), a one-thread
   // kernel turns it into s_t in place, pass 2 quantises with s_t.
   if (nv_mode != kNvWithScale) {
-    WUSH_CUDA_CHECK(cudaMemsetAsync(tensor_scale, 0, sizeof(float), s));
+    int st = launch_pdl(wush::wush_nvfp4_amax_reset_kernel, dim3(1), dim3(32), s, tensor_scale);
+    if (st != WUSH_OK) return st;
     wush::FusedParams p1 = p;
     p1.amax_word = reinterpret_cast<unsigned int*>(tensor_scale);
     p1.codes_via_tma = 0;
-    int st = launch_fused<wush::FusedCfg<16, wush::kNVFP4, IN_F32, true, false, SHARED>>(map, cmap, p1, s);
+    st = launch_fused<wush::FusedCfg<16, wush::kNVFP4, IN_F32, true, false, SHARED>>(map, cmap, p1, s);
     if (st != WUSH_OK) return st;
     if (nv_mode == kNvAmaxOnly) return WUSH_OK;
-    wush::wush_nvfp4_tensor_scale_kernel<<<1, 32, 0, s>>>(tensor_scale);
-    WUSH_CUDA_CHECK(cudaGetLastError());
+    st = launch_pdl(wush::wush_nvfp4_tensor_scale_kernel, dim3(1), dim3(32), s, tensor_scale);
+    if (st != WUSH_OK) return st;
   }
   p.tensor_scale = tensor_scale;
   return launch_pick_y<16, wush::kNVFP4, IN_F32, false, SHARED>(map, cmap, p, emit_y, s);
@@ -259,10 +277,8 @@ int launch_small(const void* x, const wush::FusedParams& p, bool emit_y, cudaStr
   const dim3 grid(static_cast<unsigned>(p.C), static_cast<unsigned>((p.n_rows + wush::kSmallRows - 1) / wush::kSmallRows));
   const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
   if (emit_y && !AMAX_ONLY)
-    wush::wush_small_kernel<G, FMT, AMAX_ONLY, true, SHARED><<<grid, wush::kSmallRows, 0, s>>>(xb, p);
-  else
-    wush::wush_small_kernel<G, FMT, AMAX_ONLY, false, SHARED><<<grid, wush::kSmallRows, 0, s>>>(xb, p);
-  return launch_status(__LINE__);
+    return launch_pdl(wush::wush_small_kernel<G, FMT, AMAX_ONLY, true, SHARED>, grid, dim3(wush::kSmallRows), s, xb, p);
+  return launch_pdl(wush::wush_small_kernel<G, FMT, AMAX_ONLY, false, SHARED>, grid, dim3(wush::kSmallRows), s, xb, p);
 }
 
 template <bool SHARED>
@@ -273,13 +289,14 @@ int small_dispatch(const void* x, wush::FusedParams p, int G, int fmt, bool emit
     return G == 32 ? launch_small<32, wush::kINT4, false, SHARED>(x, p, emit_y, s)
                    : launch_small<16, wush::kINT4, false, SHARED>(x, p, emit_y, s);
   if (nv_mode != kNvWithScale) {   // NVFP4: amax pass, tensor scale, quantising pass
-    WUSH_CUDA_CHECK(cudaMemsetAsync(tensor_scale, 0, sizeof(float), s));
+    int st = launch_pdl(wush::wush_nvfp4_amax_reset_kernel, dim3(1), dim3(32), s, tensor_scale);
+    if (st != WUSH_OK) return st;
     wush::FusedParams p1 = p;
     p1.amax_word = reinterpret_cast<unsigned int*>(tensor_scale);
-    const int st = launch_small<16, wush::kNVFP4, true, SHARED>(x, p1, false, s);
+    st = launch_small<16, wush::kNVFP4, true, SHARED>(x, p1, false, s);
     if (st != WUSH_OK || nv_mode == kNvAmaxOnly) return st;
-    wush::wush_nvfp4_tensor_scale_kernel<<<1, 32, 0, s>>>(tensor_scale);
-    WUSH_CUDA_CHECK(cudaGetLastError());
+    st = launch_pdl(wush::wush_nvfp4_tensor_scale_kernel, dim3(1), dim3(32), s, tensor_scale);
+    if (st != WUSH_OK) return st;
   }
   p.tensor_scale = tensor_scale;
   return launch_small<16, wush::kNVFP4, false, SHARED>(x, p, emit_y, s);

@@ -770,11 +770,23 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
 
 // NVFP4: turn the running |y| maximum (float bits) into the fp32 tensor scale
 // s_t = amax / (6 * 448), in place.
+// Both one-thread kernels below wait for the previous kernel in the stream before touching
+// the word (a no-op unless launched with programmatic stream serialisation) and then let
+// the next kernel start its set-up.
 __global__ void wush_nvfp4_tensor_scale_kernel(float* tensor_scale) {
+  grid_dependency_wait();
   if (threadIdx.x == 0 && blockIdx.x == 0) {
     const float amax = __uint_as_float(*reinterpret_cast<unsigned int*>(tensor_scale));
     *tensor_scale = __fdiv_rn(amax, 2688.0f);
   }
+  grid_launch_dependents();
+}
+
+// Clears the running-max word of the NVFP4 amax pass.
+__global__ void wush_nvfp4_amax_reset_kernel(float* word) {
+  grid_dependency_wait();
+  if (threadIdx.x == 0 && blockIdx.x == 0) *word = 0.0f;
+  grid_launch_dependents();
 }
 
 }  // namespace wush

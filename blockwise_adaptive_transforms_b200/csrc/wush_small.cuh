@@ -58,6 +58,9 @@ template <int G, int FMT, bool AMAX_ONLY, bool EMIT_Y, bool SHARED_T>
 __global__ void __launch_bounds__(kSmallRows)
     wush_small_kernel(const __nv_bfloat16* __restrict__ x, const FusedParams p) {
   __shared__ __align__(16) float Ts[G * G];
+  // launched with programmatic stream serialisation: nothing is read before this wait
+  grid_dependency_wait();
+  grid_launch_dependents();
   const int blk = static_cast<int>(blockIdx.x);
   float y[G];
   bool valid;
