@@ -184,7 +184,23 @@ int launch_fused(const CUtensorMap& map, const CUtensorMap& cmap, wush::FusedPar
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES));
     configured.fetch_or(bit, std::memory_order_acq_rel);
   }
-  const int grid = p.total_tiles < sms ? p.total_tiles : sms;
+  int grid = p.total_tiles < sms ? p.total_tiles : sms;
+  // Long bf16 MXFP4 runs take the largest grid (down to 3/4 of the SMs) that gives every
+  // CTA the same whole fraction, or whole multiple, of a column tile.  The CTAs then step
+  // through the same row band together and read whole rows between them.  Measured on
+  // B200: 16384 x 8192 takes 61.5 us on 128 CTAs against 72.7 us on 148.  The fp32 weight
+  // path (60.3 -> 66.5 us), NVFP4 (59.0 -> 67.4 us on 112) and INT4 (21.2 -> 23.1 us at
+  // 8192 x 4096) do more work per tile and lose more with the SMs than they gain.
+  if (Cfg::FMT == wush::kMXFP4 && !Cfg::IN_F32 && p.total_tiles / grid >= 32) {
+    for (int g = grid; g >= (3 * grid) / 4; --g) {
+      if (p.total_tiles % g) continue;
+      const int per = p.total_tiles / g;
+      if (per % p.n_row_tiles == 0 || p.n_row_tiles % per == 0) {
+        grid = g;
+        break;
+      }
+    }
+  }
   // Input tiles each CTA warms in L2 before its dependency wait.  Measured on B200: one
   // for runs of a few tiles per CTA (4096 x 4096 MXFP4: 9.93 -> 9.65 us; two 9.77, three
   // 10.0, all seven 11.3, as the prefetches still in flight delay the first loads), three
