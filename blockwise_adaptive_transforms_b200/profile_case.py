@@ -1,0 +1,43 @@
+"""Run one quantiser configuration a few times, for a profiler to capture.
+
+``python -m blockwise_adaptive_transforms_b200.profile_case --fmt mxfp4 --rows 16384 --d-in 8192``
+quantises seeded bf16 activations (near-identity per-block transforms) ``--launches``
+times on one stream, after ``--warmup`` untimed calls, and checks the device error word.
+Use ``ncu -k regex:wush_fused_kernel -s <warmup launches>`` to capture the timed calls.
+"""
+from __future__ import annotations
+
+import argparse
+
+import torch
+
+import blockwise_adaptive_transforms_b200 as W
+
+GROUP = {"mxfp4": 32, "nvfp4": 16, "int4": 32}
+
+
+def main(argv=None) -> None:
+    ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
+    ap.add_argument("--fmt", choices=sorted(GROUP), default="mxfp4")
+    ap.add_argument("--rows", type=int, default=16384)
+    ap.add_argument("--d-in", type=int, default=8192)
+    ap.add_argument("--warmup", type=int, default=2)
+    ap.add_argument("--launches", type=int, default=2)
+    args = ap.parse_args(argv)
+    G = GROUP[args.fmt]
+    C = args.d_in // G
+    g = torch.Generator().manual_seed(0)
+    x = torch.randn(args.rows, args.d_in, generator=g).to(torch.bfloat16).cuda()
+    T = (torch.eye(G).repeat(C, 1, 1) + 0.05 * torch.randn(C, G, G, generator=g)).float().cuda()
+    out = W.wush_quant_act(x, T, G, args.fmt)
+    for _ in range(args.warmup + args.launches - 1):
+        W.wush_quant_act(x, T, G, args.fmt, codes=out[0], scales=out[1], tensor_scale=out[2])
+    torch.cuda.synchronize()
+    st, bits = W.wush_device_status()
+    if st != 0:
+        raise SystemExit(f"device error word {bits:#x}")
+    print(f"ok: {args.fmt} {args.rows} x {args.d_in}, {args.warmup + args.launches} calls")
+
+
+if __name__ == "__main__":
+    main()
