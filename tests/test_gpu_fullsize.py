@@ -1,6 +1,7 @@
 """Full-size parity: the production entry points at the workloads' full sizes, in the
-launch configuration the benchmark times (persistent grid of min(tiles, SMs) CTAs,
-same instantiation), against the fp64 oracle.
+launch configuration the benchmark times (same instantiation and grid rule: one
+persistent CTA per SM, or for long bf16 MXFP4 runs the aligned grid of fewer CTAs),
+against the fp64 oracle.
 
 The oracle cannot quantise a 16384 x 8192 matrix in seconds, so these tests compare
 sampled (row, block) groups that it computes one by one, and check properties that hold
@@ -141,3 +142,24 @@ def test_int4_token_sweep_in_full(n_tok):
     assert_bit_exact(c.cpu().numpy(), s.cpu().numpy(), None, y.cpu().numpy(), "int4", wl.G)
     y_ref = O.block_transform(O.bf16_to_f64(x_bits), O_T64(b["T_wush32"]))
     assert_end_to_end(c.cpu().numpy(), s.cpu().numpy(), None, y_ref, "int4", wl.G)
+
+
+@pytest.mark.parametrize("rows,d_in", [(12288, 8192), (8192, 16384), (20000, 4160)])
+def test_every_group_is_written_whatever_the_grid(rows, d_in):
+    # 12288 x 8192: aligned grid, half a column tile per CTA; 8192 x 16384: aligned grid, a
+    # whole column tile per CTA; 20000 x 4160: no aligned grid (one CTA per SM), ragged
+    # last row and column tiles.  E8M0 byte 0xFF is never emitted, so a scale still 0xFF
+    # after the call marks a group that no CTA wrote.
+    G, C = 32, d_in // 32
+    gen = torch.Generator(device="cuda").manual_seed(rows + d_in)
+    x = torch.randn(rows, d_in, device="cuda", generator=gen).to(torch.bfloat16)
+    T = (torch.eye(G, device="cuda").repeat(C, 1, 1)
+         + 0.05 * torch.randn(C, G, G, device="cuda", generator=gen)).float()
+    codes = torch.empty((rows, d_in // 2), dtype=torch.uint8, device="cuda")
+    scales = torch.full((rows, C), 0xFF, dtype=torch.uint8, device="cuda")
+    W.wush_quant_act(x, T, G, "mxfp4", codes=codes, scales=scales)
+    torch.cuda.synchronize()
+    st, bits = W.wush_device_status()
+    assert st == 0 and bits == 0, f"device error word {bits:#x}"
+    unwritten = (scales == 0xFF).nonzero()
+    assert unwritten.numel() == 0, f"{unwritten.shape[0]} groups unwritten, first {unwritten[:4].tolist()}"
