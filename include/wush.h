@@ -44,6 +44,15 @@
  * `stream` (0 = legacy default stream), never synchronise the host, allocate nothing
  * and keep no state between calls except the device error word described at
  * wush_device_status().  Inputs must be finite; NaN or Inf gives unspecified codes.
+ * Calls may be made from several host threads and on several streams at once.
+ *
+ * Launch order.  The quantisers, the NVFP4 steps and the FP4 GEMMs launch with
+ * programmatic stream serialisation.  Each kernel lets the next kernel in the stream
+ * begin early, but reads nothing before the previous kernel has completed
+ * (griddepcontrol.wait).  A kernel of the caller's that follows one of these
+ * launches in the same stream behaves normally.  If it is launched with the
+ * programmatic-serialisation attribute itself, it must likewise wait
+ * (griddepcontrol.wait, or cudaGridDependencySynchronize) before reading their outputs.
  *
  * Errors.  Arguments are checked on the host before any launch:
  *   WUSH_ERR_INVALID_ARG   NULL pointer, n_tok/d_out < 0, d_in <= 0, d_in % G != 0,
@@ -52,7 +61,7 @@
  *   WUSH_ERR_MISALIGNED    x, w, T_blocks, codes, y_out not 16-byte aligned; INT4 scales
  *                          or tensor_scale not 4-byte aligned
  *   WUSH_ERR_CUDA          a CUDA runtime error while launching (including a missing or
- *                          non-sm_100 device)
+ *                          non-sm_100 device); wush_last_error_detail() names the call
  * Bits of the device error word (wush_device_status): 1/2/4/8/16 a wait of the TMA
  * producer / MMA issuer / converter / epilogue / final drain expired, 32 the wait
  * self-test expired (expected), 64 a Cholesky pivot was not positive, 128 a CTA of the
