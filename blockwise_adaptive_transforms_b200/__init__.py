@@ -452,7 +452,7 @@ def nvfp4_workspace(device=None, stream=None):
     """A zeroed workspace for wush_quant_act_nvfp4_onepass (16 bytes of device memory),
     allocated and zeroed on ``stream`` (default: the device's current stream)."""
     dev = torch.device(device if device is not None else "cuda")
-    if dev.index is None:
+    if dev.type == "cuda" and dev.index is None:
         dev = torch.device("cuda", torch.cuda.current_device())
     return _empty(4, torch.int32, _launch_stream(stream, dev), zero=True)
 

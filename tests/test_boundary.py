@@ -168,3 +168,18 @@ def test_cuda_failure_names_the_failing_call(lib):
     assert detail.startswith("cudaStreamSynchronize(") and "failed: cudaError" in detail, detail
     e = W.WushError(4, "wush_device_status")
     assert e.detail == detail and detail in str(e)
+
+
+def test_binding_rejects_host_tensors_before_any_cuda_call():
+    # the binding's type checks come before it looks for a stream or a device
+    import torch
+    x = torch.zeros((4, 32), dtype=torch.bfloat16)
+    T = torch.zeros((1, 32, 32), dtype=torch.float32)
+    with pytest.raises(TypeError):
+        W.wush_quant_act(x, T, 32, "mxfp4")
+    with pytest.raises(TypeError):
+        W.wush_quant_act_mx_atoms(x, T)
+    with pytest.raises(TypeError):
+        W.nvfp4_workspace("cpu")
+    with pytest.raises(TypeError):
+        W._launch_stream(None, torch.device("cpu"))
