@@ -609,3 +609,89 @@ def test_generator_bf16_rounding_is_rne():
     # 1 + 2^-8 is a tie between 1 and 1 + 2^-7 -> even (1.0); 1 + 3*2^-9 rounds up to 1 + 2^-7;
     # 1 + 2^-7 + 2^-8 ties between 1+2^-7 (odd) and 1+2^-6 (even) -> 1 + 2^-6.
     assert np.array_equal(O.bf16_to_f64(bits), [1.0, 1.0, 1.0 + 2 ** -7, -2.5, 1.0 + 2 ** -6])
+
+
+# ---------------------------------------------------------------- grid-step distance (rule 2)
+
+
+def _read_grid_steps():
+    rows = []
+    with open(os.path.join(GOLDEN, "grid_steps.txt")) as f:
+        for line in f:
+            if line.startswith("#") or not line.strip():
+                continue
+            fmt, a, b, steps, _ = (t.strip() for t in line.split("|"))
+            rows.append((fmt, int(a, 16), int(b, 16), int(steps)))
+    return rows
+
+
+@pytest.mark.parametrize("row", _read_grid_steps(), ids=lambda r: f"{r[0]}:{r[1]:x}-{r[2]:x}")
+def test_grid_step_distance_hand_worked(row):
+    fmt, a, b, steps = row
+    ofmt = "mxfp4" if fmt == "e2m1" else "int4"
+    assert int(O.grid_step_distance(np.array([a]), np.array([b]), ofmt)[0]) == steps
+    assert int(O.grid_step_distance(np.array([b]), np.array([a]), ofmt)[0]) == steps
+    if ofmt == "mxfp4":    # NVFP4 shares the E2M1 grid
+        assert int(O.grid_step_distance(np.array([a]), np.array([b]), "nvfp4")[0]) == steps
+
+
+def test_grid_step_distance_is_the_rank_difference_on_the_signed_grid():
+    """Brute force over every code pair: the distance equals the difference of the two
+    values' ranks in the sorted list of distinct signed grid points (a table written
+    here from the E2M1 magnitudes, not the oracle's code arithmetic)."""
+    mags = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+    val = {c: (-mags[c & 7] if c & 8 else mags[c & 7]) for c in range(16)}
+    line = sorted(set(v + 0.0 for v in val.values()))           # -0.0 + 0.0 == 0.0
+    assert len(line) == 15
+    rank = {c: line.index(val[c] + 0.0) for c in range(16)}
+    a, b = np.meshgrid(np.arange(16), np.arange(16), indexing="ij")
+    d = O.grid_step_distance(a.ravel(), b.ravel(), "mxfp4")
+    want = np.array([abs(rank[i] - rank[j]) for i, j in zip(a.ravel(), b.ravel())])
+    assert np.array_equal(d, want)
+    # INT4: the 15 valid nibbles (0x8 = -8 is never emitted) on the integer line
+    codes = [c for c in range(16) if c != 8]
+    ival = {c: c if c < 8 else c - 16 for c in codes}
+    ia, ib = np.meshgrid(codes, codes, indexing="ij")
+    d = O.grid_step_distance(ia.ravel(), ib.ravel(), "int4")
+    assert np.array_equal(d, np.array([abs(ival[i] - ival[j]) for i, j in zip(ia.ravel(), ib.ravel())]))
+
+
+# ---------------------------------------------------------------- Eq. (5) with pre-quantised weights
+
+
+def test_layer_loss_prequantised_hand_computed():
+    """Two outputs, one token, one INT4 group of 16 (T_X = I).  x = (7, 1.4, 0, ...) so
+    q(x) = (7, 1, 0, ...) at s = 1 (the 1.4 -> 1 rounding makes q(x) != x).  With
+    w rows (1, 1, 0...) and (0, 2, 0...), and given dequantised weights wq rows
+    (0.5, 0.25, 0...) and (0, 3, 0...):
+      output 0: 7 + x1 - (0.5 * 7 + 0.25 * 1) = 3.25 + x1
+      output 1: 2 x1 - 3 * 1                    = 2 x1 - 3
+    and Eq. (5) divides the squared sum by d_out * d_batch = 2."""
+    G = 16
+    I = np.eye(G, dtype=np.float32)[None]
+    x = np.zeros((1, G)); x[0, 0] = 7.0; x[0, 1] = 1.4
+    xb = bf16_bits_from_f64(x)
+    x1 = O.bf16_to_f64(xb)[0, 1]
+    w = np.zeros((2, G), np.float32); w[0, 0] = 1.0; w[0, 1] = 1.0; w[1, 1] = 2.0
+    wq = np.zeros((2, G)); wq[0, 0] = 0.5; wq[0, 1] = 0.25; wq[1, 1] = 3.0
+    expect = ((3.25 + x1) ** 2 + (2 * x1 - 3.0) ** 2) / 2.0
+    got = O.layer_loss_prequantised(wq, w, xb, I, "int4", G)
+    assert abs(got - expect) < 1e-12
+    # swapping the roles of w and wq changes the value (x is not exactly representable)
+    swapped = O.layer_loss_prequantised(w.astype(np.float64), wq.astype(np.float32), xb, I, "int4", G)
+    assert abs(swapped - expect) > 1e-3
+
+
+def test_layer_loss_prequantised_equals_layer_loss_on_rtn_weights():
+    """With wq = the RTN dequantisation of T_W W, Eq. (5) for pre-quantised weights is
+    the plain layerwise loss (the GPTQ-free case of the same objective)."""
+    wl = workload("tiny_mxfp4")
+    inp = make_inputs(wl)
+    b = O.build_transforms(inp.w, inp.xcal_bits, wl.G)
+    for fmt, G in (("mxfp4", 32), ("int4", 32)):
+        bb = b if G == wl.G else O.build_transforms(inp.w, inp.xcal_bits, G)
+        cw, sw, tw, _ = O.quant_weight(inp.w, bb["T_xvsh32"], G, fmt)
+        wq = O.dequant(O.unpack_nibbles(cw), sw, fmt, G, tw)
+        ref = O.layer_loss(inp.w, inp.x_bits, bb["T_xvsh32"], bb["T_wush32"], fmt, G)
+        got = O.layer_loss_prequantised(wq, inp.w, inp.x_bits, bb["T_wush32"], fmt, G)
+        assert got == pytest.approx(ref, rel=1e-12)
