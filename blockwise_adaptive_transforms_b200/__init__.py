@@ -19,7 +19,7 @@ __all__ = ["FMT", "WushError", "wush_quant_act", "wush_quant_weight", "wush_quan
            "wush_quant_weight_debug", "wush_quant_act_shared", "wush_quant_act_shared_debug",
            "wush_build_transforms", "wush_device_status", "wush_set_wait_limit_ns",
            "wush_selftest_wait_timeout", "wush_status_string", "wush_version", "load_library",
-           "EXPORTED_SYMBOLS", "output_shapes", "hadamard_matrix", "wush_dequant", "wush_gemm_mxfp4",
+           "EXPORTED_SYMBOLS", "output_shapes", "wush_hadamard", "wush_dequant", "wush_gemm_mxfp4",
            "wush_mx_scales_to_atoms", "atom_bytes", "wush_quant_act_mx_atoms", "wush_quant_weight_mx_atoms",
            "wush_quant_act_shared_mx_atoms", "wush_gemm_nvfp4", "wush_quant_act_nv_atoms",
            "wush_quant_weight_nv_atoms", "wush_quant_act_nvfp4_amax", "wush_nvfp4_scale_from_amax",
@@ -38,7 +38,7 @@ EXPORTED_SYMBOLS = ("wush_quant_act", "wush_quant_weight", "wush_quant_act_debug
                     "wush_quant_act_nvfp4_amax", "wush_nvfp4_scale_from_amax", "wush_quant_act_nvfp4_with_scale",
                     "wush_set_small_batch_rows", "wush_quant_act_nvfp4_onepass",
                     "wush_quant_act_nvfp4_onepass_noalloc", "wush_set_gemm_cta_pairs",
-                    "wush_build_transforms", "wush_device_status",
+                    "wush_build_transforms", "wush_hadamard", "wush_device_status",
                     "wush_set_wait_limit_ns",
                     "wush_selftest_wait_timeout", "wush_status_string", "wush_last_error_detail",
                     "wush_version")
@@ -104,6 +104,8 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
     lib.wush_build_transforms.argtypes = [_P, _P, _I64, _I64, _I64, _I32, ctypes.c_double, _I32,
                                           _P, _P, _P, _P, _P, _P]
     lib.wush_build_transforms.restype = ctypes.c_int
+    lib.wush_hadamard.argtypes = [_I32, _I64, _P, _P]
+    lib.wush_hadamard.restype = ctypes.c_int
     lib.wush_device_status.argtypes = [_P, ctypes.POINTER(ctypes.c_uint32)]
     lib.wush_device_status.restype = ctypes.c_int
     lib.wush_quant_act_nvfp4_onepass.argtypes = [_P, _P, _I64, _I64, _P, _P, _P, _P, _P]
@@ -555,15 +557,22 @@ def wush_gemm_nvfp4(a_codes, a_atoms, a_tensor_scale, b_codes, b_atoms, b_tensor
     return out
 
 
-def hadamard_matrix(G, device=None):
-    """The normalised Sylvester Hadamard matrix of order G (entries +-G^-1/2, H H^T = I)
-    as an fp32 [G][G] tensor: the shared matrix of the H+Quant comparator."""
-    if G < 1 or G & (G - 1):
-        raise ValueError("G must be a power of two")
-    H = torch.ones((1, 1), dtype=torch.float64)
-    while H.shape[0] < G:
-        H = torch.cat([torch.cat([H, H], 1), torch.cat([H, -H], 1)], 0)
-    return (H / G ** 0.5).to(torch.float32).to(device if device is not None else "cuda")
+def wush_hadamard(G, copies=None, device=None, stream=None):
+    """The normalised Sylvester Hadamard matrix of order G, written on the device by the
+    library: fp32 [G][G], or [copies][G][G] when ``copies`` is given (the per-block form of
+    the Hadamard-only transform).  One copy is the shared matrix of the H+Quant comparator."""
+    lib = load_library()
+    dev = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
+    if dev.type != "cuda":
+        raise TypeError("wush_hadamard writes device memory; give a CUDA device")
+    n = 1 if copies is None else int(copies)
+    s = _launch_stream(stream, dev)
+    out = _empty((n, G, G) if copies is not None else (G, G), torch.float32, s)
+    with torch.cuda.device(dev):
+        st = lib.wush_hadamard(int(G), n, _ptr(out), s.cuda_stream)
+    if st != 0:
+        raise WushError(st, "wush_hadamard")
+    return out
 
 
 def wush_build_transforms(w, xcal, G, lam=0.01, use_hadamard=True, want_f64=False, stream=None):

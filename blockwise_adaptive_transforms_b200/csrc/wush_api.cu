@@ -687,15 +687,27 @@ int wush_quant_act_nvfp4_with_scale(const void* x_bf16, const float* T_blocks, i
                       const_cast<float*>(tensor_scale), nullptr, false, stream, false, false, kNvWithScale);
 }
 
-int wush_quant_act_nvfp4_onepass(const void* x_bf16, const float* T_blocks, int64_t n_tok, int64_t d_in,
-                                 uint8_t* codes, uint8_t* scales, float* tensor_scale, uint32_t* workspace,
-                                 wush_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+// Host-side checks shared by both one-launch NVFP4 entry points, made before any CUDA
+// call.  Returns WUSH_OK when the call should go on to the launch, kSkipLaunch for an
+// empty batch, or the error status.
+constexpr int kSkipLaunch = -1;
+int onepass_check(const void* x_bf16, const float* T_blocks, int64_t n_tok, int64_t d_in, const uint8_t* codes,
+                  const uint8_t* scales, const float* tensor_scale) {
   if (n_tok < 0 || d_in <= 0 || d_in % 16 != 0 || n_tok > INT_MAX || d_in > INT_MAX) return WUSH_ERR_INVALID_ARG;
-  if (n_tok == 0) return WUSH_OK;
-  if (!x_bf16 || !T_blocks || !codes || !scales || !tensor_scale || !workspace) return WUSH_ERR_INVALID_ARG;
-  if (!aligned(x_bf16, 16) || !aligned(T_blocks, 16) || !aligned(codes, 16) || !aligned(tensor_scale, 4) ||
-      !aligned(workspace, 16))
+  if (n_tok == 0) return kSkipLaunch;
+  if (!x_bf16 || !T_blocks || !codes || !scales || !tensor_scale) return WUSH_ERR_INVALID_ARG;
+  if (!aligned(x_bf16, 16) || !aligned(T_blocks, 16) || !aligned(codes, 16) || !aligned(tensor_scale, 4))
     return WUSH_ERR_MISALIGNED;
+  return WUSH_OK;
+}
+
+// The one-launch NVFP4 kernel on a checked argument set and a 16-byte aligned workspace.
+int onepass_launch(const void* x_bf16, const float* T_blocks, int64_t n_tok, int64_t d_in, uint8_t* codes,
+                   uint8_t* scales, float* tensor_scale, uint32_t* workspace, wush_stream_t stream) {
   const long long C = d_in / 16;
   const long long gy = (n_tok + wush::kSmallRows - 1) / wush::kSmallRows;
   int dev = 0, sms = 0, per_sm = 0;
@@ -724,30 +736,77 @@ int wush_quant_act_nvfp4_onepass(const void* x_bf16, const float* T_blocks, int6
   lc.attrs = attr;
   lc.numAttrs = 1;
   WUSH_CUDA_CHECK(cudaLaunchKernelEx(&lc, kern, static_cast<const __nv_bfloat16*>(x_bf16), p,
-                         reinterpret_cast<unsigned int*>(workspace)));
+                                     reinterpret_cast<unsigned int*>(workspace)));
   return launch_status(__LINE__);
+}
+
+PFN_cuCtxGetId_v12000 context_id_getter() {
+  static PFN_cuCtxGetId_v12000 fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return static_cast<PFN_cuCtxGetId_v12000>(nullptr);
+    return reinterpret_cast<PFN_cuCtxGetId_v12000>(p);
+  }();
+  return fn;
+}
+
+}  // namespace
+
+extern "C" {
+
+int wush_quant_act_nvfp4_onepass(const void* x_bf16, const float* T_blocks, int64_t n_tok, int64_t d_in,
+                                 uint8_t* codes, uint8_t* scales, float* tensor_scale, uint32_t* workspace,
+                                 wush_stream_t stream) {
+  const int st = onepass_check(x_bf16, T_blocks, n_tok, d_in, codes, scales, tensor_scale);
+  if (st == kSkipLaunch) return WUSH_OK;
+  if (st != WUSH_OK) return st;
+  if (!workspace) return WUSH_ERR_INVALID_ARG;
+  if (!aligned(workspace, 16)) return WUSH_ERR_MISALIGNED;
+  return onepass_launch(x_bf16, T_blocks, n_tok, d_in, codes, scales, tensor_scale, workspace, stream);
 }
 
 int wush_quant_act_nvfp4_onepass_noalloc(const void* x_bf16, const float* T_blocks, int64_t n_tok, int64_t d_in,
                                          uint8_t* codes, uint8_t* scales, float* tensor_scale, wush_stream_t stream) {
+  // the arguments first: a rejected call touches neither CUDA nor the scratch record
+  const int st = onepass_check(x_bf16, T_blocks, n_tok, d_in, codes, scales, tensor_scale);
+  if (st == kSkipLaunch) return WUSH_OK;
+  if (st != WUSH_OK) return st;
   int dev = 0;
   WUSH_CUDA_CHECK(cudaGetDevice(&dev));
   if (dev < 0 || dev >= 64) return WUSH_ERR_UNSUPPORTED;
+  // The scratch address belongs to the module as loaded into one context.  It is recorded
+  // per device together with that context's id and taken again when the id changes (the
+  // primary context was reset and the module reloaded).
+  const int ctx_st = ensure_context();
+  if (ctx_st != WUSH_OK) return ctx_st;
+  auto get_ctx = context_getter();
+  auto get_id = context_id_getter();
+  if (!get_id) return cuda_fail(0, "cudaGetDriverEntryPoint(cuCtxGetId)", __LINE__, true);
+  CUcontext ctx = nullptr;
+  unsigned long long ctx_id = 0;
+  CUresult r = get_ctx(&ctx);
+  if (r != CUDA_SUCCESS) return cuda_fail(r, "cuCtxGetCurrent", __LINE__, true);
+  r = get_id(ctx, &ctx_id);
+  if (r != CUDA_SUCCESS) return cuda_fail(r, "cuCtxGetId", __LINE__, true);
   static std::mutex mu;
   static void* scratch[64] = {};
+  static unsigned long long scratch_ctx[64] = {};
   void* ws = nullptr;
   {
     std::lock_guard<std::mutex> lock(mu);
-    if (!scratch[dev]) {   // once per device, with that device current
+    if (!scratch[dev] || scratch_ctx[dev] != ctx_id) {   // with that device current
       void* a = nullptr;
       WUSH_CUDA_CHECK(cudaGetSymbolAddress(&a, wush::g_noalloc_scratch));
       if (!a) return cuda_fail(cudaErrorInvalidSymbol, "cudaGetSymbolAddress", __LINE__);
       scratch[dev] = a;
+      scratch_ctx[dev] = ctx_id;
     }
     ws = scratch[dev];
   }
-  return wush_quant_act_nvfp4_onepass(x_bf16, T_blocks, n_tok, d_in, codes, scales, tensor_scale,
-                                      static_cast<uint32_t*>(ws), stream);
+  return onepass_launch(x_bf16, T_blocks, n_tok, d_in, codes, scales, tensor_scale, static_cast<uint32_t*>(ws),
+                        stream);
 }
 
 int wush_set_gemm_cta_pairs(int enable) {
@@ -798,6 +857,19 @@ int wush_build_transforms(const float* w_f32, const void* xcal_bf16, int64_t d_o
         cudaFuncSetAttribute(wush::wush_build_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes));
     wush::wush_build_kernel<16><<<p.C, wush::kBuildThreads, bytes, s>>>(p);
   }
+  return launch_status(__LINE__);
+}
+
+int wush_hadamard(int G, int64_t copies, float* out, wush_stream_t stream) {
+  if (G < 1 || G > 256 || (G & (G - 1)) != 0) return WUSH_ERR_UNSUPPORTED;
+  if (copies < 0 || copies > (int64_t(1) << 40) / (int64_t(G) * G)) return WUSH_ERR_INVALID_ARG;
+  if (copies == 0) return WUSH_OK;
+  if (!out) return WUSH_ERR_INVALID_ARG;
+  if (!aligned(out, 4)) return WUSH_ERR_MISALIGNED;
+  const long long total = static_cast<long long>(copies) * G * G;
+  const long long blocks = (total + 255) / 256;
+  wush::wush_hadamard_kernel<<<static_cast<unsigned>(blocks < 4096 ? blocks : 4096), 256, 0,
+                               reinterpret_cast<cudaStream_t>(stream)>>>(G, total, out);
   return launch_status(__LINE__);
 }
 

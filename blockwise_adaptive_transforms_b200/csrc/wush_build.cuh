@@ -291,4 +291,21 @@ __global__ void __launch_bounds__(kBuildThreads) wush_build_kernel(const BuildPa
   }
 }
 
+
+// `copies` back-to-back copies of the normalised Sylvester Hadamard matrix of order G
+// (paper-graph-ui analysis, section 3.4.4: H is the orthonormal Hadamard that spreads
+// S^-1/2 evenly over a block): entry (r, c) = (-1)^popcount(r & c) / sqrt(G), the
+// recursion H_2n = [[H, H], [H, -H]] written out, formed in fp64 and rounded once to
+// fp32.  Grid-stride over the copies * G * G outputs.
+__global__ void wush_hadamard_kernel(int G, long long total, float* out) {
+  const double hs = 1.0 / sqrt(static_cast<double>(G));
+  const long long GG = static_cast<long long>(G) * G;
+  for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const int e = static_cast<int>(i % GG);
+    const int r = e / G, c = e - (e / G) * G;
+    out[i] = static_cast<float>((__popc(r & c) & 1) ? -hs : hs);
+  }
+}
+
 }  // namespace wush

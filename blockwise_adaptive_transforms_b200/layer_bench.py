@@ -25,7 +25,7 @@ import sys
 
 import torch
 
-from . import (hadamard_matrix, wush_gemm_mxfp4, wush_gemm_nvfp4, wush_quant_act_mx_atoms, wush_quant_act_nv_atoms,
+from . import (wush_hadamard, wush_gemm_mxfp4, wush_gemm_nvfp4, wush_quant_act_mx_atoms, wush_quant_act_nv_atoms,
                wush_quant_act_shared_mx_atoms, wush_quant_weight_mx_atoms, wush_quant_weight_nv_atoms)
 
 # (N, K) per projection kind.  The Qwen3-8B shapes are the pages' own; the other two rows
@@ -69,7 +69,7 @@ def bench_shape(M: int, N: int, K: int, device="cuda", seed=0) -> dict:
     w = (torch.randn(N, K, generator=gen) / K ** 0.5).to(device)
     C = K // 32
     T = (torch.eye(32) + 0.1 * torch.randn(C, 32, 32, generator=gen)).to(device)
-    H = hadamard_matrix(32, device)
+    H = wush_hadamard(32, device=device)
     w_bf16 = w.to(torch.bfloat16)
     cw, aw = wush_quant_weight_mx_atoms(w, T)             # offline
     cx, ax = wush_quant_act_mx_atoms(x, T)

@@ -34,7 +34,7 @@ import sys
 import numpy as np
 import torch
 
-from . import (hadamard_matrix, wush_build_transforms, wush_dequant, wush_quant_act,
+from . import (wush_hadamard, wush_build_transforms, wush_dequant, wush_quant_act,
                wush_quant_weight)
 
 FORMATS = (("mxfp4", 32), ("nvfp4", 16), ("int4", 32))
@@ -74,7 +74,7 @@ def transforms(kind: str, w: torch.Tensor, xcal: torch.Tensor, G: int, seed: int
         T = torch.eye(G, device=dev).repeat(C, 1, 1).contiguous()
         return T, T
     if kind == "H":
-        T = hadamard_matrix(G, dev).repeat(C, 1, 1).contiguous()
+        T = wush_hadamard(G, copies=C, device=dev)
         return T, T
     if kind == "R":
         T = random_orthogonal_blocks(C, G, seed, dev)

@@ -253,6 +253,19 @@ int wush_build_transforms(const float* w_f32, const void* xcal_bf16, int64_t d_o
                           float* T_xvsh, double* T_wush64, double* T_xvsh64, double* s_out,
                           wush_stream_t stream);
 
+/* Writes `copies` consecutive copies of the normalised Sylvester Hadamard matrix H of
+ * order G into out, fp32 [copies][G][G] row-major: entry (r, c) = (-1)^popcount(r & c) /
+ * sqrt(G), i.e. H_1 = [1], H_2n = [[H_n, H_n], [H_n, -H_n]] scaled by G^-1/2, so that
+ * H H^T = I.  This is the H of T = H S^-1/2 U^T W'^T (paper-graph-ui analysis, sections
+ * 3.4.4 "Hadamard" and 3.2; papernotes.org "关键设计"); one copy is the shared matrix of
+ * wush_quant_act_shared (the H+Quant comparator), `C` copies are the per-block matrices of
+ * the Hadamard-only transform.  Entries are formed in fp64 and rounded once to fp32.
+ * out: caller-owned device memory of copies * G * G floats, 4-byte aligned.
+ * Errors: WUSH_ERR_UNSUPPORTED (G not a power of two in [1, 256]), WUSH_ERR_INVALID_ARG
+ * (copies < 0 or more than 2^40 entries, out NULL with copies > 0), WUSH_ERR_MISALIGNED,
+ * WUSH_ERR_CUDA.  copies = 0 returns WUSH_OK without a launch.  Asynchronous on `stream`. */
+int wush_hadamard(int G, int64_t copies, float* out, wush_stream_t stream);
+
 /* Every wait inside the kernels is bounded in time (default 2 s).  When one expires
  * the kernel records a bit in a per-device error word and returns early; outputs of
  * that call are then unspecified.  wush_device_status() synchronises `stream`, reads
@@ -295,8 +308,11 @@ int wush_quant_act_nvfp4_onepass(const void* x_bf16, const float* T_blocks, int6
  * must not be used again in the process (wush_quant_act_nvfp4_onepass with a fresh
  * workspace still works).  All calls share the one scratch per device: calls that may
  * overlap (several streams, several host threads) race and give wrong results — use
- * wush_quant_act_nvfp4_onepass with a workspace each there.  Make the first call on each
- * device before any stream capture (it resolves the scratch address).  Requests the
+ * wush_quant_act_nvfp4_onepass with a workspace each there.  Arguments are checked
+ * first; a rejected call makes no CUDA call.  The first accepted call on a device, and
+ * the first after that device's context was reset (the library notices the new context
+ * id and takes the address again), resolves the scratch address: make it before any
+ * stream capture.  Requests the
  * one-launch path cannot take (a grid of d_in/16 x ceil(n_tok/128) CTAs that is not
  * resident at once) return WUSH_ERR_UNSUPPORTED; a current device ordinal above 63 also
  * returns WUSH_ERR_UNSUPPORTED; otherwise as wush_quant_act_nvfp4_onepass.

@@ -183,3 +183,28 @@ def test_binding_rejects_host_tensors_before_any_cuda_call():
         W.nvfp4_workspace("cpu")
     with pytest.raises(TypeError):
         W._launch_stream(None, torch.device("cpu"))
+
+
+def test_hadamard_argument_checks(lib):
+    assert lib.wush_hadamard(3, 1, A16, None) == UNSUPPORTED          # not a power of two
+    assert lib.wush_hadamard(0, 1, A16, None) == UNSUPPORTED
+    assert lib.wush_hadamard(512, 1, A16, None) == UNSUPPORTED        # above 256
+    assert lib.wush_hadamard(32, -1, A16, None) == INVALID
+    assert lib.wush_hadamard(32, 2 ** 40, A16, None) == INVALID       # more than 2^40 entries
+    assert lib.wush_hadamard(32, 1, None, None) == INVALID
+    assert lib.wush_hadamard(32, 1, A1, None) == MISALIGNED
+    assert lib.wush_hadamard(32, 0, None, None) == OK                 # nothing to write
+
+
+def test_noalloc_checks_arguments_before_any_cuda_call(lib):
+    f = lib.wush_quant_act_nvfp4_onepass_noalloc
+    assert f(None, A16, 8, 64, A16, A16, A4, None) == INVALID
+    assert f(A16, A16, 8, 64, A16, A16, None, None) == INVALID        # tensor_scale is an output
+    assert f(A16, A16, -1, 64, A16, A16, A4, None) == INVALID
+    assert f(A16, A16, 8, 40, A16, A16, A4, None) == INVALID          # d_in % 16
+    assert f(A1, A16, 8, 64, A16, A16, A4, None) == MISALIGNED
+    assert f(A16, A16, 8, 64, A16, A16, A1, None) == MISALIGNED
+    assert f(A16, A16, 0, 64, None, None, None, None) == OK           # empty batch
+    g = lib.wush_quant_act_nvfp4_onepass
+    assert g(A16, A16, 8, 64, A16, A16, A4, None, None) == INVALID    # workspace required
+    assert g(A16, A16, 8, 64, A16, A16, A4, A4, None) == MISALIGNED

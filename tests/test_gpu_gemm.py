@@ -95,7 +95,7 @@ def test_quantiser_writes_scale_atoms_directly(n_tok, d_in):
     ca, at = W.wush_quant_act_mx_atoms(x, T)
     cw, sw, _ = W.wush_quant_weight(dev(inp.w), dev(b["T_xvsh32"]), 32, "mxfp4")
     cwa, atw = W.wush_quant_weight_mx_atoms(dev(inp.w), dev(b["T_xvsh32"]))
-    H = W.hadamard_matrix(32)
+    H = W.wush_hadamard(32)
     ch, sh, _ = W.wush_quant_act_shared(x, H, 32, "mxfp4")
     cha, ath = W.wush_quant_act_shared_mx_atoms(x, H)
     torch.cuda.synchronize()

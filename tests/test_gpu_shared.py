@@ -74,3 +74,17 @@ def test_shared_matrix_shape_is_checked():
     x = torch.zeros((128, 64), dtype=torch.bfloat16, device="cuda")
     with pytest.raises(ValueError):
         W.wush_quant_act_shared(x, torch.zeros((2, 32, 32), device="cuda"), 32, "mxfp4")
+
+
+@pytest.mark.parametrize("G", [1, 2, 4, 8, 16, 32, 64, 128, 256])
+def test_device_hadamard_equals_the_oracle_matrix(G):
+    """wush_hadamard writes the oracle's normalised Sylvester matrix rounded once to fp32,
+    bit for bit, in every copy."""
+    want = O.sylvester_hadamard(G).astype(np.float32)
+    one = W.wush_hadamard(G).cpu().numpy()
+    assert one.shape == (G, G) and np.array_equal(one, want)
+    many = W.wush_hadamard(G, copies=5).cpu().numpy()
+    assert many.shape == (5, G, G)
+    for k in range(5):
+        assert np.array_equal(many[k], want)
+    assert W.wush_hadamard(G, copies=0).shape == (0, G, G)

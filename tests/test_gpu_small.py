@@ -75,7 +75,7 @@ def test_small_batches_against_the_oracle(name, fmt, G, d_in, n_tok):
 
 def test_shared_matrix_small_batch_equals_per_block_copies():
     inp, b, x, _ = _data("attn_mxfp4_4096", "mxfp4", 32, 1024, 5)
-    H = W.hadamard_matrix(32)
+    H = W.wush_hadamard(32)
     c, s, _ = W.wush_quant_act_shared(x, H, 32, "mxfp4")
     c2, s2, _ = W.wush_quant_act(x, H.repeat(32, 1, 1).contiguous(), 32, "mxfp4")
     torch.cuda.synchronize()
