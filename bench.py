@@ -4,10 +4,12 @@ attention-input workload: 4096 tokens x d_in = 4096, G = 32, bf16 activations.
 
 One step = one call of wush_quant_act over the whole 4096 x 4096 batch.  Inputs are
 resident in HBM; eight rotating input/output sets (8 x 43 MB > 126 MB L2) make every
-step read its activations from DRAM.  The timed region replays CUDA graphs of the
-launches, bracketed by a barrier + synchronize and CUDA events on the launching
-stream; under torchrun every rank runs its own batch (weak scaling) and the time is
-the maximum over ranks.
+step read its activations from DRAM.  The timed region is seven spans, each bracketed
+by a barrier + synchronize and CUDA events on the launching stream, each replaying a
+CUDA graph of back-to-back launches max(K, 20000) times over; the median span gives
+the time per step, so the figure does not depend on how small K is.  Under torchrun
+every rank runs its own batch (weak scaling) and each span's time is the maximum over
+ranks.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
 
@@ -32,8 +34,9 @@ sys.path.insert(0, ROOT)
 METRIC = "WUSH+quant GB/s & tokens/s at d=4096 G=32 MXFP4; % of HBM roofline"
 WORKLOAD = "attn_mxfp4_4096"
 N_SETS = 8
-GRAPH_LEN = 100
-H_STEPS = 5000       # launches of the H+Quant comparator timed after the main region
+GRAPH_LEN = 200          # launches per captured graph
+SPAN_MIN_LAUNCHES = 20000  # launches per timed span (about 0.2 s at this size)
+N_SPANS = 7              # timed spans; the median is reported
 FALLBACK_HBM_GBS = 6650.0
 PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "wush_fused_mxfp4_attn_4096.md")
 KERNEL_SOURCES = ("blockwise_adaptive_transforms_b200/csrc/wush_fused.cuh",
@@ -47,6 +50,8 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=2000)
     ap.add_argument("--impl", choices=("native", "reference"), default="native")
     ap.add_argument("--e2e-steps", type=int, default=30)
+    ap.add_argument("--span-launches", type=int, default=SPAN_MIN_LAUNCHES,
+                    help="least launches per timed span (a short value suits profiler runs)")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-rows", action="store_true",
@@ -173,43 +178,75 @@ class ClockSampler:
                 "samples": len(self.samples)}
 
 
-def cpu_baseline(inp, wl, seconds: float):
-    """The float64 oracle, as it stands, on the host cores: repeated calls on 256-token
-    samples of the workload for about `seconds`, scaled to the metric's bytes."""
+def _oracle_pool_init(root: str) -> None:
+    """Worker set-up: one thread per worker process (the pool supplies the parallelism)."""
+    for k in ("OMP_NUM_THREADS", "OPENBLAS_NUM_THREADS", "MKL_NUM_THREADS"):
+        os.environ[k] = "1"
+    if root not in sys.path:
+        sys.path.insert(0, root)
+
+
+def _oracle_slice(task) -> int:
+    """One bounded sample for a pool worker: the oracle's whole path on a row slice."""
+    x_bits, T32, G, fmt = task
     from oracle import wush_oracle as O
-    from threadpoolctl import threadpool_info
+    O.quant_act(x_bits, T32, G, fmt)
+    return int(x_bits.shape[0])
+
+
+def host_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def oracle_pool(n: int):
+    """A process pool of n oracle workers, started with spawn (safe after CUDA is up)."""
+    import multiprocessing as mp
+    return mp.get_context("spawn").Pool(n, initializer=_oracle_pool_init, initargs=(ROOT,))
+
+
+def _slices(x_bits, rows: int, k0: int, n: int):
+    n_tok = x_bits.shape[0]
+    return [x_bits[((k0 + j) * rows) % n_tok:((k0 + j) * rows) % n_tok + rows] for j in range(n)]
+
+
+def cpu_baseline(inp, wl, seconds: float):
+    """The float64 oracle, as it stands, on the host cores: 256-token samples of the
+    workload, on all cores (one worker process per core, each running the oracle on its
+    own slice) and on one core, about `seconds` each, scaled to the metric's bytes."""
+    from oracle import wush_oracle as O
+    from threadpoolctl import threadpool_limits
     b = O.build_transforms(inp.w, inp.xcal_bits, wl.G)
     T32 = b["T_wush32"]
     rows = 256
-    O.quant_act(inp.x_bits[:rows], T32, wl.G, wl.fmt)
-    done, t0, i = 0, time.perf_counter(), 0
-    while time.perf_counter() - t0 < seconds / 4:
-        r0 = (i * rows) % wl.n_tok
-        O.quant_act(inp.x_bits[r0:r0 + rows], T32, wl.G, wl.fmt)
-        done += rows
-        i += 1
-    dt = time.perf_counter() - t0
     per_tok = algorithmic_bytes(wl.n_tok, wl.d_in, wl.G) / wl.n_tok
-    threads = max([p.get("num_threads", 1) for p in threadpool_info()] + [1])
-    # the same sample on one core (the baseline proper, see below)
-    from threadpoolctl import threadpool_limits
-    done1, t1, j = 0, time.perf_counter(), 0
+    # one core
     with threadpool_limits(limits=1):
+        O.quant_act(inp.x_bits[:rows], T32, wl.G, wl.fmt)
+        done1, t1, j = 0, time.perf_counter(), 0
         while time.perf_counter() - t1 < seconds:
-            r0 = (j * rows) % wl.n_tok
-            O.quant_act(inp.x_bits[r0:r0 + rows], T32, wl.G, wl.fmt)
-            done1 += rows
+            done1 += _oracle_slice((_slices(inp.x_bits, rows, j, 1)[0], T32, wl.G, wl.fmt))
             j += 1
-    dt1 = time.perf_counter() - t1
-    # numpy's einsum over the block index and the elementwise quantisation run on one
-    # thread whatever the BLAS pool holds, so the one-core run is the baseline itself
-    return {"value": round(done1 / dt1 * per_tok / 1e9, 6), "unit": "GB/s", "cores": 1, "kind": "oracle",
-            "tokens_per_s": round(done1 / dt1, 1),
-            "with_thread_pool": {"value": round(done / dt * per_tok / 1e9, 6), "tokens_per_s": round(done / dt, 1),
-                                 "threads": threads},
+        dt1 = time.perf_counter() - t1
+    # every core: one slice per worker per round
+    n = host_cores()
+    with oracle_pool(n) as pool:
+        pool.map(_oracle_slice, [(x, T32, wl.G, wl.fmt) for x in _slices(inp.x_bits, rows, 0, n)])
+        done, t0, k = 0, time.perf_counter(), 0
+        while time.perf_counter() - t0 < seconds:
+            done += sum(pool.map(_oracle_slice, [(x, T32, wl.G, wl.fmt) for x in _slices(inp.x_bits, rows, k, n)]))
+            k += n
+        dt = time.perf_counter() - t0
+    return {"value": round(done / dt * per_tok / 1e9, 6), "unit": "GB/s", "cores": n, "kind": "oracle",
+            "tokens_per_s": round(done / dt, 1),
+            "one_core": {"value": round(done1 / dt1 * per_tok / 1e9, 6), "tokens_per_s": round(done1 / dt1, 1),
+                         "cores": 1},
             "cpu_model": _cpu_model(),
-            "sample": f"{done1} tokens in {rows}-token slices of the {wl.n_tok}x{wl.d_in} workload on one core, "
-                      f"{dt1:.1f} s ({done} tokens in {dt:.1f} s with a {threads}-thread pool); bytes scaled per token"}
+            "sample": f"{done} tokens in {rows}-token slices of the {wl.n_tok}x{wl.d_in} workload on {n} worker "
+                      f"processes (one per core), {dt:.1f} s; one core: {done1} tokens in {dt1:.1f} s; "
+                      f"bytes scaled per token"}
 
 
 def _cpu_model() -> str:
@@ -224,40 +261,42 @@ def _cpu_model() -> str:
 
 
 def run_reference(args):
-    """--impl reference: the float64 CPU oracle, on rank 0 only."""
+    """--impl reference: the float64 CPU oracle on every host core, rank 0 only.  Each
+    step is one bounded sample: a row slice per core, run by one worker process each."""
     if int(os.environ.get("RANK", "0")) != 0:
         return
     from workloads import make_inputs, workload
     from oracle import wush_oracle as O
-    from threadpoolctl import threadpool_limits
     wl = workload(WORKLOAD)
     inp = make_inputs(wl)
     b = O.build_transforms(inp.w, inp.xcal_bits, wl.G)
     T32 = b["T_wush32"]
-    limit = threadpool_limits(limits=1)   # the oracle's steps run on one thread anyway
+    n = host_cores()
     total = max(1, args.steps + args.warmup)
+    # about 0.22 ms of one core per token: keep the whole run near a minute or less
     rows = max(1, min(256, int(60.0 / (total * 2.5e-4))))
     per_tok = algorithmic_bytes(wl.n_tok, wl.d_in, wl.G) / wl.n_tok
-    for i in range(args.warmup):
-        r0 = (i * rows) % wl.n_tok
-        O.quant_act(inp.x_bits[r0:r0 + rows], T32, wl.G, wl.fmt)
-    t0 = time.perf_counter()
-    for i in range(args.steps):
-        r0 = (i * rows) % wl.n_tok
-        O.quant_act(inp.x_bits[r0:r0 + rows], T32, wl.G, wl.fmt)
-    dt = time.perf_counter() - t0
-    limit.restore_original_limits()
-    toks = rows * args.steps
+    with oracle_pool(n) as pool:
+        def step(k):
+            return sum(pool.map(_oracle_slice, [(x, T32, wl.G, wl.fmt) for x in _slices(inp.x_bits, rows, k * n, n)]))
+        step(0)
+        for i in range(args.warmup):
+            step(i)
+        toks, t0 = 0, time.perf_counter()
+        for i in range(args.steps):
+            toks += step(i)
+        dt = time.perf_counter() - t0
     value = toks / dt * per_tok / 1e9
-    sample = f"{rows} tokens per step of the {wl.n_tok}x{wl.d_in} workload on one core; bytes scaled per token"
+    sample = (f"{rows} tokens per core per step ({n} worker processes, one per core) of the "
+              f"{wl.n_tok}x{wl.d_in} workload; bytes scaled per token")
     line = {"impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "GB/s",
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(dt / args.steps * 1e3, 4), "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "tokens_per_s": round(toks / dt, 1),
             "config": {"workload": WORKLOAD, "tokens": wl.n_tok, "d_in": wl.d_in, "G": wl.G, "fmt": wl.fmt},
-            "cpu_baseline": {"value": round(value, 6), "unit": "GB/s", "cores": 1, "kind": "oracle",
-                             "sample": sample},
+            "cpu_baseline": {"value": round(value, 6), "unit": "GB/s", "cores": n, "kind": "oracle",
+                             "cpu_model": _cpu_model(), "sample": sample},
             "e2e": {"value": round(value, 6), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -439,94 +478,81 @@ def run_native(args):
         k = i % N_SETS
         W.wush_quant_act(xs[k], T, G, wl.fmt, codes=codes[k], scales=scales[k], stream=stream)
 
-    # warm-up: eager launches, then capture the graphs
-    with torch.cuda.stream(stream):
-        for i in range(min(args.warmup, 64)):
-            launch(i)
-        stream.synchronize()
-        graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(graph, stream=stream):
-            for i in range(GRAPH_LEN):
-                launch(i)
-        rem = args.steps % GRAPH_LEN
-        tail = None
-        if rem:
-            tail = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(tail, stream=stream):
-                for i in range(rem):
-                    launch(i)
-        done = min(args.warmup, 64)
-        while done < args.warmup:
-            graph.replay()
-            done += GRAPH_LEN
-        graph.replay()                      # each graph once before the timed region: its
-        if tail is not None:                # first replay uploads it to the device
-            tail.replay()
-        stream.synchronize()
+    span_launches = -(-max(args.steps, args.span_launches) // GRAPH_LEN) * GRAPH_LEN
+
+    def capture(fn):
+        """Warm-up launches, then one graph of GRAPH_LEN launches, replayed once (its first
+        replay uploads it to the device)."""
+        with torch.cuda.stream(stream):
+            for i in range(min(max(args.warmup, 3), 64)):
+                fn(i)
+            stream.synchronize()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                for i in range(GRAPH_LEN):
+                    fn(i)
+            done = min(max(args.warmup, 3), 64)
+            while done < args.warmup:
+                g.replay()
+                done += GRAPH_LEN
+            g.replay()
+            stream.synchronize()
+        return g
+
+    def timed_spans(g):
+        """N_SPANS spans of span_launches launches each, every span bracketed by a barrier
+        + synchronize and events on the launching stream; seconds per span, max over ranks."""
+        out = []
+        for _ in range(N_SPANS):
+            if world > 1:
+                dist.barrier()
+            torch.cuda.synchronize()
+            t0 = torch.cuda.Event(enable_timing=True)
+            t1 = torch.cuda.Event(enable_timing=True)
+            with torch.cuda.stream(stream):
+                t0.record(stream)
+                for _ in range(span_launches // GRAPH_LEN):
+                    g.replay()
+                t1.record(stream)
+            t1.synchronize()
+            out.append(max_over_ranks(t0.elapsed_time(t1) / 1e3, dev))
+        return out
+
+    graph = capture(launch)
     st, bits = W.wush_device_status(stream)
     if st != 0:
         raise RuntimeError(f"device error word {bits:#x} after warm-up")
-
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
     with ClockSampler(local) as clocks:
-        with torch.cuda.stream(stream):
-            e0.record(stream)
-            for _ in range(args.steps // GRAPH_LEN):
-                graph.replay()
-            if tail is not None:
-                tail.replay()
-            e1.record(stream)
-        e1.synchronize()
+        spans = timed_spans(graph)
     torch.cuda.synchronize()
-    elapsed_s = max_over_ranks(e0.elapsed_time(e1) / 1e3, dev)
     if world > 1:
         dist.barrier()
     st, bits = W.wush_device_status(stream)
     if st != 0:
         raise RuntimeError(f"device error word {bits:#x} after the timed region")
+    del graph
+    span_s = statistics.median(spans)
+    per_launch_s = span_s / span_launches
+    elapsed_s = per_launch_s * args.steps          # K steps at the median span's rate
+    value = job_throughput(world, span_launches, step_bytes, span_s)
 
-    per_launch_s = elapsed_s / args.steps
-    value = job_throughput(world, args.steps, step_bytes, elapsed_s)
-
-    # H+Quant comparator: the same kernel with one shared G x G Hadamard matrix, same
-    # inputs, outputs and timing method (the pages compare the two fused kernels)
-    H = W.hadamard_matrix(G, dev)
+    # H+Quant comparator: the same kernel with one shared G x G Hadamard matrix (written
+    # by the library), same inputs, outputs, launch count and timing method (the pages
+    # compare the two fused kernels)
+    H = W.wush_hadamard(G, device=dev)
 
     def launch_h(i):
         k = i % N_SETS
         W.wush_quant_act_shared(xs[k], H, G, wl.fmt, codes=codes[k], scales=scales[k], stream=stream)
 
-    h_reps = max(1, min(args.steps, H_STEPS) // GRAPH_LEN)
-    with torch.cuda.stream(stream):
-        for i in range(8):
-            launch_h(i)
-        stream.synchronize()
-        graph_h = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(graph_h, stream=stream):
-            for i in range(GRAPH_LEN):
-                launch_h(i)
-        graph_h.replay()
-        stream.synchronize()
-        if world > 1:
-            dist.barrier()
-        h0 = torch.cuda.Event(enable_timing=True)
-        h1 = torch.cuda.Event(enable_timing=True)
-        h0.record(stream)
-        for _ in range(h_reps):
-            graph_h.replay()
-        h1.record(stream)
-        h1.synchronize()
-    h_elapsed = max_over_ranks(h0.elapsed_time(h1) / 1e3, dev)
-    h_per_launch_s = h_elapsed / (h_reps * GRAPH_LEN)
+    graph_h = capture(launch_h)
+    h_spans = timed_spans(graph_h)
+    del graph_h
+    h_per_launch_s = statistics.median(h_spans) / span_launches
     h_bytes = step_bytes - C * G * G * 4 + G * G * 4
     st, bits = W.wush_device_status(stream)
     if st != 0:
         raise RuntimeError(f"device error word {bits:#x} after the H+Quant timing")
-    del graph_h
     tokens_s = world * args.steps * n / elapsed_s
     achieved = step_bytes / per_launch_s / 1e9
     peak, peak_kind = hbm_peak()
@@ -598,13 +624,17 @@ def run_native(args):
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(per_launch_s * 1e3, 6),
+        "launches_timed": N_SPANS * span_launches,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
         "tokens_per_s": round(tokens_s, 1),
         "hbm_roofline_frac": round(achieved / peak, 4),
         "config": {"workload": WORKLOAD, "tokens": n, "d_in": d, "G": G, "fmt": wl.fmt,
                    "l2": f"{N_SETS} rotating input/output sets ({N_SETS * step_bytes / 1e6:.0f} MB > 126 MB L2)",
-                   "launch": f"CUDA graphs of {GRAPH_LEN} launches", "transform_build_ms": round(build_ms, 2)},
+                   "launch": f"CUDA graphs of {GRAPH_LEN} back-to-back launches",
+                   "timing": f"median of {N_SPANS} spans of {span_launches} launches each "
+                             f"(span times {', '.join(f'{1e6 * t / span_launches:.3f}' for t in spans)} us per launch)",
+                   "transform_build_ms": round(build_ms, 2)},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "traffic": measured_traffic(),
                      "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
@@ -613,13 +643,13 @@ def run_native(args):
         "e2e": {"value": round(e2e_value, 3), "unit": "GB/s", "h2d_bytes_per_step": n * d * 2,
                 "d2h_bytes_per_step": n * d // 2 + n * C, "steps": args.e2e_steps,
                 "overlap": "each step's copy in, kernel and copy out on three streams, beside its neighbours"},
-        "h_quant": {"value": round(job_throughput(world, h_reps * GRAPH_LEN, h_bytes, h_elapsed), 2),
+        "h_quant": {"value": round(world * h_bytes / h_per_launch_s / 1e9, 2),
                     "unit": "GB/s", "us_per_launch": round(h_per_launch_s * 1e6, 3),
-                    "launches": h_reps * GRAPH_LEN,
+                    "launches": N_SPANS * span_launches,
                     "wush_time_over_h_time": round(per_launch_s / h_per_launch_s, 4),
                     "what": "same fused kernel, one shared Hadamard matrix for every block"},
         "rows": rows,
-        "gpu_launches": args.steps,
+        "gpu_launches": N_SPANS * span_launches,
         "clocks": clk,
     }
     print(json.dumps(line), flush=True)

@@ -3,6 +3,8 @@
 ``python -m blockwise_adaptive_transforms_b200.profile_case --fmt mxfp4 --rows 16384 --d-in 8192``
 quantises seeded bf16 activations (near-identity per-block transforms) ``--launches``
 times on one stream, after ``--warmup`` untimed calls, and checks the device error word.
+``--sets N`` rotates over N input/output sets, so that, as in the benchmark, each call
+reads its input from DRAM and the previous calls' outputs are written back while it runs.
 Use ``ncu -k regex:wush_fused_kernel -s <warmup launches>`` to capture the timed calls.
 """
 from __future__ import annotations
@@ -23,15 +25,17 @@ def main(argv=None) -> None:
     ap.add_argument("--d-in", type=int, default=8192)
     ap.add_argument("--warmup", type=int, default=2)
     ap.add_argument("--launches", type=int, default=2)
+    ap.add_argument("--sets", type=int, default=1)
     args = ap.parse_args(argv)
     G = GROUP[args.fmt]
     C = args.d_in // G
     g = torch.Generator().manual_seed(0)
-    x = torch.randn(args.rows, args.d_in, generator=g).to(torch.bfloat16).cuda()
+    xs = [torch.randn(args.rows, args.d_in, generator=g).to(torch.bfloat16).cuda() for _ in range(args.sets)]
     T = (torch.eye(G).repeat(C, 1, 1) + 0.05 * torch.randn(C, G, G, generator=g)).float().cuda()
-    out = W.wush_quant_act(x, T, G, args.fmt)
-    for _ in range(args.warmup + args.launches - 1):
-        W.wush_quant_act(x, T, G, args.fmt, codes=out[0], scales=out[1], tensor_scale=out[2])
+    outs = [W.wush_quant_act(x, T, G, args.fmt) for x in xs]
+    for i in range(args.sets, args.warmup + args.launches):
+        k = i % args.sets
+        W.wush_quant_act(xs[k], T, G, args.fmt, codes=outs[k][0], scales=outs[k][1], tensor_scale=outs[k][2])
     torch.cuda.synchronize()
     st, bits = W.wush_device_status()
     if st != 0:
