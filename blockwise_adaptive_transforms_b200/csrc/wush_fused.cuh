@@ -760,6 +760,12 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
     if (store_leader && p.codes_via_tma) bulk_wait_read_all();
   }
 
+  // Every warp reconverges before the CTA-wide barrier: the producer and MMA roles ran on
+  // one lane, and an aligned barrier reached by a diverged warp did not hold the late
+  // lane's warp-mates back (observed on B200: the producer lane passed it while the
+  // epilogue warps were still at work).  TMEM is released only after every warp, the
+  // epilogue's last accumulator reads included, has passed it.
+  __syncwarp();
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {

@@ -10,7 +10,10 @@ namespace wush {
 
 // Device-wide error word, read and cleared by wush_device_status().  Bits:
 //   1 producer wait expired, 2 MMA wait expired, 4 converter wait expired,
-//   8 epilogue wait expired, 16 drain wait expired, 32 self-test wait expired.
+//   8 epilogue wait expired, 16 drain wait expired, 32 self-test wait expired,
+//   64 a Cholesky pivot of the transform builder was not positive, 128 a CTA of the
+//   one-launch NVFP4 path gave up waiting for the rest of its grid (its workspace,
+//   or the no-alloc scratch, is then left non-zero).
 // Defined here because the library is a single translation unit (wush_api.cu).
 __device__ unsigned int g_wush_device_error = 0u;
 
