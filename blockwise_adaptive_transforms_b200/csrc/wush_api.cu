@@ -201,11 +201,12 @@ int launch_fused(const CUtensorMap& map, const CUtensorMap& cmap, wush::FusedPar
       }
     }
   }
-  // Input tiles each CTA warms in L2 before its dependency wait.  Measured on B200: one
-  // for runs of a few tiles per CTA (4096 x 4096 MXFP4: 9.93 -> 9.65 us; two 9.77, three
-  // 10.0, all seven 11.3, as the prefetches still in flight delay the first loads), three
-  // for long runs, whose predecessor ends over a longer window (16384 x 8192: 74.8 -> 73.0).
-  p.prefetch_tiles = p.total_tiles / grid >= 32 ? 3 : 1;
+  // Input tiles each CTA warms in L2 before its dependency wait.  Measured on B200: two for
+  // runs of a few tiles per CTA (4096 x 4096 MXFP4 with the short runs on the last CTAs:
+  // 9.81 us with one, 9.75 with two; deeper prefetches still in flight delay the first
+  // loads), three for long runs, whose predecessor ends over a longer window (16384 x 8192:
+  // 74.8 -> 73.0).
+  p.prefetch_tiles = p.total_tiles / grid >= 32 ? 3 : 2;
   // programmatic stream serialisation: the CTAs may be scheduled while the previous kernel
   // in the stream drains; they do their set-up and then wait (griddepcontrol.wait) for it
   // to complete before reading any input

@@ -107,7 +107,8 @@ struct FusedCfg {
   // tload[2], tread[2]
   static constexpr int N_BARS = 2 * STAGES + 13 + 2 * NACC;
   static constexpr int OFF_MISC = OFF_BAR + 8 * N_BARS;
-  static constexpr int SMEM_BYTES = OFF_MISC + 64 + 1024;   // + alignment slack
+  static constexpr int OFF_NVTAB = OFF_MISC + 64;     // NVFP4: 128 fp32 scale reciprocals
+  static constexpr int SMEM_BYTES = OFF_NVTAB + 512 + 1024;   // + alignment slack
   static_assert(G == 16 || G == 32, "G must be 16 or 32");
   static_assert(!(SHARED_T && IN_F32), "the shared-matrix variant is an activation path");
   static_assert(!(FMT == kMXFP4 && G != 32) && !(FMT == kNVFP4 && G != 16), "format/group mismatch");
@@ -233,6 +234,47 @@ __device__ __forceinline__ uint32_t quant_nv(const float* v, float s_t, float d6
   return sb;
 }
 
+// The same NVFP4 group quantiser with the per-call constants of its scale chain hoisted:
+//  * r = fl32(amax / d6) by Markstein's correction of a reciprocal product (P. Markstein,
+//    IBM J. Res. Dev. 34(1), 1990; see also Muller et al., Handbook of Floating-Point
+//    Arithmetic, the theorem on division by fused multiply-add): with inv_d6 = RN(1/d6),
+//    q = RN(amax * inv_d6) is within one ulp of the quotient, the residual amax - q * d6 is
+//    exact in one FMA, and RN(q + residual * inv_d6) is the correctly rounded quotient,
+//    for normal results.  A quotient below the fp32 normal range is far below E4M3's
+//    smallest step (2^-9) and encodes as 0 either way; one far above 448 saturates either
+//    way.  `exact_div` selects the division
+//    itself when inv_d6 is not a normal number (d6 = 0 or extreme);
+//  * inv = fl32(1 / fl32(dec(sb) * s_t)) is looked up in a table of the 128 possible block
+//    scale bytes, filled once per CTA with those very operations.
+// The results are bit-identical to quant_nv.
+template <int NV>
+__device__ __forceinline__ uint32_t quant_nv_tab(const float* v, float d6, float inv_d6, bool exact_div,
+                                                 const float* inv_tab, uint32_t* words) {
+  const float amax = group_absmax<NV>(v);
+  float r;
+  if (exact_div) {
+    r = d6 > 0.0f ? __fdiv_rn(amax, d6) : 0.0f;
+  } else {
+    const float q = __fmul_rn(amax, inv_d6);
+    const float res = __fmaf_rn(-q, d6, amax);
+    // far above E4M3's largest value (a caller's tensor scale below amax / 2688) the
+    // quotient only needs to saturate, and the correction could overflow
+    r = q <= 1048576.0f ? __fmaf_rn(res, inv_d6, q) : q;
+  }
+  const uint32_t sb = e4m3_byte(r);
+  const float inv = inv_tab[sb & 127u];
+  float w[NV];
+#pragma unroll
+  for (int j = 0; j < NV; j += 2) {   // each product rounded to fp32
+    w[j] = v[j];
+    w[j + 1] = v[j + 1];
+    mul2_rn(w[j], w[j + 1], inv);
+  }
+#pragma unroll
+  for (int k = 0; k < NV / 8; ++k) words[k] = e2m1_pack8(w + 8 * k);
+  return sb;
+}
+
 // INT4 symmetric: s = amax / 7, q = clamp(rne(y * (1/s)), -7, 7), two's-complement nibbles.
 template <int NV>
 __device__ __forceinline__ float quant_int4(const float* v, uint32_t* words) {
@@ -282,8 +324,13 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int total = p.total_tiles, nrt = p.n_row_tiles;
-  const int t_begin = static_cast<int>(static_cast<long long>(blockIdx.x) * total / gridDim.x);
-  const int t_end = static_cast<int>(static_cast<long long>(blockIdx.x + 1) * total / gridDim.x);
+  // Runs of total / grid tiles, one longer for the first total % grid CTAs.  The CTAs with
+  // the highest indices are dispatched last, onto the SMs the previous kernel frees last,
+  // and so start late: they take the short runs.
+  const int run_s = total / static_cast<int>(gridDim.x), n_long = total - run_s * static_cast<int>(gridDim.x);
+  const int bx = static_cast<int>(blockIdx.x);
+  const int t_begin = bx < n_long ? bx * (run_s + 1) : n_long * (run_s + 1) + (bx - n_long) * run_s;
+  const int t_end = t_begin + run_s + (bx < n_long ? 1 : 0);
   const uint64_t lim = p.wait_limit_ns;
 
   if (threadIdx.x == 0) {
@@ -343,37 +390,60 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
     mbar_arrive_expect_tx(BAR(B_TLOAD + slot), bytes);
     bulk_load_1d(sbase + Cfg::OFF_T + slot * Cfg::TSLOT_BYTES, src, bytes, BAR(B_TLOAD + slot));
   };
-  // raw fp32 chunks of a slot -> registers
+  // one 8-value chunk q of a slot's raw fp32 matrices -> registers (the shared-matrix
+  // variant reads the one matrix for every block)
+  auto load_chunk = [&](int q, const uint8_t* slot_raw, float4& a, float4& b) {
+    const int qs = Cfg::SHARED_T ? q % (G * (G / 8)) : q;
+    const float4* src = reinterpret_cast<const float4*>(slot_raw + qs * 32);
+    a = src[0];
+    b = src[1];
+  };
+  // its hi/lo split into the K-major SW128 panels of the slot
+  auto store_chunk = [&](int q, const float4& a, const float4& b4, uint8_t* tdst) {
+    const int b = q / (G * (G / 8));
+    const int rem = q - b * (G * (G / 8));
+    const int r = rem / (G / 8), j = rem - r * (G / 8);
+    const float vals[8] = {a.x, a.y, a.z, a.w, b4.x, b4.y, b4.z, b4.w};
+    uint4 hi, lo;
+    split8(vals, hi, lo);
+    uint8_t* panel = tdst + (b / Cfg::BPP) * Cfg::PANEL_BYTES;
+    const int c = (b % Cfg::BPP) * (G / 8) + j;     // 16-byte chunk along K
+    *reinterpret_cast<uint4*>(panel + sw128_off(r, c)) = hi;
+    *reinterpret_cast<uint4*>(panel + sw128_off(G + r, c)) = lo;
+  };
+  // raw fp32 chunks of a slot -> registers (converter id v takes v, v + 64, ...)
   auto read_T = [&](int v, const uint8_t* slot_raw, float4 (&u)[T_PER_THREAD][2]) {
 #pragma unroll
-    for (int k = 0; k < T_PER_THREAD; ++k) {
-      const int q = v + 64 * k;
-      const int qs = Cfg::SHARED_T ? q % (G * (G / 8)) : q;   // shared: every block reads the one matrix
-      if (q < T_CHUNKS) {
-        const float4* src = reinterpret_cast<const float4*>(slot_raw + qs * 32);
-        u[k][0] = src[0];
-        u[k][1] = src[1];
-      }
-    }
+    for (int k = 0; k < T_PER_THREAD; ++k)
+      if (v + 64 * k < T_CHUNKS) load_chunk(v + 64 * k, slot_raw, u[k][0], u[k][1]);
   };
-  // hi/lo split of the chunks into the K-major SW128 panels of the slot
   auto store_T = [&](int v, const float4 (&u)[T_PER_THREAD][2], uint8_t* tdst) {
 #pragma unroll
-    for (int k = 0; k < T_PER_THREAD; ++k) {
-      const int q = v + 64 * k;
-      if (q >= T_CHUNKS) break;
-      const int b = q / (G * (G / 8));
-      const int rem = q - b * (G * (G / 8));
-      const int r = rem / (G / 8), j = rem - r * (G / 8);
-      const float vals[8] = {u[k][0].x, u[k][0].y, u[k][0].z, u[k][0].w,
-                             u[k][1].x, u[k][1].y, u[k][1].z, u[k][1].w};
-      uint4 hi, lo;
-      split8(vals, hi, lo);
-      uint8_t* panel = tdst + (b / Cfg::BPP) * Cfg::PANEL_BYTES;
-      const int c = (b % Cfg::BPP) * (G / 8) + j;     // 16-byte chunk along K
-      *reinterpret_cast<uint4*>(panel + sw128_off(r, c)) = hi;
-      *reinterpret_cast<uint4*>(panel + sw128_off(G + r, c)) = lo;
-    }
+    for (int k = 0; k < T_PER_THREAD; ++k)
+      if (v + 64 * k < T_CHUNKS) store_chunk(v + 64 * k, u[k][0], u[k][1], tdst);
+  };
+  // On the bf16 path the first column tile's matrices are split by the converter and the
+  // epilogue warps together (warps 2-11, at most two chunks per thread): the first MMA
+  // waits for this split, and the epilogue has nothing to do before the first
+  // accumulator lands.  Both roles call it exactly once; the named barriers are reached
+  // whether or not the copy arrived in time.
+  constexpr int NC0 = 320;
+  constexpr int PER0 = (T_CHUNKS + NC0 - 1) / NC0;
+  auto first_split = [&]() -> bool {
+    const int c0 = static_cast<int>(threadIdx.x) - 64;
+    uint8_t* tdst = smem + Cfg::OFF_T;
+    const bool ok = wait_bounded(BAR(B_TLOAD), 0u, abort_flag, 4u, lim);
+    float4 u[PER0][2];
+#pragma unroll
+    for (int k = 0; k < PER0; ++k)
+      if (ok && c0 + NC0 * k < T_CHUNKS) load_chunk(c0 + NC0 * k, tdst, u[k][0], u[k][1]);
+    named_bar_sync(4, NC0);   // every raw chunk is in registers before any panel overwrites it
+#pragma unroll
+    for (int k = 0; k < PER0; ++k)
+      if (ok && c0 + NC0 * k < T_CHUNKS) store_chunk(c0 + NC0 * k, u[k][0], u[k][1], tdst);
+    fence_proxy_async_smem();
+    named_bar_sync(4, NC0);   // the panels are complete
+    return ok;
   };
   // Thread 0, which initialised the barriers, issues the first input tile, then the
   // transform copies of the CTA's first (and, if its tiles reach it, second) column tile,
@@ -516,9 +586,19 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
     int epoch = -1, prev_ct = -1;
     int stage = 0, obuf = 0;
     uint32_t phase = 0, ophase = 0;
-    for (int t = t_begin; t < t_end; ++t) {
+    bool conv_ok = true;
+    if (!Cfg::IN_F32 && t_begin < t_end) {
+      conv_ok = first_split();
+      if (conv_ok) {
+        mbar_arrive(BAR(B_TFULL));   // slot 0 holds the first column tile's panels
+        t_landed[0] = 1;
+        epoch = 0;
+        prev_ct = t_begin / nrt;
+      }
+    }
+    for (int t = t_begin; conv_ok && t < t_end; ++t) {
       const int ct = t / nrt;
-      if (t_conv && (Cfg::SHARED_T ? t == t_begin : ct != prev_ct)) {
+      if (t_conv && (Cfg::SHARED_T ? epoch < 0 : ct != prev_ct)) {
         ++epoch;
         prev_ct = ct;
         const int slot = epoch & 1;
@@ -588,10 +668,24 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
     const int code_row_bytes = p.d_in / 2;
     const bool vec16 = (code_row_bytes % 16) == 0;
     using ScaleT = typename std::conditional<Cfg::FMT == kINT4, float, uint8_t>::type;
-    float s_t = 0.0f, d6 = 0.0f;
-    if (Cfg::FMT == kNVFP4 && !Cfg::AMAX_ONLY) {
+    if (!Cfg::IN_F32 && t_begin < t_end) first_split();   // with the converter warps
+    float s_t = 0.0f, d6 = 0.0f, inv_d6 = 0.0f;
+    bool exact_div = true;
+    float* nv_tab = reinterpret_cast<float*>(smem + Cfg::OFF_NVTAB);
+    if constexpr (Cfg::FMT == kNVFP4 && !Cfg::AMAX_ONLY) {
       s_t = *p.tensor_scale;
       d6 = __fmul_rn(6.0f, s_t);
+      inv_d6 = d6 > 0.0f ? __frcp_rn(d6) : 0.0f;
+      exact_div = !(inv_d6 >= 1.17549435e-38f && inv_d6 <= 3.40282347e+38f);   // not a normal fp32
+      // the 128 block-scale reciprocals, one per thread of the first 128 epilogue threads
+      const int e_tid = threadIdx.x - 128;
+      if (e_tid < 128) {
+        const float S = __fmul_rn(e4m3_value(static_cast<uint32_t>(e_tid)), s_t);
+        float inv = S > 0.0f ? __frcp_rn(S) : 0.0f;
+        if (isinf(inv)) inv = 0.0f;
+        nv_tab[e_tid] = inv;
+      }
+      named_bar_sync(3, 128 * Cfg::N_GROUPS);   // the table is complete
     }
     bool live = true;
     float run_max = 0.0f;
@@ -648,7 +742,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
               for (int k = 0; k < G / 4; ++k) yd[k] = make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
             }
             if (Cfg::FMT == kMXFP4) sc[b] = static_cast<ScaleT>(quant_mx<G>(v, words[u]));
-            else if (Cfg::FMT == kNVFP4) sc[b] = static_cast<ScaleT>(quant_nv<G>(v, s_t, d6, words[u]));
+            else if (Cfg::FMT == kNVFP4) sc[b] = static_cast<ScaleT>(quant_nv_tab<G>(v, d6, inv_d6, exact_div, nv_tab, words[u]));
             else sc[b] = static_cast<ScaleT>(quant_int4<G>(v, words[u]));
           }
           // the load's 32 elements are one 16-byte chunk of this row's codes

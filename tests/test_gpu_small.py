@@ -118,3 +118,29 @@ def test_small_batches_write_scale_atoms(fmt, n_tok, d_in):
     if fmt == "nvfp4":
         assert torch.equal(ts, tsa)
     assert np.array_equal(at.cpu().numpy(), O.scale_atoms(s.cpu().numpy()))
+
+
+def test_narrow_layer_rule2_statistic():
+    """Rule 2 on a deliberately narrow layer (transforms from 128 output channels), the
+    case where a single legitimate one-step flip of a top-magnitude NVFP4 code moves the
+    relative Frobenius error past 2e-3.  The flip budget and the one-step bound still hold;
+    the Frobenius figure is recorded (printed) and held to the 4e-3 that one such flip in
+    this batch can produce, not to 2e-3 (the other tests build their transforms from
+    realistically wide layers)."""
+    from parity_rules import end_to_end_report
+    wl = workload("mlp_down_nvfp4_14336", n_tok=64, d_in=1040, d_out=128, n_cal=512)
+    inp = make_inputs(wl)
+    b = O.build_transforms(inp.w, inp.xcal_bits, 16)
+    x = torch.from_numpy(np.ascontiguousarray(inp.x_bits).view(np.int16)).cuda().view(torch.bfloat16)
+    T = torch.from_numpy(b["T_wush32"]).cuda()
+    W.wush_set_small_batch_rows(0)                 # the tensor-core kernel (hi/lo split)
+    c, s, ts = W.wush_quant_act(x, T, 16, "nvfp4")
+    torch.cuda.synchronize()
+    st, bits = W.wush_device_status()
+    assert st == 0 and bits == 0, f"device error word {bits:#x}"
+    y_ref = O.block_transform(O.bf16_to_f64(inp.x_bits), b["T_wush32"].astype(np.float64))
+    rel, frac, nsd, mx = end_to_end_report(c.cpu().numpy(), s.cpu().numpy(), ts.item(), y_ref, "nvfp4", 16)
+    print(f"narrow layer (128 outputs), NVFP4 64 x 1040: rel-Frobenius {rel:.3e}, "
+          f"codes differing {frac:.3e}, groups with a different scale {nsd}, max steps {mx}")
+    assert mx <= 1 and frac <= 1e-3
+    assert rel <= 4e-3
