@@ -4,9 +4,9 @@ attention-input workload: 4096 tokens x d_in = 4096, G = 32, bf16 activations.
 
 One step = one call of wush_quant_act over the whole 4096 x 4096 batch.  Inputs are
 resident in HBM; eight rotating input/output sets (8 x 43 MB > 126 MB L2) make every
-step read its activations from DRAM.  The timed region is seven spans, each bracketed
+step read its activations from DRAM.  The timed region is nine spans, each bracketed
 by a barrier + synchronize and CUDA events on the launching stream, each replaying a
-CUDA graph of back-to-back launches max(K, 20000) times over; the median span gives
+CUDA graph of back-to-back launches max(K, 4000) times over; the median span gives
 the time per step, so the figure does not depend on how small K is.  Under torchrun
 every rank runs its own batch (weak scaling) and each span's time is the maximum over
 ranks.
@@ -34,9 +34,9 @@ sys.path.insert(0, ROOT)
 METRIC = "WUSH+quant GB/s & tokens/s at d=4096 G=32 MXFP4; % of HBM roofline"
 WORKLOAD = "attn_mxfp4_4096"
 N_SETS = 8
-GRAPH_LEN = 200          # launches per captured graph
-SPAN_MIN_LAUNCHES = 20000  # launches per timed span (about 0.2 s at this size)
-N_SPANS = 7              # timed spans; the median is reported
+GRAPH_LEN = 1000         # launches per captured graph
+SPAN_MIN_LAUNCHES = 4000   # launches per timed span (about 40 ms at this size)
+N_SPANS = 9              # timed spans; the median is reported
 FALLBACK_HBM_GBS = 6650.0
 PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "wush_fused_mxfp4_attn_4096.md")
 KERNEL_SOURCES = ("blockwise_adaptive_transforms_b200/csrc/wush_fused.cuh",
