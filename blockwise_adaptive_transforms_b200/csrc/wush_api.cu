@@ -45,6 +45,9 @@ static_assert(kOnepassWorkspaceWords <= kNoAllocScratchWords, "scratch too small
 #ifndef WUSH_USE_PDL
 #define WUSH_USE_PDL 1
 #endif
+#ifndef WUSH_NV_REVERSE
+#define WUSH_NV_REVERSE true
+#endif
 
 namespace {
 
@@ -172,7 +175,7 @@ int encode_u8_sw128(CUtensorMap* map, const void* base, int64_t rows, int64_t co
   return r == CUDA_SUCCESS ? WUSH_OK : cuda_fail(r, "cuTensorMapEncodeTiled", __LINE__, true);
 }
 
-template <class Cfg>
+template <class Cfg, bool REV = false>
 int launch_fused(const CUtensorMap& map, const CUtensorMap& cmap, wush::FusedParams p, cudaStream_t stream) {
   int dev = 0, sms = 0;
   WUSH_CUDA_CHECK(cudaGetDevice(&dev));
@@ -180,7 +183,7 @@ int launch_fused(const CUtensorMap& map, const CUtensorMap& cmap, wush::FusedPar
   static std::atomic<unsigned long long> configured{0ull};   // one bit per device ordinal
   const unsigned long long bit = 1ull << (dev & 63);
   if (!(configured.load(std::memory_order_acquire) & bit)) {
-    WUSH_CUDA_CHECK(cudaFuncSetAttribute(wush::wush_fused_kernel<Cfg>,
+    WUSH_CUDA_CHECK(cudaFuncSetAttribute(wush::wush_fused_kernel<Cfg, REV>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES));
     configured.fetch_or(bit, std::memory_order_acq_rel);
   }
@@ -220,7 +223,7 @@ int launch_fused(const CUtensorMap& map, const CUtensorMap& cmap, wush::FusedPar
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   lc.attrs = attr;
   lc.numAttrs = WUSH_USE_PDL ? 1 : 0;
-  WUSH_CUDA_CHECK(cudaLaunchKernelEx(&lc, wush::wush_fused_kernel<Cfg>, map, cmap, p));
+  WUSH_CUDA_CHECK(cudaLaunchKernelEx(&lc, wush::wush_fused_kernel<Cfg, REV>, map, cmap, p));
   return launch_status(__LINE__);
 }
 
@@ -241,11 +244,11 @@ int launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, cudaStream_t s, Ar
   return launch_status(__LINE__);
 }
 
-template <int G, int FMT, bool IN_F32, bool AMAX_ONLY, bool SHARED>
+template <int G, int FMT, bool IN_F32, bool AMAX_ONLY, bool SHARED, bool REV = false>
 int launch_pick_y(const CUtensorMap& map, const CUtensorMap& cmap, const wush::FusedParams& p, bool emit_y,
                   cudaStream_t s) {
-  if (emit_y) return launch_fused<wush::FusedCfg<G, FMT, IN_F32, AMAX_ONLY, true, SHARED>>(map, cmap, p, s);
-  return launch_fused<wush::FusedCfg<G, FMT, IN_F32, AMAX_ONLY, false, SHARED>>(map, cmap, p, s);
+  if (emit_y) return launch_fused<wush::FusedCfg<G, FMT, IN_F32, AMAX_ONLY, true, SHARED>, REV>(map, cmap, p, s);
+  return launch_fused<wush::FusedCfg<G, FMT, IN_F32, AMAX_ONLY, false, SHARED>, REV>(map, cmap, p, s);
 }
 
 // NVFP4 stages: the whole call, the amax pass alone (for a max-reduction across ranks
@@ -275,7 +278,8 @@ int dispatch(const CUtensorMap& map, const CUtensorMap& cmap, wush::FusedParams 
     if (st != WUSH_OK) return st;
   }
   p.tensor_scale = tensor_scale;
-  return launch_pick_y<16, wush::kNVFP4, IN_F32, false, SHARED>(map, cmap, p, emit_y, s);
+  // walked backwards: the quantising pass first reads what the amax pass loaded last
+  return launch_pick_y<16, wush::kNVFP4, IN_F32, false, SHARED, WUSH_NV_REVERSE>(map, cmap, p, emit_y, s);
 }
 
 // Activation batches of at most this many rows take the CUDA-core path (wush_small.cuh);

@@ -302,7 +302,10 @@ __device__ __forceinline__ T* offset_ptr(void* base, long long bytes) {
 }
 
 // ---------------------------------------------------------------- the kernel
-template <class Cfg>
+// REV: walk the tiles from the last to the first (CTA b takes the run CTA grid-1-b would
+// take, backwards).  The NVFP4 quantising pass does, so that it first reads the tiles the
+// amax pass loaded last, while they are still in L2.
+template <class Cfg, bool REV = false>
 __global__ void __launch_bounds__(Cfg::THREADS, 1)
     wush_fused_kernel(const __grid_constant__ CUtensorMap tmap_in, const __grid_constant__ CUtensorMap tmap_codes,
                       const FusedParams p) {
@@ -332,6 +335,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
   const int t_begin = bx < n_long ? bx * (run_s + 1) : n_long * (run_s + 1) + (bx - n_long) * run_s;
   const int t_end = t_begin + run_s + (bx < n_long ? 1 : 0);
   const uint64_t lim = p.wait_limit_ns;
+  auto tile_at = [&](int t) { return REV ? total - 1 - t : t; };   // tile number -> tile
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -362,13 +366,13 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
     // L2 is the point of coherence, so the loads issued after the dependency wait still
     // see everything the previous kernel wrote.
     for (int k = 0; k < p.prefetch_tiles && t_begin + k < t_end; ++k) {
-      const int t = t_begin + k;
+      const int t = tile_at(t_begin + k);
       const int ct = t / nrt, rt = t - ct * nrt;
 #pragma unroll
       for (int s = 0; s < Cfg::SUB; ++s) tma_prefetch_l2_2d(&tmap_in, ct * CH + 64 * s, rt * 128);
     }
     if (p.prefetch_tiles > 0 && t_begin < t_end) {
-      const int ct = t_begin / nrt;
+      const int ct = tile_at(t_begin) / nrt;
       const int nblk = Cfg::SHARED_T ? 1 : min(BPT, p.C - ct * BPT);
       bulk_prefetch_l2(p.T + (Cfg::SHARED_T ? 0ll : static_cast<long long>(ct) * BPT * G * G),
                        static_cast<uint32_t>(nblk * G * G * 4));
@@ -451,14 +455,15 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
   // set-up (this order and depth measured fastest: the first tile and its matrices
   // arrive ahead of the rest of the burst).  Every converter thread knows which copies
   // exist.
-  const bool t_second = !Cfg::SHARED_T && t_begin < t_end && (t_end - 1) / nrt > t_begin / nrt;
+  const int ct_first = tile_at(t_begin) / nrt;        // the run's first column tile
+  const bool t_second = !Cfg::SHARED_T && t_begin < t_end && tile_at(t_end - 1) / nrt != ct_first;
   int t_issued[2] = {t_begin < t_end ? 1 : 0, t_second ? 1 : 0};
   const uint64_t l2_pol = l2_policy_evict_first();
   int n_preloaded = 0;
   if (threadIdx.x == 0) {
     auto issue_x = [&]() {
       if (n_preloaded < STAGES && t_begin + n_preloaded < t_end) {
-        const int t = t_begin + n_preloaded;
+        const int t = tile_at(t_begin + n_preloaded);
         const int ct = t / nrt, rt = t - ct * nrt;
         const uint32_t dst = sbase + Cfg::OFF_STAGE + n_preloaded * Cfg::STAGE_BYTES;
         mbar_arrive_expect_tx(BAR(B_FULL + n_preloaded), Cfg::STAGE_BYTES);
@@ -469,8 +474,8 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
       }
     };
     issue_x();
-    if (t_begin < t_end) t_copy(t_begin / nrt, 0);
-    if (t_second) t_copy(t_begin / nrt + 1, 1);
+    if (t_begin < t_end) t_copy(ct_first, 0);
+    if (t_second) t_copy(REV ? ct_first - 1 : ct_first + 1, 1);
     while (n_preloaded < 2 && t_begin + n_preloaded < t_end) issue_x();   // the rest after the set-up
   }
   __syncwarp();
@@ -492,7 +497,8 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
       uint32_t phase = n_preloaded == STAGES ? 1u : 0u;
       for (int t = t_begin + n_preloaded; t < t_end; ++t) {
         if (!wait_bounded(BAR(B_EMPTY + stage), phase ^ 1u, abort_flag, 1u, lim)) break;
-        const int ct = t / nrt, rt = t - ct * nrt;
+        const int tt = tile_at(t);
+        const int ct = tt / nrt, rt = tt - ct * nrt;
         const uint32_t dst = sbase + Cfg::OFF_STAGE + stage * Cfg::STAGE_BYTES;
         mbar_arrive_expect_tx(BAR(B_FULL + stage), Cfg::STAGE_BYTES);
         if (Cfg::IN_F32) {
@@ -531,7 +537,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
       uint32_t full_bar = full_first;
       int epoch = -1, prev_ct = -1;
       int it = 0;
-      int ct = t_begin / nrt, rt = t_begin - (t_begin / nrt) * nrt;
+      int ct = ct_first, rt = tile_at(t_begin) - ct_first * nrt;
       uint64_t db = db_slot0;
       for (int t = t_begin; t < t_end; ++t, ++it) {
         if (Cfg::SHARED_T ? it == 0 : ct != prev_ct) {
@@ -563,8 +569,13 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
         }
         umma_commit(BAR(B_AFULL + acc));
         if (Cfg::IN_F32) umma_commit(BAR(B_OEMPTY + buf));
-        if (!Cfg::SHARED_T && (t + 1 == t_end || rt + 1 == nrt)) umma_commit(BAR(B_TEMPTY + (epoch & 1)));
-        if (++rt == nrt) rt = 0, ++ct;
+        if (!Cfg::SHARED_T && (t + 1 == t_end || (REV ? rt == 0 : rt + 1 == nrt)))
+          umma_commit(BAR(B_TEMPTY + (epoch & 1)));
+        if constexpr (REV) {
+          if (rt-- == 0) rt = nrt - 1, --ct;
+        } else {
+          if (++rt == nrt) rt = 0, ++ct;
+        }
         if (++buf == NBUF) {
           buf = 0, phase ^= 1u, da_hi = da_first, full_bar = full_first;
         } else {
@@ -593,11 +604,11 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
         mbar_arrive(BAR(B_TFULL));   // slot 0 holds the first column tile's panels
         t_landed[0] = 1;
         epoch = 0;
-        prev_ct = t_begin / nrt;
+        prev_ct = ct_first;
       }
     }
     for (int t = t_begin; conv_ok && t < t_end; ++t) {
-      const int ct = t / nrt;
+      const int ct = tile_at(t) / nrt;
       if (t_conv && (Cfg::SHARED_T ? epoch < 0 : ct != prev_ct)) {
         ++epoch;
         prev_ct = ct;
@@ -691,7 +702,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
     float run_max = 0.0f;
     int m = 0;                                  // tiles handled by this group so far
     for (int it = grp; t_begin + it < t_end; it += Cfg::N_GROUPS, ++m) {
-      const int t = t_begin + it;
+      const int t = tile_at(t_begin + it);
       const int ct = t / nrt, rt = t - ct * nrt;
       const int acc = it % NACC;
       if (live && !wait_bounded(BAR(B_AFULL + acc), static_cast<uint32_t>((it / NACC) & 1), abort_flag, 8u, lim))
