@@ -296,6 +296,56 @@ __device__ __forceinline__ float quant_int4(const float* v, uint32_t* words) {
   return s;
 }
 
+// The same INT4 quantiser, bit-identical, without a per-element float-to-integer
+// conversion (a reduced-rate instruction):
+//  * s = fl32(amax / 7) by the Markstein-corrected reciprocal product (see quant_nv_tab)
+//    with inv7 = RN(1/7), for amax >= 2^-122 where the quotient is a normal fp32; the
+//    division itself below that;
+//  * each product y * inv is clamped to [-7, 7] (equivalent to clamping after rounding,
+//    the range being symmetric and integer-bounded) and 1.5 * 2^23 is added: in
+//    [2^23, 2^24) the fp32 spacing is 1, so the sum is RNE(v) + 1.5 * 2^23 (that constant
+//    is even, so ties still go to the even integer), and the low 4 bits of the sum's
+//    encoding are RNE(v) as a two's-complement nibble;
+//  * each nibble enters its word by one bit-field insert.
+__device__ __forceinline__ uint32_t bfi4(uint32_t word, uint32_t bits, int pos) {
+  uint32_t out;
+  asm("bfi.b32 %0, %1, %2, %3, 4;" : "=r"(out) : "r"(bits), "r"(word), "r"(pos));
+  return out;
+}
+template <int NV>
+__device__ __forceinline__ float quant_int4_fast(const float* v, float inv7, uint32_t* words) {
+  const float amax = group_absmax<NV>(v);
+  float s;
+  if (amax >= 1.8807909613e-37f) {   // 2^-122
+    const float q = __fmul_rn(amax, inv7);
+    const float res = __fmaf_rn(-q, 7.0f, amax);
+    s = __fmaf_rn(res, inv7, q);
+  } else {
+    s = __fdiv_rn(amax, 7.0f);
+  }
+  float inv = s > 0.0f ? __frcp_rn(s) : 0.0f;
+  if (isinf(inv)) inv = 0.0f;
+  constexpr float kRound = 12582912.0f;   // 1.5 * 2^23
+#pragma unroll
+  for (int k = 0; k < NV / 8; ++k) {
+    float w[8];
+#pragma unroll
+    for (int e = 0; e < 8; e += 2) {
+      w[e] = v[8 * k + e];
+      w[e + 1] = v[8 * k + e + 1];
+      mul2_rn(w[e], w[e + 1], inv);
+      w[e] = fminf(fmaxf(w[e], -7.0f), 7.0f);
+      w[e + 1] = fminf(fmaxf(w[e + 1], -7.0f), 7.0f);
+      add2_rn(w[e], w[e + 1], kRound, kRound);
+    }
+    uint32_t wd = 0;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) wd = bfi4(wd, __float_as_uint(w[e]), 4 * e);
+    words[k] = wd;
+  }
+  return s;
+}
+
 template <typename T>
 __device__ __forceinline__ T* offset_ptr(void* base, long long bytes) {
   return reinterpret_cast<T*>(reinterpret_cast<uint8_t*>(base) + bytes);
@@ -680,6 +730,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
     const bool vec16 = (code_row_bytes % 16) == 0;
     using ScaleT = typename std::conditional<Cfg::FMT == kINT4, float, uint8_t>::type;
     if (!Cfg::IN_F32 && t_begin < t_end) first_split();   // with the converter warps
+    const float inv7 = __frcp_rn(7.0f);   // INT4: RN(1/7)
     float s_t = 0.0f, d6 = 0.0f, inv_d6 = 0.0f;
     bool exact_div = true;
     float* nv_tab = reinterpret_cast<float*>(smem + Cfg::OFF_NVTAB);
@@ -754,7 +805,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
             }
             if (Cfg::FMT == kMXFP4) sc[b] = static_cast<ScaleT>(quant_mx<G>(v, words[u]));
             else if (Cfg::FMT == kNVFP4) sc[b] = static_cast<ScaleT>(quant_nv_tab<G>(v, d6, inv_d6, exact_div, nv_tab, words[u]));
-            else sc[b] = static_cast<ScaleT>(quant_int4<G>(v, words[u]));
+            else sc[b] = static_cast<ScaleT>(quant_int4_fast<G>(v, inv7, words[u]));
           }
           // the load's 32 elements are one 16-byte chunk of this row's codes
           const int pc = bl ^ ((row >> SW_SHIFT) & (NCH - 1));
