@@ -460,7 +460,8 @@ def nvfp4_workspace(device=None, stream=None):
 
 
 def wush_quant_act_nvfp4_onepass(x, T, workspace, codes=None, scales=None, tensor_scale=None, stream=None):
-    """NVFP4 activations of a decode-sized batch in one launch: (codes, scales, tensor_scale).
+    """NVFP4 activations in one launch: (codes, scales, tensor_scale).  Decode-sized batches
+    on CUDA cores, larger ones on the tensor-core kernel (one cooperative launch).
     ``workspace``: from nvfp4_workspace(); zero before the first call, left zero by each."""
     lib = load_library()
     n, d = _nv_stage_input(x, T)

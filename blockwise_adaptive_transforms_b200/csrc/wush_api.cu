@@ -175,7 +175,7 @@ int encode_u8_sw128(CUtensorMap* map, const void* base, int64_t rows, int64_t co
   return r == CUDA_SUCCESS ? WUSH_OK : cuda_fail(r, "cuTensorMapEncodeTiled", __LINE__, true);
 }
 
-template <class Cfg, bool REV = false>
+template <class Cfg, bool REV = false, bool ONEPASS = false>
 int launch_fused(const CUtensorMap& map, const CUtensorMap& cmap, wush::FusedParams p, cudaStream_t stream) {
   int dev = 0, sms = 0;
   WUSH_CUDA_CHECK(cudaGetDevice(&dev));
@@ -183,7 +183,7 @@ int launch_fused(const CUtensorMap& map, const CUtensorMap& cmap, wush::FusedPar
   static std::atomic<unsigned long long> configured{0ull};   // one bit per device ordinal
   const unsigned long long bit = 1ull << (dev & 63);
   if (!(configured.load(std::memory_order_acquire) & bit)) {
-    WUSH_CUDA_CHECK(cudaFuncSetAttribute(wush::wush_fused_kernel<Cfg, REV>,
+    WUSH_CUDA_CHECK(cudaFuncSetAttribute(wush::wush_fused_kernel<Cfg, REV, ONEPASS>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES));
     configured.fetch_or(bit, std::memory_order_acq_rel);
   }
@@ -219,11 +219,16 @@ int launch_fused(const CUtensorMap& map, const CUtensorMap& cmap, wush::FusedPar
   lc.dynamicSmemBytes = Cfg::SMEM_BYTES;
   lc.stream = stream;
   cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  if (ONEPASS) {   // the CTAs wait on one another: all of them must be resident at once
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+  } else {
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+  }
   lc.attrs = attr;
-  lc.numAttrs = WUSH_USE_PDL ? 1 : 0;
-  WUSH_CUDA_CHECK(cudaLaunchKernelEx(&lc, wush::wush_fused_kernel<Cfg, REV>, map, cmap, p));
+  lc.numAttrs = (ONEPASS || WUSH_USE_PDL) ? 1 : 0;
+  WUSH_CUDA_CHECK(cudaLaunchKernelEx(&lc, wush::wush_fused_kernel<Cfg, REV, ONEPASS>, map, cmap, p));
   return launch_status(__LINE__);
 }
 
@@ -710,9 +715,51 @@ int onepass_check(const void* x_bf16, const float* T_blocks, int64_t n_tok, int6
   return WUSH_OK;
 }
 
-// The one-launch NVFP4 kernel on a checked argument set and a 16-byte aligned workspace.
+// NVFP4 in one launch of the tensor-core kernel (batches above the CUDA-core threshold):
+// one CTA per SM at most, launched cooperatively, the workspace's three words shared by
+// the CTAs (see the ONEPASS walk of wush_fused_kernel).
+int onepass_fused(const void* x_bf16, const float* T_blocks, int64_t n_tok, int64_t d_in, uint8_t* codes,
+                  uint8_t* scales, float* tensor_scale, uint32_t* workspace, wush_stream_t stream) {
+  const int ch = WUSH_ACT_TILE_CH;
+  const long long n_row_tiles = (n_tok + 127) / 128;
+  const long long n_col_tiles = (d_in + ch - 1) / ch;
+  if (n_row_tiles * n_col_tiles > INT_MAX) return WUSH_ERR_INVALID_ARG;
+  CUtensorMap map;
+  int st = encode_2d(&map, x_bf16, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, n_tok, d_in, 64, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (st != WUSH_OK) return st;
+  CUtensorMap cmap = map;
+  const bool codes_tma = ((d_in / 2) % 16) == 0;
+  if (codes_tma) {
+    st = encode_2d(&cmap, codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, n_tok, d_in / 2, ch / 2,
+                   ch == 128 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B);
+    if (st != WUSH_OK) return st;
+  }
+  wush::FusedParams p{};
+  p.codes_via_tma = codes_tma ? 1 : 0;
+  p.atom_cols = static_cast<int>((d_in / 16 + 3) / 4);
+  p.T = T_blocks;
+  p.codes = codes;
+  p.scales = scales;
+  p.amax_word = reinterpret_cast<unsigned int*>(workspace);
+  p.tensor_scale = tensor_scale;
+  p.n_rows = n_tok;
+  p.d_in = static_cast<int>(d_in);
+  p.C = static_cast<int>(d_in / 16);
+  p.n_row_tiles = static_cast<int>(n_row_tiles);
+  p.total_tiles = static_cast<int>(n_row_tiles * n_col_tiles);
+  p.wait_limit_ns = g_wait_limit_ns.load(std::memory_order_relaxed);
+  return launch_fused<wush::FusedCfg<16, wush::kNVFP4, false, false, false, false>, false, true>(
+      map, cmap, p, reinterpret_cast<cudaStream_t>(stream));
+}
+
+// The one-launch NVFP4 kernel on a checked argument set and a 16-byte aligned workspace:
+// batches above the CUDA-core threshold on the tensor-core kernel when `allow_fused`,
+// the CUDA-core kernel otherwise.
 int onepass_launch(const void* x_bf16, const float* T_blocks, int64_t n_tok, int64_t d_in, uint8_t* codes,
-                   uint8_t* scales, float* tensor_scale, uint32_t* workspace, wush_stream_t stream) {
+                   uint8_t* scales, float* tensor_scale, uint32_t* workspace, wush_stream_t stream,
+                   bool allow_fused) {
+  if (allow_fused && n_tok > small_rows_limit(WUSH_NVFP4))
+    return onepass_fused(x_bf16, T_blocks, n_tok, d_in, codes, scales, tensor_scale, workspace, stream);
   const long long C = d_in / 16;
   const long long gy = (n_tok + wush::kSmallRows - 1) / wush::kSmallRows;
   int dev = 0, sms = 0, per_sm = 0;
@@ -769,7 +816,7 @@ int wush_quant_act_nvfp4_onepass(const void* x_bf16, const float* T_blocks, int6
   if (st != WUSH_OK) return st;
   if (!workspace) return WUSH_ERR_INVALID_ARG;
   if (!aligned(workspace, 16)) return WUSH_ERR_MISALIGNED;
-  return onepass_launch(x_bf16, T_blocks, n_tok, d_in, codes, scales, tensor_scale, workspace, stream);
+  return onepass_launch(x_bf16, T_blocks, n_tok, d_in, codes, scales, tensor_scale, workspace, stream, true);
 }
 
 int wush_quant_act_nvfp4_onepass_noalloc(const void* x_bf16, const float* T_blocks, int64_t n_tok, int64_t d_in,
@@ -811,7 +858,7 @@ int wush_quant_act_nvfp4_onepass_noalloc(const void* x_bf16, const float* T_bloc
     ws = scratch[dev];
   }
   return onepass_launch(x_bf16, T_blocks, n_tok, d_in, codes, scales, tensor_scale, static_cast<uint32_t*>(ws),
-                        stream);
+                        stream, false);
 }
 
 int wush_set_gemm_cta_pairs(int enable) {

@@ -355,7 +355,13 @@ __device__ __forceinline__ T* offset_ptr(void* base, long long bytes) {
 // REV: walk the tiles from the last to the first (CTA b takes the run CTA grid-1-b would
 // take, backwards).  The NVFP4 quantising pass does, so that it first reads the tiles the
 // amax pass loaded last, while they are still in L2.
-template <class Cfg, bool REV = false>
+//
+// ONEPASS (NVFP4 only): the whole NVFP4 call in one cooperative launch.  Each CTA walks its
+// run twice, forwards for max |y| and then backwards to quantise (so that its first
+// quantised tiles are the ones it loaded last, still in L2); in between, the CTAs fold
+// their maxima into a three-word workspace (p.amax_word) and wait for one another
+// (bounded in time, error bit 128), then quantise with the common tensor scale.
+template <class Cfg, bool REV = false, bool ONEPASS = false>
 __global__ void __launch_bounds__(Cfg::THREADS, 1)
     wush_fused_kernel(const __grid_constant__ CUtensorMap tmap_in, const __grid_constant__ CUtensorMap tmap_codes,
                       const FusedParams p) {
@@ -386,6 +392,12 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
   const int t_end = t_begin + run_s + (bx < n_long ? 1 : 0);
   const uint64_t lim = p.wait_limit_ns;
   auto tile_at = [&](int t) { return REV ? total - 1 - t : t; };   // tile number -> tile
+  static_assert(!ONEPASS || (Cfg::FMT == kNVFP4 && !Cfg::AMAX_ONLY && !Cfg::IN_F32 && !Cfg::SHARED_T && !REV),
+                "the one-launch walk is an NVFP4 activation path");
+  // the walk: the CTA's run, and for ONEPASS the same run backwards after it
+  const int run_len = t_end - t_begin;
+  const int walk_len = ONEPASS ? 2 * run_len : run_len;
+  auto walk_tile = [&](int i) { return (!ONEPASS || i < run_len) ? t_begin + i : t_end - 1 - (i - run_len); };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -545,9 +557,9 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
       int n_loaded = n_preloaded;
       int stage = n_preloaded % STAGES;
       uint32_t phase = n_preloaded == STAGES ? 1u : 0u;
-      for (int t = t_begin + n_preloaded; t < t_end; ++t) {
+      for (int i = n_preloaded; i < walk_len; ++i) {
         if (!wait_bounded(BAR(B_EMPTY + stage), phase ^ 1u, abort_flag, 1u, lim)) break;
-        const int tt = tile_at(t);
+        const int tt = tile_at(walk_tile(i));
         const int ct = tt / nrt, rt = tt - ct * nrt;
         const uint32_t dst = sbase + Cfg::OFF_STAGE + stage * Cfg::STAGE_BYTES;
         mbar_arrive_expect_tx(BAR(B_FULL + stage), Cfg::STAGE_BYTES);
@@ -589,7 +601,12 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
       int it = 0;
       int ct = ct_first, rt = tile_at(t_begin) - ct_first * nrt;
       uint64_t db = db_slot0;
-      for (int t = t_begin; t < t_end; ++t, ++it) {
+      for (int t = t_begin; t < (ONEPASS ? t_begin + walk_len : t_end); ++t, ++it) {
+        if constexpr (ONEPASS) {   // coordinates from the walk (this mode is not the hot loop)
+          const int tw = walk_tile(it);
+          ct = tw / nrt;
+          rt = tw - ct * nrt;
+        }
         if (Cfg::SHARED_T ? it == 0 : ct != prev_ct) {
           ++epoch;
           prev_ct = ct;
@@ -619,8 +636,11 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
         }
         umma_commit(BAR(B_AFULL + acc));
         if (Cfg::IN_F32) umma_commit(BAR(B_OEMPTY + buf));
-        if (!Cfg::SHARED_T && (t + 1 == t_end || (REV ? rt == 0 : rt + 1 == nrt)))
+        if constexpr (ONEPASS) {   // the slot is free once the walk leaves its column tile
+          if (it + 1 == walk_len || walk_tile(it + 1) / nrt != ct) umma_commit(BAR(B_TEMPTY + (epoch & 1)));
+        } else if (!Cfg::SHARED_T && (t + 1 == t_end || (REV ? rt == 0 : rt + 1 == nrt))) {
           umma_commit(BAR(B_TEMPTY + (epoch & 1)));
+        }
         if constexpr (REV) {
           if (rt-- == 0) rt = nrt - 1, --ct;
         } else {
@@ -650,6 +670,10 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
     bool conv_ok = true;
     if (!Cfg::IN_F32 && t_begin < t_end) {
       conv_ok = first_split();
+      // the split kept the slot's read-done barrier out of it: arrive on it here so that
+      // its phases stay in step with the slot's later refills (a third column tile of the
+      // walk lands in slot 0 again and waits on that barrier's next phase)
+      mbar_arrive(BAR(B_TREAD));
       if (conv_ok) {
         mbar_arrive(BAR(B_TFULL));   // slot 0 holds the first column tile's panels
         t_landed[0] = 1;
@@ -657,8 +681,8 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
         prev_ct = ct_first;
       }
     }
-    for (int t = t_begin; conv_ok && t < t_end; ++t) {
-      const int ct = tile_at(t) / nrt;
+    for (int i = 0; conv_ok && i < walk_len; ++i) {
+      const int ct = tile_at(walk_tile(i)) / nrt;
       if (t_conv && (Cfg::SHARED_T ? epoch < 0 : ct != prev_ct)) {
         ++epoch;
         prev_ct = ct;
@@ -734,7 +758,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
     float s_t = 0.0f, d6 = 0.0f, inv_d6 = 0.0f;
     bool exact_div = true;
     float* nv_tab = reinterpret_cast<float*>(smem + Cfg::OFF_NVTAB);
-    if constexpr (Cfg::FMT == kNVFP4 && !Cfg::AMAX_ONLY) {
+    if constexpr (Cfg::FMT == kNVFP4 && !Cfg::AMAX_ONLY && !ONEPASS) {
       s_t = *p.tensor_scale;
       d6 = __fmul_rn(6.0f, s_t);
       inv_d6 = d6 > 0.0f ? __frcp_rn(d6) : 0.0f;
@@ -752,8 +776,98 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
     bool live = true;
     float run_max = 0.0f;
     int m = 0;                                  // tiles handled by this group so far
-    for (int it = grp; t_begin + it < t_end; it += Cfg::N_GROUPS, ++m) {
-      const int t = tile_at(t_begin + it);
+    int it_first = grp;
+    if constexpr (ONEPASS) {
+      // ---- first half of the walk: max |y| over this CTA's run
+      for (int it = grp; it < run_len; it += Cfg::N_GROUPS) {
+        const int t = tile_at(walk_tile(it));
+        const int ct = t / nrt, rt = t - ct * nrt;
+        const int acc = it % NACC;
+        if (live && !wait_bounded(BAR(B_AFULL + acc), static_cast<uint32_t>((it / NACC) & 1), abort_flag, 8u, lim))
+          live = false;
+        if (quad == 0 && lane == 0 && live) mbar_arrive(BAR(B_EMPTY + it % STAGES));
+        const bool warp_live = __all_sync(0xffffffffu, live) && !*abort_flag;
+        const bool row_ok = static_cast<long long>(rt) * 128 + row < p.n_rows;
+        const uint32_t tq = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(acc * Cfg::ACC_COLS);
+        if (warp_live) tc_fence_after();
+        constexpr int BPL = 32 / G;
+#pragma unroll
+        for (int bl = 0; bl < BPT / BPL; ++bl) {
+          float hl[64];
+          if (warp_live) tmem_ld64_sync(tq + static_cast<uint32_t>(bl * 64), hl);
+          if (bl == BPT / BPL - 1) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(BAR(B_AEMPTY + acc));
+          }
+          if (!warp_live) continue;
+#pragma unroll
+          for (int u = 0; u < BPL; ++u) {
+            float* v = hl + u * 2 * G;
+#pragma unroll
+            for (int jj = 0; jj < G; jj += 2) add2_rn(v[jj], v[jj + 1], v[G + jj], v[G + jj + 1]);  // hi + lo
+            if (row_ok && ct * BPT + bl * BPL + u < C) run_max = fmaxf(run_max, group_absmax<G>(v));
+          }
+        }
+      }
+      // ---- the grid's maximum: one value per CTA into the workspace, then wait for all
+      // CTAs (they are resident together: cooperative launch), bounded in time
+      float* scratch = nv_tab;                   // the table is filled only after this
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) run_max = fmaxf(run_max, __shfl_xor_sync(0xffffffffu, run_max, o));
+      if (lane == 0) scratch[warp - 4] = run_max;
+      named_bar_sync(5, 128 * Cfg::N_GROUPS);
+      if (threadIdx.x == 128) {
+        unsigned int* ws = p.amax_word;          // [0] max bits, [1] arrivals, [2] departures
+        float cm = scratch[0];
+        for (int w = 1; w < 4 * Cfg::N_GROUPS; ++w) cm = fmaxf(cm, scratch[w]);
+        const unsigned int grid = gridDim.x;
+        if (cm > 0.0f) atomicMax(&ws[0], __float_as_uint(cm));
+        __threadfence();
+        atomicAdd(&ws[1], 1u);
+        const uint64_t t0 = global_timer_ns();
+        int ok = 1;
+        while (atomicAdd(&ws[1], 0u) < grid) {
+          __nanosleep(100);
+          if (global_timer_ns() - t0 > lim) {     // a CTA never arrived
+            atomicOr(&g_wush_device_error, 128u);
+            ok = 0;
+            break;
+          }
+        }
+        __threadfence();
+        const float amax = __uint_as_float(atomicAdd(&ws[0], 0u));
+        if (ok && atomicAdd(&ws[2], 1u) == grid - 1) {   // every CTA has read the maximum
+          ws[0] = 0u;
+          ws[1] = 0u;
+          ws[2] = 0u;
+          __threadfence();
+        }
+        const float st = __fdiv_rn(amax, 2688.0f);
+        if (ok && blockIdx.x == 0) *const_cast<float*>(p.tensor_scale) = st;
+        scratch[8] = st;
+        scratch[9] = ok ? 1.0f : 0.0f;
+      }
+      named_bar_sync(5, 128 * Cfg::N_GROUPS);
+      s_t = scratch[8];
+      if (scratch[9] == 0.0f) live = false;
+      named_bar_sync(5, 128 * Cfg::N_GROUPS);   // read before the table overwrites them
+      d6 = __fmul_rn(6.0f, s_t);
+      inv_d6 = d6 > 0.0f ? __frcp_rn(d6) : 0.0f;
+      exact_div = !(inv_d6 >= 1.17549435e-38f && inv_d6 <= 3.40282347e+38f);
+      const int e_tid = threadIdx.x - 128;
+      if (e_tid < 128) {
+        const float S = __fmul_rn(e4m3_value(static_cast<uint32_t>(e_tid)), s_t);
+        float inv = S > 0.0f ? __frcp_rn(S) : 0.0f;
+        if (isinf(inv)) inv = 0.0f;
+        nv_tab[e_tid] = inv;
+      }
+      named_bar_sync(5, 128 * Cfg::N_GROUPS);   // the table is complete
+      // ---- second half of the walk: quantise, backwards
+      it_first = run_len + ((grp ^ run_len) & 1);
+    }
+    for (int it = it_first; it < walk_len; it += Cfg::N_GROUPS, ++m) {
+      const int t = tile_at(walk_tile(it));
       const int ct = t / nrt, rt = t - ct * nrt;
       const int acc = it % NACC;
       if (live && !wait_bounded(BAR(B_AFULL + acc), static_cast<uint32_t>((it / NACC) & 1), abort_flag, 8u, lim))

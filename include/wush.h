@@ -281,21 +281,29 @@ int wush_device_status(wush_stream_t stream, uint32_t* bits);
  * Applies to later calls; returns WUSH_OK. */
 int wush_set_gemm_cta_pairs(int enable);
 
-/* NVFP4 activations of a decode-sized batch in ONE launch (the staged or single-call
- * NVFP4 paths take three: amax pass, tensor scale, quantising pass).  The CTAs (one per
- * 16-channel block and 128 rows, on CUDA cores as in wush_set_small_batch_rows) fold their
- * max |y| into workspace[0], count themselves into workspace[1] and wait — bounded by the
- * wait limit, error bit 128 on expiry — until the whole grid has arrived, then quantise
- * with s_t = amax / 2688; the last CTA to leave returns the words to zero.  Outputs and
- * layouts as wush_quant_act with fmt = NVFP4, G = 16 (codes and scales bit-identical to
- * it whenever both take the CUDA-core path).
+/* NVFP4 activations in ONE launch (wush_quant_act with fmt = NVFP4 takes four: a clear of
+ * the tensor-scale word, the amax pass, the tensor-scale step and the quantising pass).
+ * The tensor scale s_t = amax|y| / 2688 needs the whole batch's maximum before any group
+ * can be quantised, so the CTAs meet once through the caller's workspace: each folds its
+ * max |y| into workspace[0], counts itself into workspace[1] and waits — bounded by the
+ * wait limit, error bit 128 on expiry — until the whole grid has arrived, then quantises
+ * with s_t; the last CTA to leave returns the words to zero.  The grid is launched
+ * cooperatively (all of it resident at once).
+ *   - Batches of at most the CUDA-core threshold (wush_set_small_batch_rows; 256 rows by
+ *     default) run on CUDA cores, one CTA per 16-channel block and 128 rows; such a grid
+ *     that cannot be resident at once returns WUSH_ERR_UNSUPPORTED (use wush_quant_act).
+ *   - Larger batches run on the tensor-core kernel, one CTA per SM: each CTA walks its
+ *     tiles forwards for max |y| and, after the meeting, backwards to quantise, so that it
+ *     first re-reads the tiles it loaded last while they are still in L2.
+ * Outputs and layouts as wush_quant_act with fmt = NVFP4, G = 16; codes, scales and
+ * tensor scale bit-identical to it whenever both take the same kind of kernel (both at
+ * most the threshold, or both above it).
  * workspace: device memory of at least 16 bytes, 16-byte aligned, ZERO before the first
  * call; every call that completes without a device error leaves it zero again.  Calls
  * that may overlap (other streams) need workspaces of their own.
- * The grid (d_in/16 x ceil(n_tok/128) CTAs) must be resident on the device at once; it is
- * launched cooperatively, and a larger batch returns WUSH_ERR_UNSUPPORTED (use
- * wush_quant_act).  Other errors as wush_quant_act; the workspace must be 16-byte aligned.
- * The pages have no counterpart: it is a latency path for small batches. */
+ * Other errors as wush_quant_act; the workspace must be 16-byte aligned.
+ * The pages have no counterpart: it is a launch-count path (the tensor scale's two passes
+ * in one launch). */
 int wush_quant_act_nvfp4_onepass(const void* x_bf16, const float* T_blocks, int64_t n_tok,
                                  int64_t d_in, uint8_t* codes, uint8_t* scales,
                                  float* tensor_scale, uint32_t* workspace, wush_stream_t stream);
@@ -316,6 +324,8 @@ int wush_quant_act_nvfp4_onepass(const void* x_bf16, const float* T_blocks, int6
  * one-launch path cannot take (a grid of d_in/16 x ceil(n_tok/128) CTAs that is not
  * resident at once) return WUSH_ERR_UNSUPPORTED; a current device ordinal above 63 also
  * returns WUSH_ERR_UNSUPPORTED; otherwise as wush_quant_act_nvfp4_onepass.
+ * It always takes the CUDA-core kernel (batches above the CUDA-core threshold included);
+ * wush_quant_act_nvfp4_onepass with a workspace also has the tensor-core one-launch path.
  * The pages have no counterpart: it only spares the caller a workspace allocation. */
 int wush_quant_act_nvfp4_onepass_noalloc(const void* x_bf16, const float* T_blocks, int64_t n_tok,
                                          int64_t d_in, uint8_t* codes, uint8_t* scales,

@@ -1,10 +1,12 @@
-"""One-launch NVFP4 for decode-sized batches (needs a B200).
+"""One-launch NVFP4 (needs a B200): decode-sized batches on CUDA cores, larger ones on the
+tensor-core kernel.
 
 The CTAs meet once through a caller's workspace to agree on the tensor scale.  Checked:
 codes, scales and tensor scale equal the staged NVFP4 call on the CUDA-core path bit for
 bit; rule 2 against the fp64 oracle; the workspace is zero again after every call (two
 calls in a row on one workspace); a grid too large to be resident at once is refused; the
-call can be captured in a CUDA graph and replayed.
+call can be captured in a CUDA graph and replayed.  Above the CUDA-core threshold the
+same checks hold against the four-launch call on the tensor-core kernel.
 """
 import numpy as np
 import pytest
@@ -88,3 +90,47 @@ def test_too_large_a_grid_is_refused():
     with pytest.raises(W.WushError) as e:
         W.wush_quant_act_nvfp4_onepass(x, T, W.nvfp4_workspace())
     assert e.value.status == 2        # WUSH_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("n_tok,d_in", [(257, 1024), (1000, 2064), (4096, 14336)])
+def test_one_launch_on_the_tensor_core_kernel_equals_the_four_launch_call(n_tok, d_in):
+    """Above the CUDA-core threshold the one-launch call runs the tensor-core kernel (amax
+    walk forwards, meeting, quantising walk backwards): bit-identical to wush_quant_act on
+    the same kernel, workspace zero afterwards, two calls in a row on one workspace."""
+    W.wush_set_small_batch_rows(-1)          # default threshold: both calls on tensor cores
+    inp, b, x, T = _data(n_tok, d_in)
+    ws = W.nvfp4_workspace()
+    for scale in (1.0, -3.0):
+        xs = x if scale == 1.0 else (x.float() * scale).to(torch.bfloat16)
+        c, s, ts = W.wush_quant_act_nvfp4_onepass(xs, T, ws)
+        c2, s2, ts2 = W.wush_quant_act(xs, T, 16, "nvfp4")
+        torch.cuda.synchronize()
+        st, bits = W.wush_device_status()
+        assert st == 0 and bits == 0, f"device error word {bits:#x}"
+        assert torch.equal(ts, ts2) and torch.equal(c, c2) and torch.equal(s, s2)
+        assert torch.count_nonzero(ws).item() == 0, ws
+    if n_tok <= 1000:   # rule 2 against the float64 path (the full-size case is held by bit-equality)
+        y_ref = O.block_transform(O.bf16_to_f64(inp.x_bits), b["T_wush32"].astype(np.float64))
+        c, s, ts = W.wush_quant_act_nvfp4_onepass(x, T, ws)
+        torch.cuda.synchronize()
+        assert_end_to_end(c.cpu().numpy(), s.cpu().numpy(), float(ts.item()), y_ref, "nvfp4", 16)
+
+
+def test_one_launch_tensor_core_graph_capture():
+    W.wush_set_small_batch_rows(-1)
+    _, _, x, T = _data(600, 4096)
+    ws = W.nvfp4_workspace()
+    out = W.wush_quant_act_nvfp4_onepass(x, T, ws)
+    torch.cuda.synchronize()
+    s = torch.cuda.Stream()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        W.wush_quant_act_nvfp4_onepass(x, T, ws, codes=out[0], scales=out[1], tensor_scale=out[2], stream=s)
+    out[0].zero_()
+    g.replay()
+    g.replay()
+    torch.cuda.synchronize()
+    e = W.wush_quant_act(x, T, 16, "nvfp4")
+    torch.cuda.synchronize()
+    assert all(torch.equal(a, b) for a, b in zip(out, e))
+    assert torch.count_nonzero(ws).item() == 0

@@ -12,7 +12,7 @@ import pytest
 import torch
 
 from oracle import wush_oracle as O
-from workloads import make_inputs, workload
+from workloads import bf16_bits_from_f64, make_inputs, workload
 import blockwise_adaptive_transforms_b200 as W
 from parity_rules import assert_bit_exact, assert_end_to_end, canon_codes
 
@@ -215,3 +215,18 @@ def test_stream_ordering_on_side_stream():
         c, sc, _ = W.wush_quant_act(x, T, 32, "mxfp4")
     s.synchronize()
     assert np.array_equal(host(c), ref[0]) and np.array_equal(host(sc), ref[1])
+
+
+def test_runs_across_several_column_tiles():
+    """128 rows by 57,344 channels: 448 tiles of one row tile each, so every CTA's run
+    crosses three or four column tiles and refills both transform slots (a slot's second
+    and later fills wait on barrier phases its first fill left behind)."""
+    n, d, G = 128, 57344, 32
+    g = np.random.default_rng(31)
+    x = dev_bf16(bf16_bits_from_f64(g.standard_normal((n, d))))
+    T = torch.from_numpy((np.eye(G, dtype=np.float32)[None] +
+                          0.05 * g.standard_normal((d // G, G, G)).astype(np.float32))).cuda()
+    c, s, _, y = W.wush_quant_act_debug(x, T, G, "mxfp4")
+    torch.cuda.synchronize()
+    assert_device_clean()
+    assert_bit_exact(host(c), host(s), None, host(y).astype(np.float64), "mxfp4", G)
