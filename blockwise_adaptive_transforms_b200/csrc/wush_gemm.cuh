@@ -56,7 +56,12 @@ struct GemmCfg {
   static constexpr int SFB_BYTES = 2 * ATOMS_PER_STAGE * 512;      // and per 128-row half
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
   static constexpr int OFF_A = 0, OFF_B = A_BYTES, OFF_SFA = A_BYTES + B_BYTES, OFF_SFB = OFF_SFA + SFA_BYTES;
-  static constexpr int OFF_BAR = STAGES * STAGE_BYTES;
+  // output staging: 128 rows x D_COLS bf16, 128-byte (MX) or 64-byte (NV: its larger scale
+  // atoms leave room for half the width) swizzle
+  static constexpr int D_COLS = NV ? 32 : 64;
+  static constexpr int OFF_D = STAGES * STAGE_BYTES;
+  static constexpr int D_BYTES = BM * D_COLS * 2;
+  static constexpr int OFF_BAR = OFF_D + D_BYTES;
   static constexpr int N_BARS = 2 * STAGES + 3;        // full[S], empty[S], afull, aempty, drain
   static constexpr int OFF_MISC = OFF_BAR + 8 * N_BARS;
   static constexpr int SMEM_BYTES = OFF_MISC + 64 + 1024;
@@ -123,7 +128,7 @@ __device__ __forceinline__ void tmem_cp_32x128b_x4(uint32_t taddr, uint64_t sdes
 template <class Cfg>
 __global__ void __launch_bounds__(Cfg::THREADS, 1)
     wush_gemm_fp4_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
-                         const GemmParams p) {
+                         const __grid_constant__ CUtensorMap tmap_d, const GemmParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_addr(smem);
@@ -151,6 +156,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
     fence_barrier_init();
     tma_prefetch_desc(&tmap_a);
     tma_prefetch_desc(&tmap_b);
+    tma_prefetch_desc(&tmap_d);
   }
   grid_dependency_wait();
   grid_launch_dependents();
@@ -245,9 +251,16 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
     }
   } else if (warp >= 4) {
     // ------------------------------------------------------------ epilogue (4 warps)
+    // Thread = row of the tile.  Each D_COLS-column slice of the accumulator goes to bf16 in
+    // a shared-memory staging buffer (swizzled as the store expects) and leaves by one TMA
+    // store;
+    // before the buffer is written again the previous store must have read it.  Every
+    // thread of the four warps reaches the same named barriers, live or not.
     const int quad = warp & 3;
     const int row_in_tile = quad * 32 + lane;
+    const bool lead = quad == 0 && lane == 0;
     const float alpha = Cfg::NV ? __fmul_rn(*p.ts_a, *p.ts_b) : 1.0f;
+    uint8_t* dstage = smem + Cfg::OFF_D;
     int it = 0;
     bool live = true;
     for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++it) {
@@ -255,28 +268,47 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
       if (live && !wait_bounded(BAR(B_AFULL), static_cast<uint32_t>(it & 1), abort_flag, 8u, lim)) live = false;
       const bool warp_live = __all_sync(0xffffffffu, live) && !*abort_flag;
       if (warp_live) tc_fence_after();
-      const long long row = static_cast<long long>(tm) * Cfg::BM + row_in_tile;
-      __nv_bfloat16* drow = p.d + row * p.N + static_cast<long long>(tn) * Cfg::BN;
+      constexpr int DC = Cfg::D_COLS;
 #pragma unroll 1
-      for (int ch = 0; ch < Cfg::BN / 32; ++ch) {
-        float v[32];
-        if (warp_live) tmem_ld32_sync(tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(32 * ch), v);
-        if (!warp_live) continue;
-        uint32_t packed[16];
+      for (int q = 0; q < Cfg::BN / DC; ++q) {
+        uint32_t packed[DC / 2];
+        if (warp_live) {
 #pragma unroll
-        for (int k = 0; k < 16; ++k) {
-          const __nv_bfloat162 b2 = Cfg::NV ? __floats2bfloat162_rn(v[2 * k] * alpha, v[2 * k + 1] * alpha)
-                                            : __floats2bfloat162_rn(v[2 * k], v[2 * k + 1]);
-          packed[k] = *reinterpret_cast<const uint32_t*>(&b2);
+          for (int h = 0; h < DC / 32; ++h) {
+            float v[32];
+            tmem_ld32_sync(tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(DC * q + 32 * h), v);
+#pragma unroll
+            for (int k = 0; k < 16; ++k) {
+              const __nv_bfloat162 b2 = Cfg::NV ? __floats2bfloat162_rn(v[2 * k] * alpha, v[2 * k + 1] * alpha)
+                                                : __floats2bfloat162_rn(v[2 * k], v[2 * k + 1]);
+              packed[16 * h + k] = *reinterpret_cast<const uint32_t*>(&b2);
+            }
+          }
         }
-        uint4* dst = reinterpret_cast<uint4*>(drow + 32 * ch);
+        if (q == Cfg::BN / DC - 1) {   // the accumulator has been read: the next tile's MMAs may go
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(BAR(B_AEMPTY));
+        }
+        if (lead) bulk_wait_read_all();   // the previous store has read the staging buffer
+        named_bar_sync(1, 128);
+        if (warp_live) {
+          constexpr int NCK = DC / 8;                       // 16-byte chunks per staged row
+          const int sw = DC == 64 ? (row_in_tile & 7) : ((row_in_tile >> 1) & 3);
 #pragma unroll
-        for (int k = 0; k < 4; ++k) dst[k] = make_uint4(packed[4 * k], packed[4 * k + 1], packed[4 * k + 2], packed[4 * k + 3]);
+          for (int c = 0; c < NCK; ++c)
+            *reinterpret_cast<uint4*>(dstage + row_in_tile * (DC * 2) + ((c ^ sw) << 4)) =
+                make_uint4(packed[4 * c], packed[4 * c + 1], packed[4 * c + 2], packed[4 * c + 3]);
+        }
+        fence_proxy_async_smem();
+        named_bar_sync(1, 128);
+        if (lead && warp_live && !*abort_flag) {
+          tma_store_2d(&tmap_d, smem_addr(dstage), tn * Cfg::BN + DC * q, tm * Cfg::BM);
+          bulk_commit_group();
+        }
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(BAR(B_AEMPTY));
     }
+    if (lead) bulk_wait_read_all();   // the last store has read the buffer before the CTA exits
   }
 
   tc_fence_before();
