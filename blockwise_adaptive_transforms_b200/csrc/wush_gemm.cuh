@@ -16,11 +16,13 @@
 // Tiles of 128 x 256 outputs, 256 K-elements (128 bytes of codes per row) per pipeline
 // stage; per stage the producer brings A (16 KB) and B (32 KB) by TMA with 128-byte
 // swizzle and the stage's scale atoms (A: 2 (MX) or 4 (NV); B: twice that, for its two
-// 128-row halves) by bulk copies; the MMA thread moves the atoms into TMEM (tcgen05.cp
-// 32x128b, broadcast to the four lane quadrants) and issues four M=128, N=256, K=64 MMAs
-// (kind::mxf4 block32, or kind::mxf4nvf4 block16); four epilogue warps read the fp32
-// accumulator (tcgen05.ld), scale by alpha, round to bf16 and store.  Persistent CTAs,
-// one per SM.
+// 128-row halves) by bulk copies; four scale warps, one per TMEM lane quadrant, write the
+// atoms into the stage's TMEM scale slot with tcgen05.st (each quadrant receives the same
+// 32 rows of 16 bytes, the layout a 32x128b.warpx4 copy would give), so that no copy sits
+// in the MMA issue queue; the MMA thread waits for them and issues four M=128, N=256, K=64
+// MMAs (kind::mxf4 block32, or kind::mxf4nvf4 block16); four epilogue warps read the fp32
+// accumulator (tcgen05.ld), scale by alpha, round to bf16 and store through shared memory
+// and TMA.  Persistent CTAs, one per SM.
 #pragma once
 #include <cstdint>
 #include <cuda_bf16.h>
@@ -62,10 +64,10 @@ struct GemmCfg {
   static constexpr int OFF_D = STAGES * STAGE_BYTES;
   static constexpr int D_BYTES = BM * D_COLS * 2;
   static constexpr int OFF_BAR = OFF_D + D_BYTES;
-  static constexpr int N_BARS = 2 * STAGES + 3;        // full[S], empty[S], afull, aempty, drain
+  static constexpr int N_BARS = 3 * STAGES + 3;        // full[S], empty[S], afull, aempty, drain, scales[S]
   static constexpr int OFF_MISC = OFF_BAR + 8 * N_BARS;
   static constexpr int SMEM_BYTES = OFF_MISC + 64 + 1024;
-  static constexpr int THREADS = 8 * 32;               // producer, MMA, 2 idle, 4 epilogue warps
+  static constexpr int THREADS = 12 * 32;  // producer, MMA, 2 idle, 4 epilogue, 4 scale warps
   // TMEM: accumulator columns [0, 256); per stage slot the scale columns from 256: A atom
   // a at +4a, B atom a of half h at +4 * ATOMS_PER_STAGE + 8a + 4h
   static constexpr int TMEM_COLS = 512;
@@ -120,10 +122,14 @@ __device__ __forceinline__ uint64_t desc_sf_atom(uint32_t saddr) {
   return d;                                                // layout type 0: no swizzle
 }
 
-// 32 lanes x 128 bits from shared memory into TMEM, repeated in all four lane quadrants.
-__device__ __forceinline__ void tmem_cp_32x128b_x4(uint32_t taddr, uint64_t sdesc) {
-  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+// Four consecutive 32-bit TMEM columns of this thread's lane (in its warp's lane
+// quadrant) from registers; tmem_wait_st waits for the thread's stores to land.
+__device__ __forceinline__ void tmem_st_x4(uint32_t taddr, uint4 v) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1, %2, %3, %4};" ::"r"(taddr), "r"(v.x), "r"(v.y),
+               "r"(v.z), "r"(v.w)
+               : "memory");
 }
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 template <class Cfg>
 __global__ void __launch_bounds__(Cfg::THREADS, 1)
@@ -135,7 +141,8 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
   const uint32_t bar0 = sbase + Cfg::OFF_BAR;
   auto BAR = [&](int i) -> uint32_t { return bar0 + 8u * static_cast<uint32_t>(i); };
   constexpr int STAGES = Cfg::STAGES;
-  const int B_FULL = 0, B_EMPTY = STAGES, B_AFULL = 2 * STAGES, B_AEMPTY = 2 * STAGES + 1, B_DRAIN = 2 * STAGES + 2;
+  const int B_FULL = 0, B_EMPTY = STAGES, B_AFULL = 2 * STAGES, B_AEMPTY = 2 * STAGES + 1, B_DRAIN = 2 * STAGES + 2,
+            B_SF = 2 * STAGES + 3;
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + Cfg::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::OFF_MISC + 4);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -148,6 +155,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(BAR(B_FULL + s), 1);
       mbar_init(BAR(B_EMPTY + s), 1);
+      mbar_init(BAR(B_SF + s), 4);
     }
     mbar_init(BAR(B_AFULL), 1);
     mbar_init(BAR(B_AEMPTY), 4);
@@ -211,19 +219,15 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
         tc_fence_after();
         bool ok = true;
         for (int ks = 0; ks < k_stages; ++ks) {
-          if (!wait_bounded(BAR(B_FULL + stage), phase, abort_flag, 2u, lim)) { ok = false; break; }
+          // the operands have landed and the scale warps have written the stage's scale slot
+          if (!wait_bounded(BAR(B_FULL + stage), phase, abort_flag, 2u, lim) ||
+              !wait_bounded(BAR(B_SF + stage), phase, abort_flag, 2u, lim)) {
+            ok = false;
+            break;
+          }
           tc_fence_after();
           const uint32_t st = sbase + stage * Cfg::STAGE_BYTES;
           const uint32_t sf_cols = tmem_base + static_cast<uint32_t>(Cfg::SF_COL0 + stage * Cfg::SF_SLOT_COLS);
-          // scale atoms -> TMEM: A atom a at columns +4a, B atom a of half h at +SFB_COL + 8a + 4h
-#pragma unroll
-          for (int a = 0; a < Cfg::ATOMS_PER_STAGE; ++a) {
-            tmem_cp_32x128b_x4(sf_cols + 4 * a, desc_sf_atom(st + Cfg::OFF_SFA + a * 512));
-#pragma unroll
-            for (int h = 0; h < 2; ++h)
-              tmem_cp_32x128b_x4(sf_cols + Cfg::SFB_COL + 8 * a + 4 * h,
-                                 desc_sf_atom(st + Cfg::OFF_SFB + h * Cfg::ATOMS_PER_STAGE * 512 + a * 512));
-          }
           const uint64_t da = desc_k_sw128(st + Cfg::OFF_A);
           const uint64_t db = desc_k_sw128(st + Cfg::OFF_B);
 #pragma unroll
@@ -249,7 +253,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
       volatile int no_abort = 0;
       wait_bounded(BAR(B_DRAIN), 0u, &no_abort, 16u, lim);
     }
-  } else if (warp >= 4) {
+  } else if (warp >= 4 && warp < 8) {
     // ------------------------------------------------------------ epilogue (4 warps)
     // Thread = row of the tile.  Each D_COLS-column slice of the accumulator goes to bf16 in
     // a shared-memory staging buffer (swizzled as the store expects) and leaves by one TMA
@@ -309,6 +313,44 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
       }
     }
     if (lead) bulk_wait_read_all();   // the last store has read the buffer before the CTA exits
+  } else if (warp >= 8) {
+    // ------------------------------------------------------------ scale warps (4)
+    // Warp 8 + q writes lane quadrant q of each stage's TMEM scale slot: A atom a at
+    // columns +4a, B atom a of half h at +SFB_COL + 8a + 4h, lane 32 q + i taking row i
+    // (16 bytes) of the atom.  The slot's previous readers (the MMAs of the stage one
+    // ring round earlier) completed before the producer refilled the stage, so the
+    // operands having landed frees the slot too.  A wait that expires reports as a
+    // converter wait (error bit 4).
+    const uint32_t lane_base = tmem_base + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+    int stage = 0;
+    uint32_t phase = 0;
+    bool live = true;
+    for (int tile = blockIdx.x; tile < n_tiles && live; tile += gridDim.x) {
+      for (int ks = 0; ks < k_stages; ++ks) {
+        const bool landed = wait_bounded(BAR(B_FULL + stage), phase, abort_flag, 4u, lim);
+        if (!__all_sync(0xffffffffu, landed) || *abort_flag) {
+          live = false;
+          break;
+        }
+        tc_fence_after();
+        const uint8_t* st = smem + stage * Cfg::STAGE_BYTES;
+        const uint32_t sf_cols = lane_base + static_cast<uint32_t>(Cfg::SF_COL0 + stage * Cfg::SF_SLOT_COLS);
+#pragma unroll
+        for (int a = 0; a < Cfg::ATOMS_PER_STAGE; ++a) {
+          tmem_st_x4(sf_cols + 4 * a, *reinterpret_cast<const uint4*>(st + Cfg::OFF_SFA + a * 512 + 16 * lane));
+#pragma unroll
+          for (int h = 0; h < 2; ++h)
+            tmem_st_x4(sf_cols + Cfg::SFB_COL + 8 * a + 4 * h,
+                       *reinterpret_cast<const uint4*>(st + Cfg::OFF_SFB + h * Cfg::ATOMS_PER_STAGE * 512 +
+                                                       a * 512 + 16 * lane));
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(BAR(B_SF + stage));
+        if (++stage == STAGES) stage = 0, phase ^= 1u;
+      }
+    }
   }
 
   tc_fence_before();
