@@ -527,6 +527,10 @@ int gemm_fp4_pair(const uint8_t* a_codes, const uint8_t* a_atoms, const float* a
   if (st != WUSH_OK) return st;
   st = encode_u8_plain(&msb, b_atoms, N * c_pad / 128, 128, 128, 4 * Cfg::ATOMS_PER_STAGE);
   if (st != WUSH_OK) return st;
+  CUtensorMap md;   // the bf16 result, stored D_COLS columns x 128 rows at a time
+  st = encode_2d(&md, d_bf16, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, N, Cfg::D_COLS,
+                 Cfg::D_COLS == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B);
+  if (st != WUSH_OK) return st;
   wush::GemmParams p{};
   p.sfa = a_atoms;
   p.sfb = b_atoms;
@@ -566,7 +570,7 @@ int gemm_fp4_pair(const uint8_t* a_codes, const uint8_t* a_atoms, const float* a
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   lc.attrs = attr;
   lc.numAttrs = WUSH_USE_PDL ? 2 : 1;
-  WUSH_CUDA_CHECK(cudaLaunchKernelEx(&lc, wush::wush_gemm_fp4_pair_kernel<Cfg>, ma, mb, msa, msb, p));
+  WUSH_CUDA_CHECK(cudaLaunchKernelEx(&lc, wush::wush_gemm_fp4_pair_kernel<Cfg>, ma, mb, msa, msb, md, p));
   return launch_status(__LINE__);
 }
 

@@ -131,6 +131,78 @@ __device__ __forceinline__ void tmem_st_x4(uint32_t taddr, uint4 v) {
 }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
+// One stage's scale atoms from shared memory into this warp's lane quadrant of the
+// stage's TMEM scale slot: A atom a at columns +4a, B atom a of half h at
+// +SFB_COL + 8a + 4h, lane i of the quadrant taking row i (16 bytes) of each atom.
+template <class Cfg>
+__device__ __forceinline__ void write_scale_slot(uint32_t slot_taddr, const uint8_t* st, int lane) {
+#pragma unroll
+  for (int a = 0; a < Cfg::ATOMS_PER_STAGE; ++a) {
+    tmem_st_x4(slot_taddr + 4 * a, *reinterpret_cast<const uint4*>(st + Cfg::OFF_SFA + a * 512 + 16 * lane));
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+      tmem_st_x4(slot_taddr + Cfg::SFB_COL + 8 * a + 4 * h,
+                 *reinterpret_cast<const uint4*>(st + Cfg::OFF_SFB + h * Cfg::ATOMS_PER_STAGE * 512 + a * 512 +
+                                                 16 * lane));
+  }
+  tmem_wait_st();
+}
+
+// Epilogue of one 128 x BN accumulator by four warps (quad = warp & 3 = TMEM lane
+// quadrant; thread = row 32 quad + lane).  Each D_COLS-column slice goes from TMEM to
+// bf16 (times alpha), into the shared-memory staging buffer in the swizzle the store's
+// tensor map names, and out by one TMA store to columns [x0 + D_COLS q, ...) of rows
+// [y0, y0 + 128), issued by the first thread once all four warps have written; the
+// buffer is rewritten only after the previous store has read it.  release() runs in
+// every warp once its last slice is in registers (the accumulator may be overwritten).
+// Every thread of the four warps reaches the same named barriers, live or not.
+template <class Cfg, class Release>
+__device__ __forceinline__ void epilogue_tile(uint32_t tmem_base, int quad, int lane, bool warp_live, float alpha,
+                                              uint8_t* dstage, const CUtensorMap* tmap_d, int x0, int y0,
+                                              volatile int* abort_flag, Release release) {
+  constexpr int DC = Cfg::D_COLS;
+  const int row_in_tile = quad * 32 + lane;
+  const bool lead = quad == 0 && lane == 0;
+#pragma unroll 1
+  for (int q = 0; q < Cfg::BN / DC; ++q) {
+    uint32_t packed[DC / 2];
+    if (warp_live) {
+#pragma unroll
+      for (int h = 0; h < DC / 32; ++h) {
+        float v[32];
+        tmem_ld32_sync(tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(DC * q + 32 * h), v);
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+          const __nv_bfloat162 b2 = Cfg::NV ? __floats2bfloat162_rn(v[2 * k] * alpha, v[2 * k + 1] * alpha)
+                                            : __floats2bfloat162_rn(v[2 * k], v[2 * k + 1]);
+          packed[16 * h + k] = *reinterpret_cast<const uint32_t*>(&b2);
+        }
+      }
+    }
+    if (q == Cfg::BN / DC - 1) {
+      tc_fence_before();
+      __syncwarp();
+      release();
+    }
+    if (lead) bulk_wait_read_all();   // the previous store has read the staging buffer
+    named_bar_sync(1, 128);
+    if (warp_live) {
+      constexpr int NCK = DC / 8;                       // 16-byte chunks per staged row
+      const int sw = DC == 64 ? (row_in_tile & 7) : ((row_in_tile >> 1) & 3);
+#pragma unroll
+      for (int c = 0; c < NCK; ++c)
+        *reinterpret_cast<uint4*>(dstage + row_in_tile * (DC * 2) + ((c ^ sw) << 4)) =
+            make_uint4(packed[4 * c], packed[4 * c + 1], packed[4 * c + 2], packed[4 * c + 3]);
+    }
+    fence_proxy_async_smem();
+    named_bar_sync(1, 128);
+    if (lead && warp_live && !*abort_flag) {
+      tma_store_2d(tmap_d, smem_addr(dstage), x0 + DC * q, y0);
+      bulk_commit_group();
+    }
+  }
+}
+
 template <class Cfg>
 __global__ void __launch_bounds__(Cfg::THREADS, 1)
     wush_gemm_fp4_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
@@ -255,16 +327,8 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
     }
   } else if (warp >= 4 && warp < 8) {
     // ------------------------------------------------------------ epilogue (4 warps)
-    // Thread = row of the tile.  Each D_COLS-column slice of the accumulator goes to bf16 in
-    // a shared-memory staging buffer (swizzled as the store expects) and leaves by one TMA
-    // store;
-    // before the buffer is written again the previous store must have read it.  Every
-    // thread of the four warps reaches the same named barriers, live or not.
     const int quad = warp & 3;
-    const int row_in_tile = quad * 32 + lane;
-    const bool lead = quad == 0 && lane == 0;
     const float alpha = Cfg::NV ? __fmul_rn(*p.ts_a, *p.ts_b) : 1.0f;
-    uint8_t* dstage = smem + Cfg::OFF_D;
     int it = 0;
     bool live = true;
     for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++it) {
@@ -272,55 +336,18 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
       if (live && !wait_bounded(BAR(B_AFULL), static_cast<uint32_t>(it & 1), abort_flag, 8u, lim)) live = false;
       const bool warp_live = __all_sync(0xffffffffu, live) && !*abort_flag;
       if (warp_live) tc_fence_after();
-      constexpr int DC = Cfg::D_COLS;
-#pragma unroll 1
-      for (int q = 0; q < Cfg::BN / DC; ++q) {
-        uint32_t packed[DC / 2];
-        if (warp_live) {
-#pragma unroll
-          for (int h = 0; h < DC / 32; ++h) {
-            float v[32];
-            tmem_ld32_sync(tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(DC * q + 32 * h), v);
-#pragma unroll
-            for (int k = 0; k < 16; ++k) {
-              const __nv_bfloat162 b2 = Cfg::NV ? __floats2bfloat162_rn(v[2 * k] * alpha, v[2 * k + 1] * alpha)
-                                                : __floats2bfloat162_rn(v[2 * k], v[2 * k + 1]);
-              packed[16 * h + k] = *reinterpret_cast<const uint32_t*>(&b2);
-            }
-          }
-        }
-        if (q == Cfg::BN / DC - 1) {   // the accumulator has been read: the next tile's MMAs may go
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(BAR(B_AEMPTY));
-        }
-        if (lead) bulk_wait_read_all();   // the previous store has read the staging buffer
-        named_bar_sync(1, 128);
-        if (warp_live) {
-          constexpr int NCK = DC / 8;                       // 16-byte chunks per staged row
-          const int sw = DC == 64 ? (row_in_tile & 7) : ((row_in_tile >> 1) & 3);
-#pragma unroll
-          for (int c = 0; c < NCK; ++c)
-            *reinterpret_cast<uint4*>(dstage + row_in_tile * (DC * 2) + ((c ^ sw) << 4)) =
-                make_uint4(packed[4 * c], packed[4 * c + 1], packed[4 * c + 2], packed[4 * c + 3]);
-        }
-        fence_proxy_async_smem();
-        named_bar_sync(1, 128);
-        if (lead && warp_live && !*abort_flag) {
-          tma_store_2d(&tmap_d, smem_addr(dstage), tn * Cfg::BN + DC * q, tm * Cfg::BM);
-          bulk_commit_group();
-        }
-      }
+      epilogue_tile<Cfg>(tmem_base, quad, lane, warp_live, alpha, smem + Cfg::OFF_D, &tmap_d, tn * Cfg::BN,
+                         tm * Cfg::BM, abort_flag, [&] {   // the next tile's MMAs may go
+                           if (lane == 0) mbar_arrive(BAR(B_AEMPTY));
+                         });
     }
-    if (lead) bulk_wait_read_all();   // the last store has read the buffer before the CTA exits
+    if (quad == 0 && lane == 0) bulk_wait_read_all();   // the last store has read the buffer
   } else if (warp >= 8) {
     // ------------------------------------------------------------ scale warps (4)
-    // Warp 8 + q writes lane quadrant q of each stage's TMEM scale slot: A atom a at
-    // columns +4a, B atom a of half h at +SFB_COL + 8a + 4h, lane 32 q + i taking row i
-    // (16 bytes) of the atom.  The slot's previous readers (the MMAs of the stage one
-    // ring round earlier) completed before the producer refilled the stage, so the
-    // operands having landed frees the slot too.  A wait that expires reports as a
-    // converter wait (error bit 4).
+    // Warp 8 + q writes lane quadrant q of each stage's TMEM scale slot.  The slot's
+    // previous readers (the MMAs of the stage one ring round earlier) completed before
+    // the producer refilled the stage, so the operands having landed frees the slot too.
+    // A wait that expires reports as a converter wait (error bit 4).
     const uint32_t lane_base = tmem_base + (static_cast<uint32_t>((warp & 3) * 32) << 16);
     int stage = 0;
     uint32_t phase = 0;
@@ -333,18 +360,8 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
           break;
         }
         tc_fence_after();
-        const uint8_t* st = smem + stage * Cfg::STAGE_BYTES;
-        const uint32_t sf_cols = lane_base + static_cast<uint32_t>(Cfg::SF_COL0 + stage * Cfg::SF_SLOT_COLS);
-#pragma unroll
-        for (int a = 0; a < Cfg::ATOMS_PER_STAGE; ++a) {
-          tmem_st_x4(sf_cols + 4 * a, *reinterpret_cast<const uint4*>(st + Cfg::OFF_SFA + a * 512 + 16 * lane));
-#pragma unroll
-          for (int h = 0; h < 2; ++h)
-            tmem_st_x4(sf_cols + Cfg::SFB_COL + 8 * a + 4 * h,
-                       *reinterpret_cast<const uint4*>(st + Cfg::OFF_SFB + h * Cfg::ATOMS_PER_STAGE * 512 +
-                                                       a * 512 + 16 * lane));
-        }
-        tmem_wait_st();
+        write_scale_slot<Cfg>(lane_base + static_cast<uint32_t>(Cfg::SF_COL0 + stage * Cfg::SF_SLOT_COLS),
+                              smem + stage * Cfg::STAGE_BYTES, lane);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(BAR(B_SF + stage));
@@ -370,9 +387,10 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
 // for the same multiply-adds, which is what bounds the one-CTA kernel (operand bytes in
 // flight per SM against L2 latency).  Both CTAs' TMA loads complete on the even CTA's
 // full barrier; only the even CTA waits on it, copies the scale atoms into both CTAs'
-// TMEM and issues the MMAs; its commits reach both CTAs' barriers; the odd CTA's
-// epilogue warps arrive on the even CTA's accumulator-empty barrier.  No load is
-// multicast.
+// TMEM (tcgen05.cp.cta_group::2: writing them with tcgen05.st from each CTA's own scale
+// warps, as the single-CTA kernel does, measured 1.8x slower here) and issues the MMAs;
+// its commits reach both CTAs' barriers; the odd CTA's epilogue warps arrive on the even
+// CTA's accumulator-empty barrier.  No load is multicast.
 template <bool NV_>
 struct GemmPairCfg {
   static constexpr bool NV = NV_;
@@ -388,7 +406,10 @@ struct GemmPairCfg {
   static constexpr int SFB_BYTES = 2 * ATOMS_PER_STAGE * 512;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
   static constexpr int OFF_A = 0, OFF_B = A_BYTES, OFF_SFA = A_BYTES + B_BYTES, OFF_SFB = OFF_SFA + SFA_BYTES;
-  static constexpr int OFF_BAR = STAGES * STAGE_BYTES;
+  static constexpr int D_COLS = NV ? 64 : 32;          // output staging width (MX: six stages leave 8 KB)
+  static constexpr int OFF_D = STAGES * STAGE_BYTES;
+  static constexpr int D_BYTES = BM * D_COLS * 2;
+  static constexpr int OFF_BAR = OFF_D + D_BYTES;
   static constexpr int N_BARS = 2 * STAGES + 3;        // full[S], empty[S], afull, aempty, drain
   static constexpr int OFF_MISC = OFF_BAR + 8 * N_BARS;
   static constexpr int SMEM_BYTES = OFF_MISC + 64 + 1024;
@@ -471,11 +492,40 @@ __device__ __forceinline__ void umma_commit_pair(uint32_t bar) {
       : "memory");
 }
 
+// wait_bounded for a barrier that threads of the other CTA of the pair arrive on: the
+// wait acquires at cluster scope, so their writes before the arrive are visible.  No
+// suspend-time hint: the waiting thread polls.
+__device__ __forceinline__ bool wait_bounded_cluster(uint32_t bar, uint32_t parity, volatile int* abort,
+                                                     uint32_t code, uint64_t limit_ns) {
+  auto try_wait = [&]() -> bool {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return done != 0;
+  };
+  const uint64_t t0 = global_timer_ns();
+  for (;;) {
+    if (try_wait()) return true;
+    if (*abort) return false;
+    if (global_timer_ns() - t0 > limit_ns) {
+      atomicOr(&g_wush_device_error, code);
+      *abort = 1;
+      return false;
+    }
+  }
+}
+
 template <class Cfg>
 __global__ void __launch_bounds__(Cfg::THREADS, 1)
     wush_gemm_fp4_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                               const __grid_constant__ CUtensorMap tmap_sfa,
-                              const __grid_constant__ CUtensorMap tmap_sfb, const GemmParams p) {
+                              const __grid_constant__ CUtensorMap tmap_sfb,
+                              const __grid_constant__ CUtensorMap tmap_d, const GemmParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_addr(smem);
@@ -508,6 +558,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
     tma_prefetch_desc(&tmap_b);
     tma_prefetch_desc(&tmap_sfa);
     tma_prefetch_desc(&tmap_sfb);
+    tma_prefetch_desc(&tmap_d);
   }
   grid_dependency_wait();
   grid_launch_dependents();
@@ -554,7 +605,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
       int stage = 0, it = 0;
       uint32_t phase = 0;
       for (int tile = pair; tile < n_tiles; tile += n_pairs, ++it) {
-        if (!wait_bounded(BAR(B_AEMPTY), static_cast<uint32_t>((it & 1) ^ 1), abort_flag, 2u, lim)) break;
+        if (!wait_bounded_cluster(BAR(B_AEMPTY), static_cast<uint32_t>((it & 1) ^ 1), abort_flag, 2u, lim)) break;
         tc_fence_after();
         bool ok = true;
         for (int ks = 0; ks < k_stages; ++ks) {
@@ -593,10 +644,9 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
       volatile int no_abort = 0;
       wait_bounded(BAR(B_DRAIN), 0u, &no_abort, 16u, lim);
     }
-  } else if (warp >= 4) {
+  } else if (warp >= 4 && warp < 8) {
     // ------------------------------------------------------------ epilogue (4 warps, both CTAs)
     const int quad = warp & 3;
-    const int row_in_tile = quad * 32 + lane;
     const float alpha = Cfg::NV ? __fmul_rn(*p.ts_a, *p.ts_b) : 1.0f;
     const uint32_t aempty_leader = mapa_shared(BAR(B_AEMPTY), 0);
     int it = 0;
@@ -606,28 +656,12 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
       if (live && !wait_bounded(BAR(B_AFULL), static_cast<uint32_t>(it & 1), abort_flag, 8u, lim)) live = false;
       const bool warp_live = __all_sync(0xffffffffu, live) && !*abort_flag;
       if (warp_live) tc_fence_after();
-      const long long row = static_cast<long long>(tm) * Cfg::PAIR_M + rank * Cfg::BM + row_in_tile;
-      __nv_bfloat16* drow = p.d + row * p.N + static_cast<long long>(tn) * Cfg::BN;
-#pragma unroll 1
-      for (int ch = 0; ch < Cfg::BN / 32; ++ch) {
-        float v[32];
-        if (warp_live) tmem_ld32_sync(tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(32 * ch), v);
-        if (!warp_live) continue;
-        uint32_t packed[16];
-#pragma unroll
-        for (int k = 0; k < 16; ++k) {
-          const __nv_bfloat162 b2 = Cfg::NV ? __floats2bfloat162_rn(v[2 * k] * alpha, v[2 * k + 1] * alpha)
-                                            : __floats2bfloat162_rn(v[2 * k], v[2 * k + 1]);
-          packed[k] = *reinterpret_cast<const uint32_t*>(&b2);
-        }
-        uint4* dst = reinterpret_cast<uint4*>(drow + 32 * ch);
-#pragma unroll
-        for (int k = 0; k < 4; ++k) dst[k] = make_uint4(packed[4 * k], packed[4 * k + 1], packed[4 * k + 2], packed[4 * k + 3]);
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(aempty_leader);
+      epilogue_tile<Cfg>(tmem_base, quad, lane, warp_live, alpha, smem + Cfg::OFF_D, &tmap_d, tn * Cfg::BN,
+                         tm * Cfg::PAIR_M + static_cast<int>(rank) * Cfg::BM, abort_flag, [&] {
+                           if (lane == 0) mbar_arrive_cluster(aempty_leader);
+                         });
     }
+    if (quad == 0 && lane == 0) bulk_wait_read_all();   // the last store has read the buffer
   }
 
   tc_fence_before();
