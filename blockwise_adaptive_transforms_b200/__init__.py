@@ -25,6 +25,7 @@ __all__ = ["FMT", "WushError", "wush_quant_act", "wush_quant_weight", "wush_quan
            "wush_quant_weight_nv_atoms", "wush_quant_act_nvfp4_amax", "wush_nvfp4_scale_from_amax",
            "wush_quant_act_nvfp4_with_scale", "wush_set_small_batch_rows", "wush_quant_act_nvfp4_onepass",
            "nvfp4_workspace", "wush_quant_act_nvfp4_onepass_noalloc", "wush_set_gemm_cta_pairs",
+           "wush_quant_act_nv_atoms_onepass",
            "wush_last_error_detail"]
 
 FMT = {"mxfp4": 0, "nvfp4": 1, "int4": 2}
@@ -38,6 +39,7 @@ EXPORTED_SYMBOLS = ("wush_quant_act", "wush_quant_weight", "wush_quant_act_debug
                     "wush_quant_act_nvfp4_amax", "wush_nvfp4_scale_from_amax", "wush_quant_act_nvfp4_with_scale",
                     "wush_set_small_batch_rows", "wush_quant_act_nvfp4_onepass",
                     "wush_quant_act_nvfp4_onepass_noalloc", "wush_set_gemm_cta_pairs",
+                    "wush_quant_act_nv_atoms_onepass",
                     "wush_build_transforms", "wush_hadamard", "wush_device_status",
                     "wush_set_wait_limit_ns",
                     "wush_selftest_wait_timeout", "wush_status_string", "wush_last_error_detail",
@@ -110,6 +112,8 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
     lib.wush_device_status.restype = ctypes.c_int
     lib.wush_quant_act_nvfp4_onepass.argtypes = [_P, _P, _I64, _I64, _P, _P, _P, _P, _P]
     lib.wush_quant_act_nvfp4_onepass.restype = ctypes.c_int
+    lib.wush_quant_act_nv_atoms_onepass.argtypes = [_P, _P, _I64, _I64, _P, _P, _P, _P, _P]
+    lib.wush_quant_act_nv_atoms_onepass.restype = ctypes.c_int
     lib.wush_quant_act_nvfp4_onepass_noalloc.argtypes = [_P, _P, _I64, _I64, _P, _P, _P, _P]
     lib.wush_quant_act_nvfp4_onepass_noalloc.restype = ctypes.c_int
     lib.wush_set_gemm_cta_pairs.argtypes = [_I32]
@@ -484,6 +488,32 @@ def wush_quant_act_nvfp4_onepass(x, T, workspace, codes=None, scales=None, tenso
     if st != 0:
         raise WushError(st, "wush_quant_act_nvfp4_onepass")
     return codes, scales, tensor_scale
+
+
+def wush_quant_act_nv_atoms_onepass(x, T, workspace, codes=None, atoms=None, tensor_scale=None, stream=None):
+    """NVFP4 activations in one launch of the tensor-core kernel with the E4M3 scales in the
+    scale-atom layout: (codes, atoms, tensor_scale).  ``workspace``: from nvfp4_workspace()."""
+    lib = load_library()
+    n, d = _nv_stage_input(x, T)
+    _check_dev(workspace, "workspace", torch.int32)
+    s = _launch_stream(stream, x.device)
+    if codes is None:
+        codes = _empty((n, d // 2), torch.uint8, s)
+    if atoms is None:
+        atoms = _empty(atom_bytes(n, d // 16), torch.uint8, s, zero=True)
+    if tensor_scale is None:
+        tensor_scale = _empty(1, torch.float32, s)
+    for t, name, dt in ((codes, "codes", torch.uint8), (atoms, "scale atoms", torch.uint8),
+                        (tensor_scale, "tensor_scale", torch.float32)):
+        _check_dev(t, name, dt)
+    if tuple(codes.shape) != (n, d // 2) or atoms.numel() < atom_bytes(n, d // 16) or workspace.numel() < 4:
+        raise ValueError("output or workspace buffers have the wrong size")
+    with torch.cuda.device(x.device):
+        st = lib.wush_quant_act_nv_atoms_onepass(_ptr(x), _ptr(T), n, d, _ptr(codes), _ptr(atoms), _ptr(tensor_scale),
+                                                 _ptr(workspace), s.cuda_stream)
+    if st != 0:
+        raise WushError(st, "wush_quant_act_nv_atoms_onepass")
+    return codes, atoms, tensor_scale
 
 
 def wush_quant_act_nvfp4_onepass_noalloc(x, T, codes=None, scales=None, tensor_scale=None, stream=None):

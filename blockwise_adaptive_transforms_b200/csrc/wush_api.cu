@@ -725,9 +725,11 @@ int onepass_check(const void* x_bf16, const float* T_blocks, int64_t n_tok, int6
 
 // NVFP4 in one launch of the tensor-core kernel (batches above the CUDA-core threshold):
 // one CTA per SM at most, launched cooperatively, the workspace's three words shared by
-// the CTAs (see the ONEPASS walk of wush_fused_kernel).
+// the CTAs (see the ONEPASS walk of wush_fused_kernel).  scale_atoms: the scales go to
+// the block-scaled MMA's scale-atom layout instead of row-major [rows][C].
 int onepass_fused(const void* x_bf16, const float* T_blocks, int64_t n_tok, int64_t d_in, uint8_t* codes,
-                  uint8_t* scales, float* tensor_scale, uint32_t* workspace, wush_stream_t stream) {
+                  uint8_t* scales, float* tensor_scale, uint32_t* workspace, wush_stream_t stream,
+                  bool scale_atoms = false) {
   const int ch = WUSH_ACT_TILE_CH;
   const long long n_row_tiles = (n_tok + 127) / 128;
   const long long n_col_tiles = (d_in + ch - 1) / ch;
@@ -744,6 +746,7 @@ int onepass_fused(const void* x_bf16, const float* T_blocks, int64_t n_tok, int6
   }
   wush::FusedParams p{};
   p.codes_via_tma = codes_tma ? 1 : 0;
+  p.scale_atoms = scale_atoms ? 1 : 0;
   p.atom_cols = static_cast<int>((d_in / 16 + 3) / 4);
   p.T = T_blocks;
   p.codes = codes;
@@ -825,6 +828,17 @@ int wush_quant_act_nvfp4_onepass(const void* x_bf16, const float* T_blocks, int6
   if (!workspace) return WUSH_ERR_INVALID_ARG;
   if (!aligned(workspace, 16)) return WUSH_ERR_MISALIGNED;
   return onepass_launch(x_bf16, T_blocks, n_tok, d_in, codes, scales, tensor_scale, workspace, stream, true);
+}
+
+int wush_quant_act_nv_atoms_onepass(const void* x_bf16, const float* T_blocks, int64_t n_tok, int64_t d_in,
+                                    uint8_t* codes, uint8_t* scale_atoms, float* tensor_scale, uint32_t* workspace,
+                                    wush_stream_t stream) {
+  const int st = onepass_check(x_bf16, T_blocks, n_tok, d_in, codes, scale_atoms, tensor_scale);
+  if (st == kSkipLaunch) return WUSH_OK;
+  if (st != WUSH_OK) return st;
+  if (!workspace) return WUSH_ERR_INVALID_ARG;
+  if (!aligned(workspace, 16) || !aligned(scale_atoms, 16)) return WUSH_ERR_MISALIGNED;
+  return onepass_fused(x_bf16, T_blocks, n_tok, d_in, codes, scale_atoms, tensor_scale, workspace, stream, true);
 }
 
 int wush_quant_act_nvfp4_onepass_noalloc(const void* x_bf16, const float* T_blocks, int64_t n_tok, int64_t d_in,

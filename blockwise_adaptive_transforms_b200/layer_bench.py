@@ -8,8 +8,9 @@ for a square, a wide and a deep projection of each model) on one B200:
   none   the MXFP4 GEMM alone, operands already quantised (the upper bound),
   H      shared-Hadamard transform + quantisation of X, then the MXFP4 GEMM,
   WUSH   per-block WUSH transform + quantisation of X, then the MXFP4 GEMM;
-  nv_none / nv_WUSH   the same two for NVFP4 (G = 16 transforms, two-pass tensor scale,
-         the NVFP4 GEMM).
+  nv_none / nv_WUSH   the same two for NVFP4 (G = 16 transforms, two-pass tensor scale
+         in one cooperative launch, the NVFP4 GEMM); nv_WUSH_4launch the same layer with
+         the activation quantiser's four launches.
 
 Weights are quantised once beforehand (offline, as on the pages).  Every variant is
 timed as a CUDA graph of repeated calls with events on its stream.
@@ -25,8 +26,9 @@ import sys
 
 import torch
 
-from . import (wush_hadamard, wush_gemm_mxfp4, wush_gemm_nvfp4, wush_quant_act_mx_atoms, wush_quant_act_nv_atoms,
-               wush_quant_act_shared_mx_atoms, wush_quant_weight_mx_atoms, wush_quant_weight_nv_atoms)
+from . import (nvfp4_workspace, wush_hadamard, wush_gemm_mxfp4, wush_gemm_nvfp4, wush_quant_act_mx_atoms,
+               wush_quant_act_nv_atoms, wush_quant_act_nv_atoms_onepass, wush_quant_act_shared_mx_atoms,
+               wush_quant_weight_mx_atoms, wush_quant_weight_nv_atoms)
 
 # (N, K) per projection kind.  The Qwen3-8B shapes are the pages' own; the other two rows
 # are the same three kinds for a 14B-class (hidden 5120, MLP 17408) and a 70B-class
@@ -76,6 +78,7 @@ def bench_shape(M: int, N: int, K: int, device="cuda", seed=0) -> dict:
     Tn = (torch.eye(16) + 0.1 * torch.randn(K // 16, 16, 16, generator=gen)).to(device)
     cwn, awn, twn = wush_quant_weight_nv_atoms(w, Tn)     # offline
     cxn, axn, txn = wush_quant_act_nv_atoms(x, Tn)
+    ws = nvfp4_workspace(device=device)
     out = torch.empty((M, N), dtype=torch.bfloat16, device=device)
     out_ref = torch.empty((M, N), dtype=torch.bfloat16, device=device)
     s = torch.cuda.Stream(device=device)
@@ -97,15 +100,21 @@ def bench_shape(M: int, N: int, K: int, device="cuda", seed=0) -> dict:
     def nv_none():
         wush_gemm_nvfp4(cxn, axn, txn, cwn, awn, twn, out=out, stream=s)
 
-    def nv_wush():
+    def nv_wush():   # the two-pass quantiser in one launch
+        wush_quant_act_nv_atoms_onepass(x, Tn, ws, codes=cxn, atoms=axn, tensor_scale=txn, stream=s)
+        wush_gemm_nvfp4(cxn, axn, txn, cwn, awn, twn, out=out, stream=s)
+
+    def nv_wush4():   # the same in four launches
         wush_quant_act_nv_atoms(x, Tn, codes=cxn, atoms=axn, tensor_scale=txn, stream=s)
         wush_gemm_nvfp4(cxn, axn, txn, cwn, awn, twn, out=out, stream=s)
 
     t = {name: _time_graph(fn, s) for name, fn in (("bf16", bf16), ("none", none), ("H", h_quant), ("WUSH", wush),
-                                                   ("nv_none", nv_none), ("nv_WUSH", nv_wush))}
+                                                   ("nv_none", nv_none), ("nv_WUSH", nv_wush),
+                                                   ("nv_WUSH_4launch", nv_wush4))}
     flops = 2.0 * M * N * K
     return {"M": M, "N": N, "K": K, "us": {k: round(v, 2) for k, v in t.items()},
-            "speedup_vs_bf16": {k: round(t["bf16"] / t[k], 3) for k in ("none", "H", "WUSH", "nv_none", "nv_WUSH")},
+            "speedup_vs_bf16": {k: round(t["bf16"] / t[k], 3)
+                                for k in ("none", "H", "WUSH", "nv_none", "nv_WUSH", "nv_WUSH_4launch")},
             "fp4_gemm_tflops": round(flops / t["none"] / 1e6, 1), "bf16_tflops": round(flops / t["bf16"] / 1e6, 1)}
 
 
@@ -124,7 +133,8 @@ def main(argv=None) -> int:
             print(f"{key:10s} M={a.M} N={N:6d} K={K:6d}  bf16 {r['us']['bf16']:8.1f} us  fp4 gemm {r['us']['none']:8.1f} us"
                   f" ({r['fp4_gemm_tflops']:7.1f} TFLOP/s)  H {r['us']['H']:8.1f}  WUSH {r['us']['WUSH']:8.1f}   "
                   f"speedup none/H/WUSH {r['speedup_vs_bf16']['none']:.2f}/{r['speedup_vs_bf16']['H']:.2f}/"
-                  f"{r['speedup_vs_bf16']['WUSH']:.2f}   nvfp4 none/WUSH {r['us']['nv_none']:8.1f}/{r['us']['nv_WUSH']:8.1f} us",
+                  f"{r['speedup_vs_bf16']['WUSH']:.2f}   nvfp4 none/WUSH {r['us']['nv_none']:8.1f}/{r['us']['nv_WUSH']:8.1f} us"
+                  f" (4 launches {r['us']['nv_WUSH_4launch']:8.1f})",
                   flush=True)
     if a.json:
         with open(a.json, "w") as f:

@@ -308,6 +308,20 @@ int wush_quant_act_nvfp4_onepass(const void* x_bf16, const float* T_blocks, int6
                                  int64_t d_in, uint8_t* codes, uint8_t* scales,
                                  float* tensor_scale, uint32_t* workspace, wush_stream_t stream);
 
+/* As wush_quant_act_nvfp4_onepass, with the E4M3 scales written in the scale-atom layout
+ * wush_gemm_nvfp4 reads (as wush_quant_act_nv_atoms): the activation side of an NVFP4
+ * layer in one launch.  Every batch, decode-sized ones included, runs on the tensor-core
+ * kernel (one cooperative launch, one CTA per SM at most).  Codes, scale atoms and tensor
+ * scale are bit-identical to wush_quant_act_nv_atoms whenever that call takes the
+ * tensor-core kernel too (batches above the CUDA-core threshold).  scale_atoms (device,
+ * 16-byte aligned) must hold atom_bytes = rows_pad * C_pad bytes (C = d_in / 16); bytes of
+ * padding rows and columns are not written.  workspace: as wush_quant_act_nvfp4_onepass
+ * (16 bytes, 16-byte aligned, zero before the first call and left zero by each; one per
+ * stream whose calls may overlap).  Errors as wush_quant_act_nvfp4_onepass. */
+int wush_quant_act_nv_atoms_onepass(const void* x_bf16, const float* T_blocks, int64_t n_tok,
+                                    int64_t d_in, uint8_t* codes, uint8_t* scale_atoms,
+                                    float* tensor_scale, uint32_t* workspace, wush_stream_t stream);
+
 /* The one-launch NVFP4 path without a caller workspace: it uses a 256-byte file-scope
  * static device array of the library (3 words of it), whose address is taken once per
  * device with cudaGetSymbolAddress; nothing is allocated.  The scratch is zero when the

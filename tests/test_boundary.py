@@ -208,3 +208,9 @@ def test_noalloc_checks_arguments_before_any_cuda_call(lib):
     g = lib.wush_quant_act_nvfp4_onepass
     assert g(A16, A16, 8, 64, A16, A16, A4, None, None) == INVALID    # workspace required
     assert g(A16, A16, 8, 64, A16, A16, A4, A4, None) == MISALIGNED
+    h = lib.wush_quant_act_nv_atoms_onepass
+    assert h(A16, A16, 8, 64, A16, A16, A4, None, None) == INVALID    # workspace required
+    assert h(A16, A16, 8, 64, A16, A16, A4, A4, None) == MISALIGNED   # workspace alignment
+    assert h(A16, A16, 8, 64, A16, A4, A4, A16, None) == MISALIGNED   # scale atoms alignment
+    assert h(A16, A16, 8, 40, A16, A16, A4, A16, None) == INVALID     # d_in % 16
+    assert h(A16, A16, 0, 64, None, None, None, None, None) == OK     # empty batch

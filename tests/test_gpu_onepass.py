@@ -6,7 +6,9 @@ codes, scales and tensor scale equal the staged NVFP4 call on the CUDA-core path
 bit; rule 2 against the fp64 oracle; the workspace is zero again after every call (two
 calls in a row on one workspace); a grid too large to be resident at once is refused; the
 call can be captured in a CUDA graph and replayed.  Above the CUDA-core threshold the
-same checks hold against the four-launch call on the tensor-core kernel.
+same checks hold against the four-launch call on the tensor-core kernel, and the variant
+that writes the scales in the FP4 GEMM's scale-atom layout equals the four-launch atoms
+call.
 """
 import numpy as np
 import pytest
@@ -134,3 +136,21 @@ def test_one_launch_tensor_core_graph_capture():
     torch.cuda.synchronize()
     assert all(torch.equal(a, b) for a, b in zip(out, e))
     assert torch.count_nonzero(ws).item() == 0
+
+
+@pytest.mark.parametrize("n_tok,d_in,threshold", [(1024, 4096, -1), (300, 416, -1), (130, 1024, 0)])
+def test_one_launch_scale_atoms_equal_the_four_launch_atoms_call(n_tok, d_in, threshold):
+    """wush_quant_act_nv_atoms_onepass (always the tensor-core kernel) against
+    wush_quant_act_nv_atoms on the same kernel (threshold 0 sends small batches there too):
+    codes, scale atoms (padding included) and tensor scale bit-identical; workspace zero."""
+    W.wush_set_small_batch_rows(threshold)
+    _, _, x, T = _data(n_tok, d_in)
+    ws = W.nvfp4_workspace()
+    for _ in range(2):
+        c, a, ts = W.wush_quant_act_nv_atoms_onepass(x, T, ws)
+        c2, a2, ts2 = W.wush_quant_act_nv_atoms(x, T)
+        torch.cuda.synchronize()
+        st, bits = W.wush_device_status()
+        assert st == 0 and bits == 0, f"device error word {bits:#x}"
+        assert torch.equal(ts, ts2) and torch.equal(c, c2) and torch.equal(a, a2)
+        assert torch.count_nonzero(ws).item() == 0, ws
