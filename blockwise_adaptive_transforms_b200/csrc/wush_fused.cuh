@@ -827,7 +827,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
         atomicAdd(&ws[1], 1u);
         const uint64_t t0 = global_timer_ns();
         int ok = 1;
-        while (atomicAdd(&ws[1], 0u) < grid) {
+        while (ld_acquire_gpu(&ws[1]) < grid) {
           __nanosleep(100);
           if (global_timer_ns() - t0 > lim) {     // a CTA never arrived
             atomicOr(&g_wush_device_error, 128u);

@@ -138,7 +138,7 @@ __global__ void __launch_bounds__(kSmallRows)
     atomicAdd(&ws[1], 1u);
     const uint64_t t0 = global_timer_ns();
     int ok = 1;
-    while (atomicAdd(&ws[1], 0u) < total) {
+    while (ld_acquire_gpu(&ws[1]) < total) {
       __nanosleep(64);
       if (global_timer_ns() - t0 > p.wait_limit_ns) {   // a CTA never arrived
         atomicOr(&g_wush_device_error, 128u);
