@@ -777,6 +777,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
     float run_max = 0.0f;
     int m = 0;                                  // tiles handled by this group so far
     int it_first = grp;
+    bool met = false;                           // ONEPASS, thread 128: the grid has met
     if constexpr (ONEPASS) {
       // ---- first half of the walk: max |y| over this CTA's run
       for (int it = grp; it < run_len; it += Cfg::N_GROUPS) {
@@ -823,8 +824,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
         for (int w = 1; w < 4 * Cfg::N_GROUPS; ++w) cm = fmaxf(cm, scratch[w]);
         const unsigned int grid = gridDim.x;
         if (cm > 0.0f) atomicMax(&ws[0], __float_as_uint(cm));
-        __threadfence();
-        atomicAdd(&ws[1], 1u);
+        red_add_release_gpu(&ws[1]);             // the maximum above is ordered before the count
         const uint64_t t0 = global_timer_ns();
         int ok = 1;
         while (ld_acquire_gpu(&ws[1]) < grid) {
@@ -835,14 +835,10 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
             break;
           }
         }
-        __threadfence();
-        const float amax = __uint_as_float(atomicAdd(&ws[0], 0u));
-        if (ok && atomicAdd(&ws[2], 1u) == grid - 1) {   // every CTA has read the maximum
-          ws[0] = 0u;
-          ws[1] = 0u;
-          ws[2] = 0u;
-          __threadfence();
-        }
+        // the acquire poll above ordered this read after every CTA's maximum; a load, not an
+        // atomic: the whole grid reads the word at once here
+        const float amax = __uint_as_float(ld_acquire_gpu(&ws[0]));
+        met = ok != 0;
         const float st = __fdiv_rn(amax, 2688.0f);
         if (ok && blockIdx.x == 0) *const_cast<float*>(p.tensor_scale) = st;
         scratch[8] = st;
@@ -1028,6 +1024,20 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
     // the last stores must have read their staging buffers before the CTA's shared
     // memory goes away; their global writes complete with the grid
     if (store_leader && p.codes_via_tma) bulk_wait_read_all();
+    if constexpr (ONEPASS) {
+      // this CTA read the maximum long ago; the last one to leave puts the workspace back
+      // to zero.  Counting departures here rather than right after the meeting spreads the
+      // grid's atomics on ws[2] over the CTAs' different finishing times.
+      if (threadIdx.x == 128 && met) {
+        unsigned int* ws = p.amax_word;
+        if (atomicAdd(&ws[2], 1u) == gridDim.x - 1) {
+          ws[0] = 0u;
+          ws[1] = 0u;
+          ws[2] = 0u;
+          __threadfence();
+        }
+      }
+    }
   }
 
   // Every warp reconverges before the CTA-wide barrier: the producer and MMA roles ran on

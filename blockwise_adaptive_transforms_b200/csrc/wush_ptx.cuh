@@ -35,6 +35,12 @@ __device__ __forceinline__ unsigned int ld_acquire_gpu(const unsigned int* p) {
   return v;
 }
 
+// Atomic add of 1 with release semantics at GPU scope: this thread's earlier writes and
+// atomics (the maximum folded in just before) are visible to whoever acquires the count.
+__device__ __forceinline__ void red_add_release_gpu(unsigned int* p) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(p) : "memory");
+}
+
 // ---------------------------------------------------------------- mbarrier
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");

@@ -134,8 +134,7 @@ __global__ void __launch_bounds__(kSmallRows)
     for (int w = 1; w < kSmallRows / 32; ++w) cm = fmaxf(cm, warp_max[w]);
     const unsigned int total = gridDim.x * gridDim.y;
     if (cm > 0.0f) atomicMax(&ws[0], __float_as_uint(cm));
-    __threadfence();
-    atomicAdd(&ws[1], 1u);
+    red_add_release_gpu(&ws[1]);                // the maximum above is ordered before the count
     const uint64_t t0 = global_timer_ns();
     int ok = 1;
     while (ld_acquire_gpu(&ws[1]) < total) {
@@ -146,8 +145,7 @@ __global__ void __launch_bounds__(kSmallRows)
         break;
       }
     }
-    __threadfence();
-    s_amax = __uint_as_float(atomicAdd(&ws[0], 0u));
+    s_amax = __uint_as_float(ld_acquire_gpu(&ws[0]));   // ordered after the poll's acquire
     s_ok = ok;
     if (ok && atomicAdd(&ws[2], 1u) == total - 1) {     // every CTA has read the maximum
       ws[0] = 0u;
