@@ -364,9 +364,17 @@ def config_rows(dev, peak_gbs: float) -> dict:
                       stream, 20)
     n, d, C = wl.n_tok, wl.d_in, wl.d_in // wl.G
     one_read = n * d * 2 + n * d // 2 + n * C + C * wl.G * wl.G * 4 + 4
-    row("nvfp4_4096x14336", sec, one_read, "bytes count X once; the two passes move "
-        f"{one_read + n * d * 2 + C * wl.G * wl.G * 4} B", moved_GB_s=round((one_read + n * d * 2 + C * wl.G * wl.G * 4) / sec / 1e9, 1))
-    del xs, outs, inp
+    moved = one_read + n * d * 2 + C * wl.G * wl.G * 4
+    row("nvfp4_4096x14336", sec, one_read, f"four launches; bytes count X once; the two passes move {moved} B",
+        moved_GB_s=round(moved / sec / 1e9, 1))
+    # the same call in one cooperative launch (caller workspace): bit-identical outputs
+    ws = W.nvfp4_workspace(device=dev, stream=stream)
+    sec = _time_calls(lambda i: W.wush_quant_act_nvfp4_onepass(xs[i % 2], T, ws, codes=outs[i % 2][0],
+                                                               scales=outs[i % 2][1], tensor_scale=outs[i % 2][2],
+                                                               stream=stream), stream, 20)
+    row("nvfp4_4096x14336_one_launch", sec, one_read, "wush_quant_act_nvfp4_onepass; bytes count X once",
+        moved_GB_s=round(moved / sec / 1e9, 1))
+    del xs, outs, inp, ws
 
     # 70B-like large batch: activations 16384 x 8192 and weights 8192 x 8192, MXFP4
     wl = workload("large_mxfp4_8192")
