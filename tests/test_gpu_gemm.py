@@ -266,3 +266,31 @@ def test_cta_pair_kernel_equals_the_oracle_and_the_single_cta_kernel(M, N, K, nv
             assert_gemm_nv_close(d.float().cpu().numpy(), a_c, a_s, 0.5, b_c, b_s, 1.25, K)
         else:
             assert_gemm_close(d.float().cpu().numpy(), a_c, a_s, b_c, b_s, K)
+
+
+@pytest.mark.parametrize("nv", [False, True])
+def test_persistent_ctas_running_several_tiles(nv):
+    """2048 x 5120 x 512: 320 output tiles on at most 148 CTAs, so each CTA runs two or
+    three tiles and every ring (operand stages, TMEM scale slots, the accumulator and the
+    output staging buffer) wraps across tiles; every element within the oracle bound."""
+    M, N, K = 2048, 5120, 512
+    if nv:
+        a_c, a_s = random_nv_operand(M, K, 7)
+        b_c, b_s = random_nv_operand(N, K, 8)
+        a_t, b_t = float(np.float32(0.61)), float(np.float32(1.3))
+        ta = torch.tensor([a_t], dtype=torch.float32, device="cuda")
+        tb = torch.tensor([b_t], dtype=torch.float32, device="cuda")
+        d = W.wush_gemm_nvfp4(dev(a_c), W.wush_mx_scales_to_atoms(dev(a_s)), ta, dev(b_c),
+                              W.wush_mx_scales_to_atoms(dev(b_s)), tb)
+    else:
+        a_c, a_s = random_operand(M, K, 7)
+        b_c, b_s = random_operand(N, K, 8)
+        d = W.wush_gemm_mxfp4(dev(a_c), W.wush_mx_scales_to_atoms(dev(a_s)), dev(b_c),
+                              W.wush_mx_scales_to_atoms(dev(b_s)))
+    torch.cuda.synchronize()
+    st, bits = W.wush_device_status()
+    assert st == 0 and bits == 0, f"device error word {bits:#x}"
+    if nv:
+        assert_gemm_nv_close(d.float().cpu().numpy(), a_c, a_s, a_t, b_c, b_s, b_t, K)
+    else:
+        assert_gemm_close(d.float().cpu().numpy(), a_c, a_s, b_c, b_s, K)
