@@ -183,6 +183,14 @@ def test_binding_rejects_host_tensors_before_any_cuda_call():
         W.nvfp4_workspace("cpu")
     with pytest.raises(TypeError):
         W._launch_stream(None, torch.device("cpu"))
+    x16 = torch.zeros((4, 32), dtype=torch.bfloat16)
+    T16 = torch.zeros((2, 16, 16), dtype=torch.float32)
+    ws = torch.zeros(4, dtype=torch.int32)
+    for call in (lambda: W.wush_quant_act_nvfp4_onepass(x16, T16, ws),
+                 lambda: W.wush_quant_act_nv_atoms_onepass(x16, T16, ws),
+                 lambda: W.wush_quant_act_nvfp4_onepass_noalloc(x16, T16)):
+        with pytest.raises(TypeError):
+            call()
 
 
 def test_hadamard_argument_checks(lib):
